@@ -1,0 +1,378 @@
+// moe_api.cu -- the extern "C" entry points of libmoe.so (declared in include/moe.h).
+//
+// Host side only: argument validation (every error is returned before anything is enqueued),
+// the workspace layout, and the choice of kernels.  All arithmetic of the layer runs in the
+// kernels of k_route.cu, k_ffn.cu and k_gemm_tc.cu.
+#include <algorithm>
+#include <atomic>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <new>
+#include <vector>
+
+#include "moe_internal.cuh"
+
+struct moe_arena {
+    const uint8_t *base;
+    size_t bytes;
+    int H, F, E, shared;      // shared: index of the shared expert (== E) or -1
+    int n;                    // descriptors (E or E + 1)
+    int fmt_mask;             // bit f set when some expert uses format f
+    moe::ExpertDev *d_experts;
+    std::vector<moe_expert_desc> descs;
+};
+
+namespace moe {
+
+static std::atomic<unsigned long long> g_kernels{0};
+
+void note_launches(int n) { g_kernels.fetch_add((unsigned long long)n, std::memory_order_relaxed); }
+
+cudaError_t ensure_smem_impl(const void *kernel, size_t bytes) {
+    static std::mutex mu;
+    static std::map<std::pair<int, const void *>, size_t> done;
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return err;
+    std::lock_guard<std::mutex> lock(mu);
+    size_t &have = done[{dev, kernel}];
+    if (bytes <= have) return cudaSuccess;
+    err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (err == cudaSuccess) have = bytes;
+    return err;
+}
+
+static size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+static bool aligned(const void *p, size_t a) { return ((uintptr_t)p & (a - 1)) == 0; }
+
+WsLayout ws_layout(const moe_arena *A, int T, int k, uint32_t flags) {
+    WsLayout L{};
+    size_t p = 0;
+    auto take = [&](size_t bytes) {
+        const size_t o = p;
+        p = align256(p + bytes);
+        return o;
+    };
+    const int H = A->H, F = A->F, E = A->E;
+    const int shared = A->shared >= 0 ? 1 : 0;
+    L.slots = T * k + T;
+    L.hpad = ((F + 255) / 256) * 256;
+    L.max_jobs = std::min(E, T * k) + shared;
+    L.n_chunks = (T + kChunk - 1) / kChunk;
+    L.status = take(sizeof(uint32_t));
+    L.njobs = take(sizeof(int32_t));
+    L.jobs = take(sizeof(Job) * (size_t)L.max_jobs);
+    L.xq = take((size_t)T * H);
+    L.xd = take((size_t)T * (H / 32) * 2);
+    L.xs = take((size_t)T * (H / 32) * 2);
+    L.xsum = take((size_t)T * (H / 32) * 4);
+    L.ids = take((size_t)T * k * 4);
+    L.w = take((size_t)T * k * 4);
+    L.counts = take((size_t)E * 4);
+    L.offsets = take((size_t)(E + 1) * 4);
+    L.perm = take((size_t)T * k * 4);
+    L.inv_perm = take((size_t)T * k * 4);
+    L.chunk_counts = take((size_t)L.n_chunks * E * 4);
+    L.chunk_base = take((size_t)L.n_chunks * E * 4);
+    L.hq = take((size_t)L.slots * L.hpad);
+    L.hd = take((size_t)L.slots * (L.hpad / 32) * 2);
+    L.hs = take((size_t)L.slots * (L.hpad / 32) * 2);
+    L.hsum = take((size_t)L.slots * (L.hpad / 32) * 4);
+    L.h = (flags & MOE_F_KEEP_H) ? take((size_t)L.slots * F * 4) : 0;
+    L.y = (flags & MOE_F_DETERMINISTIC) ? take((size_t)L.slots * H * 4) : 0;
+    L.total = p;
+    return L;
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+uint64_t moe_kernels_enqueued(void) { return (uint64_t)g_kernels.load(); }
+
+const char *moe_status_string(moe_status s) {
+    switch (s) {
+        case MOE_OK: return "ok";
+        case MOE_ERR_INVALID_ARG: return "invalid argument";
+        case MOE_ERR_UNSUPPORTED: return "unsupported shape or format";
+        case MOE_ERR_ALIGNMENT: return "misaligned pointer or stride";
+        case MOE_ERR_CUDA: return "CUDA runtime error";
+        case MOE_ERR_NONFINITE: return "non-finite input";
+        case MOE_ERR_BOUNDS: return "descriptor outside the arena";
+        case MOE_ERR_TIMEOUT: return "device wait timed out";
+        case MOE_ERR_WORKSPACE: return "workspace too small";
+    }
+    return "unknown status";
+}
+
+moe_status moe_arena_create(const void *d_arena, size_t arena_bytes, int hidden, int ffn,
+                            int n_experts, int shared_expert, const moe_expert_desc *host_descs,
+                            moe_arena **out) {
+    if (!out) return MOE_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (!d_arena || !host_descs || hidden <= 0 || ffn <= 0 || n_experts <= 0) return MOE_ERR_INVALID_ARG;
+    if (hidden % 32 || ffn % 32) return MOE_ERR_INVALID_ARG;
+    if (n_experts > kMaxE) return MOE_ERR_UNSUPPORTED;
+    if (hidden > 4096 || ffn > 4096) return MOE_ERR_UNSUPPORTED;
+    if (shared_expert != -1 && shared_expert != n_experts) return MOE_ERR_INVALID_ARG;
+    if (!aligned(d_arena, 256)) return MOE_ERR_ALIGNMENT;
+    const int n = n_experts + (shared_expert >= 0 ? 1 : 0);
+    std::vector<ExpertDev> dev(n);
+    int fmt_mask = 0;
+    for (int e = 0; e < n; e++) {
+        const moe_expert_desc &d = host_descs[e];
+        if (d.fmt < 0 || d.fmt > 2 || d.reserved != 0) return MOE_ERR_INVALID_ARG;
+        const int bw = block_weights(d.fmt), bb = block_bytes(d.fmt);
+        if (hidden % bw) return MOE_ERR_UNSUPPORTED;
+        const int rows[3] = {ffn, ffn, hidden};
+        const int width[3] = {hidden, hidden, ffn};
+        for (int t = 0; t < 3; t++) {
+            const uint64_t packed = (uint64_t)((width[t] + bw - 1) / bw) * bb;
+            if (d.off[t] % 16 || d.stride[t] % 16) return MOE_ERR_ALIGNMENT;
+            if (d.stride[t] < packed || d.stride[t] > (1u << 30)) return MOE_ERR_INVALID_ARG;
+            const uint64_t end = d.off[t] + (uint64_t)(rows[t] - 1) * d.stride[t] + packed;
+            if (d.off[t] > arena_bytes || end > arena_bytes) return MOE_ERR_BOUNDS;
+            dev[e].m[t] = static_cast<const uint8_t *>(d_arena) + d.off[t];
+            dev[e].stride[t] = (uint32_t)d.stride[t];
+        }
+        dev[e].fmt = d.fmt;
+        dev[e].pad = 0;
+        fmt_mask |= 1 << d.fmt;
+    }
+    moe_arena *A = new (std::nothrow) moe_arena();
+    if (!A) return MOE_ERR_CUDA;
+    A->base = static_cast<const uint8_t *>(d_arena);
+    A->bytes = arena_bytes;
+    A->H = hidden;
+    A->F = ffn;
+    A->E = n_experts;
+    A->shared = shared_expert;
+    A->n = n;
+    A->fmt_mask = fmt_mask;
+    A->descs.assign(host_descs, host_descs + n);
+    if (cudaMalloc(&A->d_experts, sizeof(ExpertDev) * n) != cudaSuccess ||
+        cudaMemcpy(A->d_experts, dev.data(), sizeof(ExpertDev) * n, cudaMemcpyHostToDevice) !=
+            cudaSuccess) {
+        cudaFree(A->d_experts);
+        delete A;
+        return MOE_ERR_CUDA;
+    }
+    *out = A;
+    return MOE_OK;
+}
+
+void moe_arena_destroy(moe_arena *arena) {
+    if (!arena) return;
+    cudaFree(arena->d_experts);
+    delete arena;
+}
+
+moe_status moe_workspace_size(const moe_arena *arena, int max_tokens, int k, uint32_t flags,
+                              size_t *bytes) {
+    if (!arena || !bytes || max_tokens <= 0 || k <= 0 || k > kMaxK || k > arena->E)
+        return MOE_ERR_INVALID_ARG;
+    *bytes = ws_layout(arena, max_tokens, k, flags).total;
+    return MOE_OK;
+}
+
+moe_status moe_quantize_act(const float *d_x, int T, int H, int8_t *d_q, uint16_t *d_d,
+                            uint16_t *d_s, uint32_t *d_status, void *stream) {
+    if (!d_x || !d_q || !d_d || !d_s || T < 0 || H <= 0 || H % 32) return MOE_ERR_INVALID_ARG;
+    if (!aligned(d_x, 16) || !aligned(d_q, 16) || !aligned(d_d, 2) || !aligned(d_s, 2))
+        return MOE_ERR_ALIGNMENT;
+    if (launch_quantize(d_x, (int64_t)T * H / 32, d_q, d_d, d_s, nullptr, d_status,
+                        (cudaStream_t)stream) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    return MOE_OK;
+}
+
+static size_t route_ws_bytes(int T, int E, int k) {
+    const int n_chunks = (T + kChunk - 1) / kChunk;
+    size_t p = 0;
+    p = align256(p + (size_t)n_chunks * E * 4);   // chunk counts
+    p = align256(p + (size_t)n_chunks * E * 4);   // chunk cursors
+    p = align256(p + sizeof(Job) * (size_t)(std::min(E, T * k) + 1));
+    p = align256(p + 4);
+    return p;
+}
+
+moe_status moe_route_workspace_size(int T, int E, int k, size_t *bytes) {
+    if (!bytes || T <= 0 || E <= 0 || k <= 0 || k > kMaxK || k > E) return MOE_ERR_INVALID_ARG;
+    if (E > kMaxE) return MOE_ERR_UNSUPPORTED;
+    *bytes = route_ws_bytes(T, E, k);
+    return MOE_OK;
+}
+
+moe_status moe_route_topk(const float *d_logits, int T, int E, int k, int32_t *d_ids,
+                          float *d_w, int32_t *d_counts, int32_t *d_offsets, int32_t *d_perm,
+                          int32_t *d_inv_perm, uint32_t *d_status, void *d_ws, size_t ws_bytes,
+                          void *stream) {
+    if (!d_logits || !d_ids || !d_w || !d_counts || !d_offsets || !d_perm || !d_ws)
+        return MOE_ERR_INVALID_ARG;
+    if (T <= 0 || E <= 0 || k <= 0 || k > kMaxK || k > E) return MOE_ERR_INVALID_ARG;
+    if (E > kMaxE) return MOE_ERR_UNSUPPORTED;
+    if (!aligned(d_ws, 256)) return MOE_ERR_ALIGNMENT;
+    if (ws_bytes < route_ws_bytes(T, E, k)) return MOE_ERR_WORKSPACE;
+    cudaStream_t st = (cudaStream_t)stream;
+    const int n_chunks = (T + kChunk - 1) / kChunk;
+    uint8_t *ws = static_cast<uint8_t *>(d_ws);
+    int32_t *cc = reinterpret_cast<int32_t *>(ws);
+    int32_t *cb = reinterpret_cast<int32_t *>(ws + align256((size_t)n_chunks * E * 4));
+    Job *jobs = reinterpret_cast<Job *>(ws + 2 * align256((size_t)n_chunks * E * 4));
+    int32_t *nj = reinterpret_cast<int32_t *>(
+        ws + 2 * align256((size_t)n_chunks * E * 4) +
+        align256(sizeof(Job) * (size_t)(std::min(E, T * k) + 1)));
+    if (launch_topk(d_logits, T, E, k, d_ids, d_w, d_status, st) != cudaSuccess) return MOE_ERR_CUDA;
+    if (launch_group(d_ids, T, k, E, 0, d_counts, d_offsets, d_perm, d_inv_perm, cc, cb, jobs, nj,
+                     st) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    return MOE_OK;
+}
+
+moe_status moe_ws_views(const moe_arena *arena, void *d_ws, int T, int k, uint32_t flags,
+                        moe_ws_view *out) {
+    if (!arena || !d_ws || !out || T <= 0 || k <= 0 || k > kMaxK || k > arena->E)
+        return MOE_ERR_INVALID_ARG;
+    const WsLayout L = ws_layout(arena, T, k, flags);
+    uint8_t *ws = static_cast<uint8_t *>(d_ws);
+    out->status = reinterpret_cast<uint32_t *>(ws + L.status);
+    out->xq = reinterpret_cast<int8_t *>(ws + L.xq);
+    out->xd = reinterpret_cast<uint16_t *>(ws + L.xd);
+    out->xs = reinterpret_cast<uint16_t *>(ws + L.xs);
+    out->ids = reinterpret_cast<int32_t *>(ws + L.ids);
+    out->w = reinterpret_cast<float *>(ws + L.w);
+    out->counts = reinterpret_cast<int32_t *>(ws + L.counts);
+    out->offsets = reinterpret_cast<int32_t *>(ws + L.offsets);
+    out->perm = reinterpret_cast<int32_t *>(ws + L.perm);
+    out->inv_perm = reinterpret_cast<int32_t *>(ws + L.inv_perm);
+    out->hq = reinterpret_cast<int8_t *>(ws + L.hq);
+    out->hd = reinterpret_cast<uint16_t *>(ws + L.hd);
+    out->hs = reinterpret_cast<uint16_t *>(ws + L.hs);
+    out->h = (flags & MOE_F_KEEP_H) ? reinterpret_cast<float *>(ws + L.h) : nullptr;
+    out->slots = L.slots;
+    out->hpad = L.hpad;
+    return MOE_OK;
+}
+
+moe_status moe_read_status(uint32_t *d_status_word, void *stream, int clear,
+                           moe_status *device_status) {
+    if (!d_status_word || !device_status) return MOE_ERR_INVALID_ARG;
+    cudaStream_t st = (cudaStream_t)stream;
+    uint32_t v = 0;
+    if (cudaMemcpyAsync(&v, d_status_word, 4, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    if (clear && cudaMemsetAsync(d_status_word, 0, 4, st) != cudaSuccess) return MOE_ERR_CUDA;
+    *device_status = (moe_status)v;
+    return MOE_OK;
+}
+
+moe_status moe_forward(const moe_arena *arena, const float *d_x, const float *d_logits, int T,
+                       int k, float *d_out, void *d_ws, size_t ws_bytes, uint32_t flags,
+                       void *stream) {
+    if (!arena || !d_x || !d_logits || !d_out || !d_ws) return MOE_ERR_INVALID_ARG;
+    if (T <= 0 || k <= 0 || k > kMaxK || k > arena->E) return MOE_ERR_INVALID_ARG;
+    if ((flags & MOE_F_FORCE_DECODE) && (flags & MOE_F_FORCE_PREFILL)) return MOE_ERR_INVALID_ARG;
+    if (!aligned(d_x, 16) || !aligned(d_out, 16) || !aligned(d_logits, 4) || !aligned(d_ws, 256))
+        return MOE_ERR_ALIGNMENT;
+    const WsLayout L = ws_layout(arena, T, k, flags);
+    if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+    cudaStream_t st = (cudaStream_t)stream;
+    uint8_t *ws = static_cast<uint8_t *>(d_ws);
+    const int H = arena->H, E = arena->E;
+    const int shared = arena->shared >= 0 ? 1 : 0;
+    const bool decode = (flags & MOE_F_FORCE_DECODE) ||
+                        (!(flags & MOE_F_FORCE_PREFILL) && T <= kDecodeMaxT);
+
+    uint32_t *status = reinterpret_cast<uint32_t *>(ws + L.status);
+    int8_t *xq = reinterpret_cast<int8_t *>(ws + L.xq);
+    uint16_t *xd = reinterpret_cast<uint16_t *>(ws + L.xd);
+    uint16_t *xs = reinterpret_cast<uint16_t *>(ws + L.xs);
+    float *xsum = reinterpret_cast<float *>(ws + L.xsum);
+    int32_t *ids = reinterpret_cast<int32_t *>(ws + L.ids);
+    float *w = reinterpret_cast<float *>(ws + L.w);
+    int32_t *counts = reinterpret_cast<int32_t *>(ws + L.counts);
+    int32_t *offsets = reinterpret_cast<int32_t *>(ws + L.offsets);
+    int32_t *perm = reinterpret_cast<int32_t *>(ws + L.perm);
+    int32_t *inv_perm = reinterpret_cast<int32_t *>(ws + L.inv_perm);
+    Job *jobs = reinterpret_cast<Job *>(ws + L.jobs);
+    int32_t *njobs = reinterpret_cast<int32_t *>(ws + L.njobs);
+
+    // a1-a3
+    const bool small_route = T <= kDecodeMaxT && T * k <= kDecodeMaxT * kMaxK &&
+                             ((size_t)T * E + E) * 4 <= 96 * 1024;
+    cudaError_t err;
+    if (small_route) {
+        err = launch_route_small(d_x, d_logits, T, H, E, k, shared, L, ws, st);
+    } else {
+        err = launch_quantize(d_x, (int64_t)T * H / 32, xq, xd, xs, xsum, status, st);
+        if (err == cudaSuccess) err = launch_topk(d_logits, T, E, k, ids, w, status, st);
+        if (err == cudaSuccess)
+            err = launch_group(ids, T, k, E, shared, counts, offsets, perm, inv_perm,
+                               reinterpret_cast<int32_t *>(ws + L.chunk_counts),
+                               reinterpret_cast<int32_t *>(ws + L.chunk_base), jobs, njobs, st);
+    }
+    if (err != cudaSuccess) return MOE_ERR_CUDA;
+
+    FfnArgs a{};
+    a.experts = arena->d_experts;
+    a.jobs = jobs;
+    a.njobs = njobs;
+    a.perm = perm;
+    a.inv_perm = inv_perm;
+    a.w = w;
+    a.xq = xq;
+    a.xd = xd;
+    a.xsum = xsum;
+    a.hq = reinterpret_cast<int8_t *>(ws + L.hq);
+    a.hd = reinterpret_cast<uint16_t *>(ws + L.hd);
+    a.hs = reinterpret_cast<uint16_t *>(ws + L.hs);
+    a.hsum = reinterpret_cast<float *>(ws + L.hsum);
+    a.h = (flags & MOE_F_KEEP_H) ? reinterpret_cast<float *>(ws + L.h) : nullptr;
+    a.y = (flags & MOE_F_DETERMINISTIC) ? reinterpret_cast<float *>(ws + L.y) : nullptr;
+    a.out = d_out;
+    a.status = status;
+    a.T = T;
+    a.k = k;
+    a.H = H;
+    a.F = arena->F;
+    a.hpad = L.hpad;
+    a.max_jobs = L.max_jobs;
+    a.fmt_mask = arena->fmt_mask;
+
+    // a4 + a5
+    err = launch_gateup_gemv(a, st);
+    if (err != cudaSuccess) return MOE_ERR_CUDA;
+    // a6 + a7
+    if (decode && T <= kDecodeMaxT) {
+        err = launch_down_decode(a, st);
+    } else if (flags & MOE_F_DETERMINISTIC) {
+        err = launch_down_grouped(a, true, st);
+        if (err == cudaSuccess) err = launch_combine(a, shared != 0, st);
+    } else {
+        err = cudaMemsetAsync(d_out, 0, (size_t)T * H * sizeof(float), st);
+        if (err == cudaSuccess) err = launch_down_grouped(a, false, st);
+    }
+    return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status moe_debug_dequant(const moe_arena *arena, int expert, int which, float *d_out,
+                             void *stream) {
+    if (!arena || !d_out || expert < 0 || expert >= arena->n || which < 0 || which > 2)
+        return MOE_ERR_INVALID_ARG;
+    const moe_expert_desc &d = arena->descs[expert];
+    const int bw = block_weights(d.fmt);
+    const int rows = which < 2 ? arena->F : arena->H;
+    const int width = which < 2 ? arena->H : arena->F;
+    const int nb = (width + bw - 1) / bw;
+    if (launch_dequant(arena->base + d.off[which], d.fmt, rows, nb, (int)d.stride[which], d_out,
+                       (cudaStream_t)stream) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    return MOE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,152 @@
+// moe_internal.cuh -- shared declarations of the libmoe.so kernels (sm_100a only).
+//
+// Block formats (GGUF layouts, little endian; see include/moe.h):
+//   Q4_K 144 B / 256 weights: [0,2) fp16 d, [2,4) fp16 dmin, [4,16) S: packed 6-bit scales and
+//        mins of 8 sub-blocks of 32, [16,144) qs: byte 32c+r holds element 64c+r (low nibble,
+//        sub-block 2c) and element 64c+32+r (high nibble, sub-block 2c+1).
+//   Q5_K 176 B: as Q4_K with qh[32] at [16,48) and qs at [48,176); bit 2c of qh[r] is the fifth
+//        bit of element 64c+r, bit 2c+1 that of element 64c+32+r.
+//   Q8_0 34 B / 32 weights: fp16 d, int8 q[32].
+//   Q8_1 (activations, stored SoA): per 32 values int8 q[32], fp16 d, fp16 s = d * sum(q).
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "moe.h"
+
+#if defined(__CUDA_ARCH__) && (__CUDA_ARCH__ < 1000)
+#error "libmoe is built for sm_100a only"
+#endif
+
+namespace moe {
+
+constexpr int kQ = 32;            // Q8_1 / Q8_0 block length and K-quant sub-block length
+constexpr int kSB = 256;          // K-quant super-block length
+constexpr int kQ4KBytes = 144;
+constexpr int kQ5KBytes = 176;
+constexpr int kQ80Bytes = 34;
+constexpr int kMaxK = 32;         // routed experts per token
+constexpr int kMaxE = 4096;       // experts per layer
+constexpr int kDecodeMaxT = 16;   // largest batch the dequant-GEMV path takes by default
+constexpr int kChunk = 64;        // tokens per histogram chunk in the grouping kernels
+
+__host__ __device__ inline int block_weights(int fmt) { return fmt == MOE_FMT_Q8_0 ? 32 : 256; }
+__host__ __device__ inline int block_bytes(int fmt) {
+    return fmt == MOE_FMT_Q4_K ? kQ4KBytes : fmt == MOE_FMT_Q5_K ? kQ5KBytes : kQ80Bytes;
+}
+
+// Device copy of one expert (the descriptor with the arena base folded in).
+struct ExpertDev {
+    const uint8_t *m[3];      // gate, up, down
+    uint32_t stride[3];
+    int32_t fmt;
+    int32_t pad;
+};
+
+// One unit of grouped work: an expert and the contiguous run of slots routed to it.
+// Slots [slot0, slot0 + n) index the Q8_1(h) rows; routed slots are perm positions, the
+// shared expert's slots are T*k + t.
+struct Job {
+    int32_t expert;
+    int32_t slot0;
+    int32_t n;
+    int32_t shared;           // 1 for the shared expert (slot i is token i, weight 1)
+};
+
+struct moe_arena_impl;
+
+// Offsets (bytes) of everything moe_forward keeps in its workspace.
+struct WsLayout {
+    size_t status, njobs, jobs, xq, xd, xs, xsum, ids, w, counts, offsets, perm, inv_perm,
+        chunk_counts, chunk_base, hq, hd, hs, hsum, h, y, total;
+    int slots, hpad, max_jobs, n_chunks;
+};
+
+// ------------------------------------------------------------------ device helpers
+
+__device__ __forceinline__ void set_status(uint32_t *st, uint32_t code) {
+    if (st) atomicCAS(st, 0u, code);
+}
+
+__device__ __forceinline__ float half_bits_to_float(uint32_t bits16) {
+    return __half2float(__ushort_as_half((unsigned short)(bits16 & 0xFFFFu)));
+}
+
+// Byte i (0..11) of the packed scale words S0 = bytes 4..7, S1 = 8..11, S2 = 12..15 of a block.
+__device__ __forceinline__ uint32_t sbyte(uint32_t s0, uint32_t s1, uint32_t s2, int i) {
+    uint32_t w = i < 4 ? s0 : (i < 8 ? s1 : s2);
+    return (w >> (8 * (i & 3))) & 0xFFu;
+}
+
+// 6-bit scale and min of sub-block j of a K-quant block, from the 12 packed bytes.
+__device__ __forceinline__ void kq_scale_min(uint32_t s0, uint32_t s1, uint32_t s2, int j,
+                                             int &sc, int &mn) {
+    if (j < 4) {
+        sc = sbyte(s0, s1, s2, j) & 63;
+        mn = sbyte(s0, s1, s2, j + 4) & 63;
+    } else {
+        uint32_t b = sbyte(s0, s1, s2, j + 4);
+        sc = (b & 15) | ((sbyte(s0, s1, s2, j - 4) >> 6) << 4);
+        mn = (b >> 4) | ((sbyte(s0, s1, s2, j) >> 6) << 4);
+    }
+}
+
+// ------------------------------------------------------------------ launchers (host)
+
+// Kernels enqueued (or captured into a graph) by this library in this process.
+void note_launches(int n);
+
+// Raise a kernel's dynamic shared memory limit to at least `bytes` on the current device.  The
+// attribute is set once per (device, kernel, size) so that launches recorded under stream
+// capture make no attribute call.
+cudaError_t ensure_smem_impl(const void *kernel, size_t bytes);
+template <typename Kernel>
+inline cudaError_t ensure_smem(Kernel kernel, size_t bytes) {
+    return ensure_smem_impl(reinterpret_cast<const void *>(kernel), bytes);
+}
+
+cudaError_t launch_quantize(const float *x, int64_t nblocks, int8_t *q, uint16_t *d, uint16_t *s,
+                            float *dsum, uint32_t *status, cudaStream_t st);
+
+cudaError_t launch_route_small(const float *x, const float *logits, int T, int H, int E, int k,
+                               int shared, const WsLayout &L, uint8_t *ws, cudaStream_t st);
+
+cudaError_t launch_topk(const float *logits, int T, int E, int k, int32_t *ids, float *w,
+                        uint32_t *status, cudaStream_t st);
+
+cudaError_t launch_group(const int32_t *ids, int T, int k, int E, int shared, int32_t *counts,
+                         int32_t *offsets, int32_t *perm, int32_t *inv_perm,
+                         int32_t *chunk_counts, int32_t *chunk_base, Job *jobs, int32_t *njobs,
+                         cudaStream_t st);
+
+struct FfnArgs {
+    const ExpertDev *experts;
+    const Job *jobs;
+    const int32_t *njobs;
+    const int32_t *perm;
+    const int32_t *inv_perm;
+    const float *w;
+    const int8_t *xq;
+    const uint16_t *xd;
+    const float *xsum;
+    int8_t *hq;
+    uint16_t *hd, *hs;
+    float *hsum;
+    float *h;              // optional fp32 h
+    float *y;              // deterministic prefill: y per slot
+    float *out;
+    uint32_t *status;
+    int T, k, H, F, hpad, max_jobs, fmt_mask;
+};
+
+cudaError_t launch_gateup_gemv(const FfnArgs &a, cudaStream_t st);
+cudaError_t launch_down_decode(const FfnArgs &a, cudaStream_t st);
+cudaError_t launch_down_grouped(const FfnArgs &a, bool deterministic, cudaStream_t st);
+cudaError_t launch_combine(const FfnArgs &a, bool shared, cudaStream_t st);
+
+cudaError_t launch_dequant(const uint8_t *m, int fmt, int rows, int nblocks, int stride,
+                           float *out, cudaStream_t st);
+
+}  // namespace moe

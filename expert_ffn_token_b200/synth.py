@@ -364,3 +364,65 @@ def router_logits(w: Workload, layer: int, tokens: int | None = None) -> np.ndar
         L[bad] = _logit_rows(w, layer, attempt, bad)
         bad = bad[~_gaps_ok(L[bad], w.k)]
     return L
+
+
+# ------------------------------------------------------------------ device fill (multi-GB arenas)
+
+_synth_lib = None
+
+
+def _synth():
+    global _synth_lib
+    if _synth_lib is None:
+        import ctypes
+        from pathlib import Path
+        p = Path(__file__).resolve().parent / "libmoe_synth.so"
+        if not p.exists():
+            raise ImportError(f"{p} is not built: run `python -m expert_ffn_token_b200.build`")
+        _synth_lib = ctypes.CDLL(str(p))
+        _synth_lib.synth_fill_tensors.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+                                                  ctypes.c_void_p]
+    return _synth_lib
+
+
+def device_fill_layer(w: Workload, layer: int, d_base: int, stream=None) -> ArenaLayout:
+    """Write layer `layer`'s arena at device address d_base (lay.nbytes bytes, 256-aligned):
+    the same bytes as host_arena(w, layer), drawn on the GPU."""
+    import ctypes
+
+    class _T(ctypes.Structure):
+        _fields_ = [("dst_off", ctypes.c_uint64), ("key_raw", ctypes.c_uint64),
+                    ("key_d", ctypes.c_uint64), ("key_dmin", ctypes.c_uint64),
+                    ("rows", ctypes.c_int32), ("stride", ctypes.c_int32),
+                    ("nblocks", ctypes.c_int32), ("block_bytes", ctypes.c_int32),
+                    ("kquant", ctypes.c_int32), ("valid_last", ctypes.c_int32)]
+
+    fmts = layer_formats(w, layer)
+    lay = arena_layout(w, fmts)
+    tab = (_T * (lay.n * 3))()
+    for e in range(lay.n):
+        f = int(fmts[e])
+        for t in range(3):
+            rows, width = tensor_shape(w, t)
+            nb = row_blocks(f, width)
+            r = tab[e * 3 + t]
+            r.dst_off = int(lay.offs[e, t])
+            r.key_raw = key(w.seed, layer, e, t, 0)
+            r.key_d = key(w.seed, layer, e, t, 1)
+            r.key_dmin = key(w.seed, layer, e, t, 2)
+            r.rows = rows
+            r.stride = int(lay.strides[e, t])
+            r.nblocks = nb
+            r.block_bytes = BLOCK_BYTES[f]
+            r.kquant = 0 if f == Q8_0 else 1
+            r.valid_last = 8 if f == Q8_0 else (width - (nb - 1) * 256) // 32
+    rc = _synth().synth_fill_tensors(d_base, ctypes.cast(tab, ctypes.c_void_p), lay.n * 3, stream)
+    if rc != 0:
+        raise RuntimeError(f"synth_fill_tensors failed ({rc})")
+    return lay
+
+
+def layout_descs(lay: ArenaLayout):
+    """(fmt, offsets, strides) per expert, the form moe.arena_create takes."""
+    return [(int(lay.fmts[e]), tuple(int(v) for v in lay.offs[e]),
+             tuple(int(v) for v in lay.strides[e])) for e in range(lay.n)]

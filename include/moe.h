@@ -1,0 +1,179 @@
+/*
+ * moe.h -- C ABI of libmoe.so, a B200 (sm_100a) quantized mixture-of-experts layer.
+ *
+ * The layer (the per-token expert path of the Strata engine pages):
+ *   - "Strata: a 125B MoE at 94 tok/s on a 12 GB Card", section "Three architecture facts":
+ *     512 experts per layer, 10 routed + 1 always-on shared expert, hidden size 2,560;
+ *     "Strata-Sage-A1.5-GGUF": 256 experts, top-8.
+ *   - "Strata v0.1.31" release notes, section "Experimental: Unsloth UD-Q4_K_XL on a normal
+ *     PC": experts stored as Q4_K, Q5_K and Q8_0 blocks (GGUF), decoded bit for bit as
+ *     llama.cpp decodes them, dot products equal to ggml's within float rounding.
+ *   - "Strata v0.1.39" release notes, fixes list, #606: q8_1 activations;
+ *     "Strata-Sage-A1.5-GGUF", round-2 table: one activation quantization per token.
+ *
+ * For a batch of T tokens:  x fp32 [T][H], router logits fp32 [T][E]  ->  out fp32 [T][H]
+ *   a1  x is quantized once per token to Q8_1 blocks of 32 (int8 q, fp16 d, fp16 s)
+ *   a2  each token takes its k largest logits (ties: lower expert id) with weights
+ *       w = softmax over those k logits
+ *   a3  (token, slot) pairs are grouped by expert: counts, exclusive offsets, a permutation
+ *       stable in token order
+ *   a4  every chosen expert computes g = W_gate x^, u = W_up x^ from its packed weights
+ *   a5  h = silu(g) * u, re-quantized to Q8_1
+ *   a6  y = W_down h^
+ *   a7  out[t] = sum_j w[t][j] * y[t][e_j] + y[t][shared]     (shared expert: weight 1)
+ *
+ * Conventions for every entry point:
+ *   - Pointers named d_* are DEVICE pointers (cudaMalloc / torch CUDA memory) of the current
+ *     device; host_* are host pointers.  The caller owns all memory passed in.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).
+ *   - Work is enqueued asynchronously; MOE_OK means "validated and enqueued".
+ *   - Argument errors are detected on the host and returned before anything is enqueued.
+ *   - Problems only the device can see (a non-finite input, a bounded wait that ran out)
+ *     are recorded as the first error code in a 32-bit status word that the caller reads
+ *     with moe_read_status.  No kernel traps.
+ *   - No C++ exception crosses this interface.  Calls are thread-safe when they use distinct
+ *     workspaces.
+ */
+#ifndef MOE_H
+#define MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1,   /* bad size, null pointer, k > E, ...                      */
+    MOE_ERR_UNSUPPORTED = 2,   /* a shape or format this build does not handle             */
+    MOE_ERR_ALIGNMENT = 3,     /* a pointer or row stride not aligned as required          */
+    MOE_ERR_CUDA = 4,          /* a CUDA runtime call failed (launch, copy, attribute)     */
+    MOE_ERR_NONFINITE = 5,     /* device: an activation block or a logit row was not finite */
+    MOE_ERR_BOUNDS = 6,        /* descriptor offsets/strides reach outside the arena       */
+    MOE_ERR_TIMEOUT = 7,       /* device: a bounded wait gave up                           */
+    MOE_ERR_WORKSPACE = 8      /* workspace smaller than moe_workspace_size reported       */
+} moe_status;
+
+/* Block formats of the expert weights (GGUF layouts, little endian):
+ *   Q4_K  256 weights in 144 B: fp16 d, fp16 dmin, 12 B of packed 6-bit sub-block scales and
+ *         mins (8 sub-blocks of 32), 128 B of 4-bit quants; w = d*sc*q - dmin*m
+ *   Q5_K  256 weights in 176 B: as Q4_K plus a 32 B plane of fifth bits before the quants
+ *   Q8_0  32 weights in 34 B: fp16 d, 32 int8 q; w = d*q                                      */
+typedef enum { MOE_FMT_Q4_K = 0, MOE_FMT_Q5_K = 1, MOE_FMT_Q8_0 = 2 } moe_fmt;
+
+/* One expert inside the arena.  Matrices follow the GGUF convention: a row is one output
+ * neuron, blocks run along the input dimension.  gate and up: ffn rows of `hidden` weights;
+ * down: `hidden` rows of `ffn` weights rounded up to whole blocks (the weights past `ffn` must
+ * decode to 0).  off[] are byte offsets from the arena base (multiples of 16); stride[] are
+ * row strides in bytes (multiples of 16, at least the packed row size).                      */
+typedef struct {
+    int32_t fmt;          /* moe_fmt */
+    int32_t reserved;     /* must be 0 */
+    uint64_t off[3];      /* gate, up, down */
+    uint64_t stride[3];   /* gate, up, down */
+} moe_expert_desc;
+
+typedef struct moe_arena moe_arena;
+
+/* Register a device-resident expert arena: `n_experts` routed experts plus, when
+ * shared_expert >= 0, one more descriptor at index n_experts for the always-on shared expert
+ * (shared_expert must then equal n_experts).  host_descs has n_experts (+1) entries.
+ * hidden: multiple of 256 (K-quants) or 32 (Q8_0 only); ffn: multiple of 32.
+ * Checks every descriptor against arena_bytes (MOE_ERR_BOUNDS) and alignment; copies the table
+ * to the device (the one allocation the library makes, freed by moe_arena_destroy).  d_arena
+ * (256-byte aligned) must stay valid until moe_arena_destroy.                                */
+moe_status moe_arena_create(const void *d_arena, size_t arena_bytes, int hidden, int ffn,
+                            int n_experts, int shared_expert, const moe_expert_desc *host_descs,
+                            moe_arena **out);
+void moe_arena_destroy(moe_arena *arena);
+
+/* Forward flags. */
+#define MOE_F_DETERMINISTIC 1u   /* prefill: combine by gathering per-token sums (no atomics) */
+#define MOE_F_FORCE_DECODE 2u    /* use the grouped dequant-GEMV path whatever T is          */
+#define MOE_F_FORCE_PREFILL 4u   /* use the grouped tensor-core GEMM path whatever T is      */
+#define MOE_F_KEEP_H 8u          /* also store fp32 h (SwiGLU output) in the workspace       */
+
+/* Bytes of device workspace moe_forward needs for up to max_tokens tokens, k routed experts
+ * per token and the given flags.  The workspace is caller-owned scratch, 256-byte aligned. */
+moe_status moe_workspace_size(const moe_arena *arena, int max_tokens, int k, uint32_t flags,
+                              size_t *bytes);
+
+/* a1 alone.  d_x fp32 [T][H] -> d_q int8 [T][H], d_d / d_s fp16 bits [T][H/32] (SoA: the
+ * int8 rows stay contiguous).  H multiple of 32.  d_status (may be NULL): device uint32 that
+ * receives MOE_ERR_NONFINITE if a block held a non-finite value (that block is written as
+ * q = 0, d = s = 0).  All pointers 16-byte aligned.                                          */
+moe_status moe_quantize_act(const float *d_x, int T, int H, int8_t *d_q, uint16_t *d_d,
+                            uint16_t *d_s, uint32_t *d_status, void *stream);
+
+/* Bytes of workspace moe_route_topk needs for T tokens, E experts, k per token. */
+moe_status moe_route_workspace_size(int T, int E, int k, size_t *bytes);
+
+/* a2 + a3 alone.  d_logits fp32 [T][E] -> d_ids int32 [T][k] (descending logit, ties to the
+ * lower id), d_w fp32 [T][k] (softmax over the chosen logits), d_counts int32 [E],
+ * d_offsets int32 [E+1] (exclusive prefix sum), d_perm int32 [T*k]: perm[offsets[e] + r] =
+ * t*k + j for the r-th pair routed to e in ascending t; d_inv_perm (may be NULL) int32
+ * [T*k].  1 <= k <= min(E, 32), E <= 4096.  A token whose logits are not all finite gets ids
+ * 0..k-1, weights 1/k and MOE_ERR_NONFINITE in d_status (may be NULL).                       */
+moe_status moe_route_topk(const float *d_logits, int T, int E, int k, int32_t *d_ids,
+                          float *d_w, int32_t *d_counts, int32_t *d_offsets, int32_t *d_perm,
+                          int32_t *d_inv_perm, uint32_t *d_status, void *d_ws, size_t ws_bytes,
+                          void *stream);
+
+/* The whole layer, a1-a7.  d_x fp32 [T][hidden], d_logits fp32 [T][n_experts] -> d_out fp32
+ * [T][hidden] (overwritten).  1 <= T <= the max_tokens the workspace was sized for,
+ * 1 <= k <= min(n_experts, 32).  Intermediates (Q8_1 of x, ids, w, counts, offsets, perm,
+ * Q8_1 of h, optional fp32 h) are left in the workspace; moe_ws_views locates them.  They
+ * equal what moe_quantize_act / moe_route_topk produce for the same inputs.
+ * The grouped dequant-GEMV path (decode) is taken for T <= 16 unless a FORCE flag says
+ * otherwise.  The workspace's status word collects device-side errors (moe_read_status).   */
+moe_status moe_forward(const moe_arena *arena, const float *d_x, const float *d_logits, int T,
+                       int k, float *d_out, void *d_ws, size_t ws_bytes, uint32_t flags,
+                       void *stream);
+
+/* Device addresses of the intermediates inside a workspace laid out for (T, k, flags).
+ * Q8_1 of h is stored per slot: slot s < T*k is the s-th entry of perm (grouped by expert),
+ * slot T*k + t is token t's shared-expert row.  hpad = ffn rounded up to 256.                */
+typedef struct {
+    uint32_t *status;          /* 1 word                                               */
+    int8_t *xq;                /* [T][hidden]                                          */
+    uint16_t *xd, *xs;         /* [T][hidden/32] fp16 bits                             */
+    int32_t *ids;              /* [T][k]                                               */
+    float *w;                  /* [T][k]                                               */
+    int32_t *counts;           /* [E]                                                  */
+    int32_t *offsets;          /* [E+1]                                                */
+    int32_t *perm, *inv_perm;  /* [T*k]                                                */
+    int8_t *hq;                /* [slots][hpad]                                        */
+    uint16_t *hd, *hs;         /* [slots][hpad/32] fp16 bits                           */
+    float *h;                  /* [slots][ffn] fp32 (MOE_F_KEEP_H only, else NULL)     */
+    int32_t slots, hpad;
+} moe_ws_view;
+
+moe_status moe_ws_views(const moe_arena *arena, void *d_ws, int T, int k, uint32_t flags,
+                        moe_ws_view *out);
+
+/* Read the workspace's status word (blocks on `stream`), then reset it to 0 when clear != 0.
+ * d_status_word: the `status` pointer of moe_ws_views, or any d_status given above.        */
+moe_status moe_read_status(uint32_t *d_status_word, void *stream, int clear,
+                           moe_status *device_status);
+
+/* Debug export of one matrix (which: 0 gate, 1 up, 2 down; expert n_experts = shared) as
+ * fp32 [rows][row weights] where row weights = whole blocks.  Each value is
+ * RN32(RN32(d*sc)*q - RN32(dmin*m)) (K-quants) or d*q (Q8_0), bit for bit.               */
+moe_status moe_debug_dequant(const moe_arena *arena, int expert, int which, float *d_out,
+                             void *stream);
+
+/* Number of kernels this library has enqueued (or recorded into a CUDA graph under stream
+ * capture) in this process since it was loaded.  Counting a captured forward gives the
+ * kernels each replay of that graph launches. */
+uint64_t moe_kernels_enqueued(void);
+
+/* Static text of a status code. */
+const char *moe_status_string(moe_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_H */
