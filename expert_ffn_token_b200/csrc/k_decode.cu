@@ -1,0 +1,910 @@
+// k_decode.cu -- the whole layer (a1-a7) for small batches in ONE persistent kernel.
+//
+// Decode is bound by streaming the chosen experts' packed bytes once (the pages' decode chain
+// streams expert rows with register reductions, Strata-Sage-A1.5-GGUF round-2 table; the verify
+// pass packs the tokens that share an expert, Strata v0.1.39 release notes, Decode #646).  On
+// B200 that means megabytes in flight from the first microsecond and as few fixed latencies
+// as possible:
+//
+//   prologue (every CTA, identical results; CTA 0 also stores them in the workspace):
+//     logits and x are loaded at once; while warps 0..T-1 select each token's experts
+//     (logits held in registers, one redux.sync max + min per pick), the other warps quantize
+//     x to Q8_1 in shared memory; one warp then builds counts, offsets, slots and the job list
+//     from an expert bitmap (popc prefix sums), and the chosen experts' descriptors are cached.
+//   partition: the U * F/32 blocks of 32 gate/up rows go round-robin to the CTAs, so every CTA
+//     owns whole Q8_1(h) blocks and quantizes them itself; the H down rows are cut into one
+//     contiguous range per CTA sized so that every CTA streams the same number of bytes.
+//   pipeline: one producer thread streams the CTA's rows into a ring of shared-memory stages
+//     with bulk async copies (TMA engine, mbarrier byte counts, L2 evict-first) as far ahead
+//     as the ring allows; 8 consumer warps compute from shared memory.
+//   gate/up: a unit is 16 rows of gate and 16 of up; each warp takes 4 rows, each lane a fixed
+//     set of 16-byte quant chunks (activations loaded once per chunk, reused over the rows);
+//     h = silu(g) * u goes to shared memory and, once the 32-row block is complete, to Q8_1.
+//   down: after every CTA has published its blocks (bounded wait on one counter), all Q8_1(h)
+//     rows are staged in shared memory; warps run over every job's rows and add w * y into
+//     per-row sums; each output element is written once -- deterministic, no output atomics.
+// Every wait is bounded by %globaltimer and reports MOE_ERR_TIMEOUT instead of hanging.  The
+// down phase waits on the gate/up work of every CTA: the grid is one CTA per SM (all resident
+// together; a programmatically launched successor starts only once every CTA here has
+// started).  The last CTA to finish resets the counters.
+#include "dot.cuh"
+#include "ptx.cuh"
+#include "route_dev.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int kCW = 8;                       // consumer warps
+constexpr int kThreads = (kCW + 1) * 32;     // + one producer warp
+constexpr int kRG = 4;                       // gate/up rows per warp per unit
+constexpr int kUnitPairs = kRG * kCW / 2;    // 16 gate + 16 up rows per unit
+constexpr int kRD = 2;                       // down rows per warp per unit
+constexpr int kDownRows = kRD * kCW;         // 16 output rows per down unit
+constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s: far beyond any legitimate wait
+
+enum { ST_END = 0, ST_GU = 1, ST_DOWN = 2 };
+
+struct StageMeta {
+    int kind;   // ST_GU: a job, b first row, c rows      ST_DOWN: a i0, b rows, c j0, d j1, e last
+    int a, b, c, d, e, f, g;
+};
+
+struct JobX {                // a job with its expert's descriptor, cached in shared memory
+    const uint8_t *m[3];
+    uint32_t stride[3];
+    int fmt, expert, slot0, n, shared;
+};
+
+struct DecParams {
+    const ExpertDev *experts;
+    const float *x;
+    const float *logits;
+    float *out;
+    uint8_t *ws;
+    WsLayout L;
+    int T, H, F, E, k, shared, hpad;
+    int stage_bytes, nstages, max_jobs, slots;
+    int o_bar, o_meta, o_xq, o_xd, o_xs, o_jobs, o_stok, o_sw, o_hq, o_hd, o_hs, o_gu, o_h,
+        o_acc, o_misc;
+    int smem_bytes;
+};
+
+// ------------------------------------------------------------------ chunk-level math
+//
+// A K-quant row is cut into 16-byte quant chunks p = 8*sb + j (sb super-block, j = 0..7,
+// c = j/2, hh = j%2): chunk p holds elements 64c+16hh+[0,16) (low nibbles, sub-block 2c) and
+// 64c+32+16hh+[0,16) (high nibbles, sub-block 2c+1) of super-block sb.  A Q8_0 row is cut
+// into its 32-weight blocks (chunk p = block p).
+
+struct ActChunk {            // one token's activations matching one chunk
+    int4 xa, xb;             // 16 bytes for the low nibbles, 16 for the high (Q8_0: 32 bytes)
+    float dl, dh, sl, sh;    // Q8_1 d and exact d*sum(q) of the two 32-blocks (Q8_0: dl only)
+};
+
+__device__ __forceinline__ ActChunk load_act(const int8_t *q, const float *d, const float *s,
+                                             int p, bool q80) {
+    ActChunk a;
+    if (q80) {
+        a.xa = *reinterpret_cast<const int4 *>(q + 32 * p);
+        a.xb = *reinterpret_cast<const int4 *>(q + 32 * p + 16);
+        a.dl = d[p];
+        a.dh = a.sl = a.sh = 0.f;
+    } else {
+        const int sb = p >> 3, j = p & 7, c = j >> 1, hh = j & 1;
+        const int kl = sb * 256 + c * 64 + hh * 16;
+        const int bl = sb * 8 + 2 * c;
+        a.xa = *reinterpret_cast<const int4 *>(q + kl);
+        a.xb = *reinterpret_cast<const int4 *>(q + kl + 32);
+        a.dl = d[bl];
+        a.dh = d[bl + 1];
+        a.sl = s[bl];
+        a.sh = s[bl + 1];
+    }
+    return a;
+}
+
+// Weights of one chunk: unpacked quants and the scales of its two sub-blocks.  The 6-bit
+// scale/min pairs are extracted without branches: with c' = c & 1 the needed bytes sit at
+// positions 2c', 2c'+1 of the three scale words; c < 2 uses (S[j], S[j+4]) & 63, c >= 2 uses
+// the nibbles of S[j+4] with the top two bits of S[j-4] / S[j].
+struct WChunk {
+    uint32_t lo[4], hi[4];
+    float dl, dh, ml, mh;
+};
+
+template <bool Q5>
+__device__ __forceinline__ WChunk kq_chunk(const uint8_t *sbp, int j) {
+    const uint4 hdr = *reinterpret_cast<const uint4 *>(sbp);
+    const uint4 qv = *reinterpret_cast<const uint4 *>(sbp + (Q5 ? 48 : 16) + 16 * j);
+    const int c = j >> 1;
+    const int sh = 16 * (c & 1);
+    const uint32_t x0 = hdr.y >> sh, x1 = hdr.z >> sh, x2 = hdr.w >> sh;
+    uint32_t sc2, m2;
+    if (c < 2) {   // lane-constant: the compiler predicates both forms
+        sc2 = x0 & 0x3F3Fu;
+        m2 = x1 & 0x3F3Fu;
+    } else {
+        sc2 = (x2 & 0x0F0Fu) | ((x0 >> 2) & 0x3030u);
+        m2 = ((x2 >> 4) & 0x0F0Fu) | ((x1 >> 2) & 0x3030u);
+    }
+    const float d = half_bits_to_float(hdr.x), dmin = half_bits_to_float(hdr.x >> 16);
+    WChunk w;
+    w.dl = d * (float)(sc2 & 0xFFu);
+    w.dh = d * (float)((sc2 >> 8) & 0xFFu);
+    w.ml = dmin * (float)(m2 & 0xFFu);
+    w.mh = dmin * (float)((m2 >> 8) & 0xFFu);
+    const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
+    uint32_t hw[4] = {0u, 0u, 0u, 0u};
+    if (Q5) {
+        const uint4 qh = *reinterpret_cast<const uint4 *>(sbp + 16 + 16 * (j & 1));
+        hw[0] = qh.x;
+        hw[1] = qh.y;
+        hw[2] = qh.z;
+        hw[3] = qh.w;
+    }
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+        w.lo[i] = qw[i] & 0x0F0F0F0Fu;
+        w.hi[i] = (qw[i] >> 4) & 0x0F0F0F0Fu;
+        if (Q5) {
+            w.lo[i] |= ((hw[i] >> (2 * c)) & 0x01010101u) << 4;
+            w.hi[i] |= ((hw[i] >> (2 * c + 1)) & 0x01010101u) << 4;
+        }
+    }
+    return w;
+}
+
+// Lane share of sum_k w_k * xhat_k over one chunk.  `mf` is 1 on the lane that adds the two
+// sub-blocks' min terms (hh == 0) and 0 on its partner.
+__device__ __forceinline__ float kq_chunk_dot(const WChunk &w, const ActChunk &a, float mf) {
+    int il = __dp4a((int)w.lo[0], a.xa.x, 0);
+    il = __dp4a((int)w.lo[1], a.xa.y, il);
+    il = __dp4a((int)w.lo[2], a.xa.z, il);
+    il = __dp4a((int)w.lo[3], a.xa.w, il);
+    int ih = __dp4a((int)w.hi[0], a.xb.x, 0);
+    ih = __dp4a((int)w.hi[1], a.xb.y, ih);
+    ih = __dp4a((int)w.hi[2], a.xb.z, ih);
+    ih = __dp4a((int)w.hi[3], a.xb.w, ih);
+    float r = w.dl * (a.dl * (float)il);
+    r = fmaf(w.dh, a.dh * (float)ih, r);
+    r = fmaf(-mf * w.ml, a.sl, r);
+    r = fmaf(-mf * w.mh, a.sh, r);
+    return r;
+}
+
+__device__ __forceinline__ float q80_chunk_dot(const uint8_t *blk, const ActChunk &a) {
+    const float d = half_bits_to_float((uint32_t)blk[0] | ((uint32_t)blk[1] << 8));
+    uint32_t w[8];
+#pragma unroll
+    for (int i = 0; i < 8; i++)
+        w[i] = (uint32_t)blk[2 + 4 * i] | ((uint32_t)blk[3 + 4 * i] << 8) |
+               ((uint32_t)blk[4 + 4 * i] << 16) | ((uint32_t)blk[5 + 4 * i] << 24);
+    int acc = __dp4a((int)w[0], a.xa.x, 0);
+    acc = __dp4a((int)w[1], a.xa.y, acc);
+    acc = __dp4a((int)w[2], a.xa.z, acc);
+    acc = __dp4a((int)w[3], a.xa.w, acc);
+    acc = __dp4a((int)w[4], a.xb.x, acc);
+    acc = __dp4a((int)w[5], a.xb.y, acc);
+    acc = __dp4a((int)w[6], a.xb.z, acc);
+    acc = __dp4a((int)w[7], a.xb.w, acc);
+    return d * (a.dl * (float)acc);
+}
+
+// R rows (row r at base + r*stride, r < nrows) of K weights against n <= NT activation rows
+// (row t at q + act[t]*astride): lane-partial sums into acc[R][NT].  Each lane keeps its own
+// chunks p = lane, lane+32, ... and reuses their activations over the R rows.
+template <int NT, int R>
+__device__ __forceinline__ void rows_dot(int fmt, const uint8_t *base, uint32_t stride, int nrows,
+                                         int K, const int8_t *q, const float *d, const float *s,
+                                         int astride, const int *act, int n, float (&acc)[R][NT]) {
+    const int lane = threadIdx.x & 31;
+    const int nchunk = K / 32;
+    const bool q80 = fmt == MOE_FMT_Q8_0, q5 = fmt == MOE_FMT_Q5_K;
+    const int SBB = q5 ? kQ5KBytes : kQ4KBytes;
+    for (int p = lane; p < nchunk; p += 32) {
+        ActChunk a[NT];
+#pragma unroll
+        for (int t = 0; t < NT; t++)
+            if (t < n)
+                a[t] = load_act(q + (size_t)act[t] * astride, d + act[t] * (astride / 32),
+                                s + act[t] * (astride / 32), p, q80);
+        const int sb = p >> 3, j = p & 7;
+        const float mf = (j & 1) ? 0.f : 1.f;
+#pragma unroll
+        for (int r = 0; r < R; r++) {
+            if (r < nrows) {
+                const uint8_t *row = base + (size_t)r * stride;
+                if (q80) {
+#pragma unroll
+                    for (int t = 0; t < NT; t++)
+                        if (t < n) acc[r][t] += q80_chunk_dot(row + (size_t)p * kQ80Bytes, a[t]);
+                } else {
+                    const WChunk w = q5 ? kq_chunk<true>(row + (size_t)sb * SBB, j)
+                                        : kq_chunk<false>(row + (size_t)sb * SBB, j);
+#pragma unroll
+                    for (int t = 0; t < NT; t++)
+                        if (t < n) acc[r][t] += kq_chunk_dot(w, a[t], mf);
+                }
+            }
+        }
+    }
+}
+
+__device__ __forceinline__ uint32_t order_key(float f) {
+    const uint32_t u = __float_as_uint(f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float key_value(uint32_t k) {
+    return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
+// One warp: top-k of a logit row held in registers (VPL values per lane, value e at lane e%32,
+// slot e/32).  Descending logit, ties to the lower id; weights = softmax over the chosen k.
+template <int VPL>
+__device__ __forceinline__ void warp_topk_reg(const float *row, int E, int k, int *ids_out,
+                                              float *w_out, uint32_t *status) {
+    const int lane = threadIdx.x & 31;
+    uint32_t key[VPL];
+    bool fin = true;
+#pragma unroll
+    for (int i = 0; i < VPL; i++) {
+        const int e = lane + 32 * i;
+        const float v = e < E ? row[e] : 0.f;
+        fin = fin && isfinite(v);
+        key[i] = e < E ? order_key(v) : 0u;
+    }
+    if (!__all_sync(kFullMask, fin)) {
+        if (lane < k) {
+            ids_out[lane] = lane;
+            w_out[lane] = __fdiv_rn(1.0f, (float)k);
+        }
+        if (lane == 0) set_status(status, MOE_ERR_NONFINITE);
+        return;
+    }
+    uint32_t my_key = 0;
+    int my_id = 0;
+    for (int j = 0; j < k; j++) {
+        uint32_t bk = 0;
+        int bi = 0;
+#pragma unroll
+        for (int i = 0; i < VPL; i++)
+            if (key[i] > bk) {   // strict: the lower slot (lower id) wins ties within a lane
+                bk = key[i];
+                bi = i;
+            }
+        const uint32_t m = __reduce_max_sync(kFullMask, bk);
+        const uint32_t win = __reduce_min_sync(kFullMask, bk == m ? (uint32_t)(lane + 32 * bi)
+                                                                   : 0xFFFFFFFFu);
+        if (lane == j) {
+            my_key = m;
+            my_id = (int)win;
+        }
+        if ((int)(win & 31u) == lane) {
+#pragma unroll
+            for (int i = 0; i < VPL; i++)
+                if (i == (int)(win >> 5)) key[i] = 0u;
+        }
+    }
+    const float l0 = key_value(__shfl_sync(kFullMask, my_key, 0));
+    const float ex = lane < k ? expf(key_value(my_key) - l0) : 0.f;
+    float sum = ex;
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) sum += __shfl_xor_sync(kFullMask, sum, o);
+    if (lane < k) {
+        ids_out[lane] = my_id;
+        w_out[lane] = __fdiv_rn(ex, sum);
+    }
+}
+
+// Q8_1 of 32 values held one per lane; lane 0 gets d16, s16, dsum.
+__device__ __forceinline__ int q8_1_lane(float v, bool &fin, uint16_t &d16, uint16_t &s16,
+                                         float &dsum) {
+    fin = __all_sync(kFullMask, isfinite(v));
+    float a = fabsf(v);
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) a = fmaxf(a, __shfl_xor_sync(kFullMask, a, o));
+    const float d = __fdiv_rn(a, 127.0f);
+    int qi = 0;
+    if (fin && d != 0.0f) qi = max(-127, min(127, (int)roundf(__fdiv_rn(v, d))));
+    int sum = qi;
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) sum += __shfl_xor_sync(kFullMask, sum, o);
+    if (fin) {
+        const __half dh = __float2half_rn(d);
+        d16 = __half_as_ushort(dh);
+        s16 = __half_as_ushort(__float2half_rn(__fmul_rn(d, (float)sum)));
+        dsum = __fmul_rn(__half2float(dh), (float)sum);
+    } else {
+        qi = 0;
+        d16 = s16 = 0;
+        dsum = 0.f;
+    }
+    return qi;
+}
+
+// Down-row boundary of CTA c: rows are shared out in proportion to the bytes each CTA still has
+// room for after its gate/up blocks, so that every CTA streams about the same total.
+__device__ __forceinline__ int down_bound(int c, int G, int H, int n_blk, double blk_bytes,
+                                          double row_bytes) {
+    if (c >= G) return H;
+    const int q = n_blk / G, r = n_blk % G;
+    const double total = blk_bytes * n_blk + row_bytes * H;
+    const double target = total / G;
+    const double cap_hi = fmax(0.0, target - (q + 1) * blk_bytes);   // CTAs c < r own q+1 blocks
+    const double cap_lo = fmax(0.0, target - q * blk_bytes);
+    const double ctot = r * cap_hi + (G - r) * cap_lo;
+    if (ctot <= 0.0) return (int)((long long)H * c / G);
+    const double cc = fmin((double)c, (double)r) * cap_hi + fmax(0.0, (double)(c - r)) * cap_lo;
+    return (int)floor(H * (cc / ctot));
+}
+
+template <int NT>
+__global__ void __launch_bounds__(kThreads, 1) k_decode_fused(const DecParams P) {
+    extern __shared__ __align__(128) uint8_t sm[];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const WsLayout &L = P.L;
+    uint8_t *ws = P.ws;
+    uint32_t *status = reinterpret_cast<uint32_t *>(ws + L.status);
+    uint32_t *ctr = reinterpret_cast<uint32_t *>(ws + L.sync);   // [1] blocks_done [2] finished
+    const bool cta0 = blockIdx.x == 0;
+    const int T = P.T, H = P.H, F = P.F, E = P.E, k = P.k;
+    const int nbH = H / 32;
+
+    uint64_t *full = reinterpret_cast<uint64_t *>(sm + P.o_bar);
+    uint64_t *empty = full + P.nstages;
+    StageMeta *meta = reinterpret_cast<StageMeta *>(sm + P.o_meta);
+    int8_t *s_xq = reinterpret_cast<int8_t *>(sm + P.o_xq);
+    float *s_xd = reinterpret_cast<float *>(sm + P.o_xd);
+    float *s_xs = reinterpret_cast<float *>(sm + P.o_xs);
+    JobX *s_jobs = reinterpret_cast<JobX *>(sm + P.o_jobs);
+    int *s_stok = reinterpret_cast<int *>(sm + P.o_stok);
+    float *s_sw = reinterpret_cast<float *>(sm + P.o_sw);
+    int8_t *s_hq = reinterpret_cast<int8_t *>(sm + P.o_hq);
+    float *s_hd = reinterpret_cast<float *>(sm + P.o_hd);
+    float *s_hs = reinterpret_cast<float *>(sm + P.o_hs);
+    float *s_gu = reinterpret_cast<float *>(sm + P.o_gu);    // [2][16][16] gate / up sums
+    float *s_h = reinterpret_cast<float *>(sm + P.o_h);      // [32][16] one block of h
+    float *s_acc = reinterpret_cast<float *>(sm + P.o_acc);  // [16][T] down sums of a unit
+    int *s_misc = reinterpret_cast<int *>(sm + P.o_misc);    // [0] jobs [2] timeout
+    // prologue scratch inside the (still unused) stage ring
+    int *s_cnt = reinterpret_cast<int *>(sm);                // [E]
+    int *s_off = s_cnt + E;                                  // [E]
+    uint32_t *s_bits = reinterpret_cast<uint32_t *>(s_off + E);   // [32]
+    int *s_wbase = reinterpret_cast<int *>(s_bits + 32);     // [32]
+    int *s_ids = s_wbase + 32;                               // [T*k]
+    float *s_wt = reinterpret_cast<float *>(s_ids + T * k);  // [T*k]
+
+    ptx::grid_dependency_wait();
+    ptx::launch_dependents();
+
+    if (tid == 0) {
+        for (int s = 0; s < P.nstages; s++) {
+            ptx::mbar_init(&full[s], 1);
+            ptx::mbar_init(&empty[s], kCW);
+        }
+        ptx::fence_barrier_init();
+        s_misc[2] = 0;
+    }
+    for (int e = tid; e < E; e += kThreads) s_cnt[e] = 0;
+    if (tid < 32) s_bits[tid] = 0;
+    // ---- a2 on warps 0..T-1 (T <= 4), a1 on the rest, at the same time
+    const int topk_warps = T <= 4 ? T : 0;
+    if (warp < topk_warps) {
+        const float *row = P.logits + (size_t)warp * E;
+        uint32_t *st = cta0 ? status : nullptr;
+        if (E <= 256) warp_topk_reg<8>(row, E, k, s_ids + warp * k, s_wt + warp * k, st);
+        else if (E <= 512) warp_topk_reg<16>(row, E, k, s_ids + warp * k, s_wt + warp * k, st);
+        else warp_topk_reg<32>(row, E, k, s_ids + warp * k, s_wt + warp * k, st);
+    } else {
+        const int nxb = T * nbH;
+        const int qt = tid - topk_warps * 32, nq = kThreads - topk_warps * 32;
+        const int groups = nq / 8, g0 = qt >> 3, sub = qt & 7;
+        for (int b0 = 0; b0 < nxb; b0 += groups * 4) {
+            float4 v[4];
+#pragma unroll
+            for (int u = 0; u < 4; u++) {       // four loads in flight per lane
+                const int blk = b0 + g0 + u * groups;
+                v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (blk < nxb) v[u] = __ldg(reinterpret_cast<const float4 *>(P.x + (size_t)blk * 32) + sub);
+            }
+#pragma unroll
+            for (int u = 0; u < 4; u++) {
+                const int blk = b0 + g0 + u * groups;
+                const bool act = blk < nxb;
+                const int b = act ? blk : 0;
+                uint16_t d16 = 0, s16 = 0;
+                float dsum = 0.f;
+                q8_1_block8(v[u], act, sub, s_xq + b * 32, &d16, &s16, &dsum, cta0 ? status : nullptr);
+                if (act && sub == 0) {
+                    s_xd[b] = half_bits_to_float(d16);
+                    s_xs[b] = dsum;
+                    if (cta0) {
+                        reinterpret_cast<uint16_t *>(ws + L.xd)[b] = d16;
+                        reinterpret_cast<uint16_t *>(ws + L.xs)[b] = s16;
+                        reinterpret_cast<float *>(ws + L.xsum)[b] = dsum;
+                    }
+                }
+            }
+        }
+    }
+    if (topk_warps == 0) {       // larger batches: selection after quantization
+        __syncthreads();
+        for (int t = warp; t < T; t += kCW + 1) {
+            const float *row = P.logits + (size_t)t * E;
+            uint32_t *st = cta0 ? status : nullptr;
+            if (E <= 256) warp_topk_reg<8>(row, E, k, s_ids + t * k, s_wt + t * k, st);
+            else if (E <= 512) warp_topk_reg<16>(row, E, k, s_ids + t * k, s_wt + t * k, st);
+            else warp_topk_reg<32>(row, E, k, s_ids + t * k, s_wt + t * k, st);
+        }
+    }
+    __syncthreads();
+    // ---- a3: counts and an expert bitmap, then one warp builds offsets and jobs
+    const int A = T * k;
+    for (int a = tid; a < A; a += kThreads) {
+        const int e = s_ids[a];
+        atomicAdd(&s_cnt[e], 1);
+        atomicOr(&s_bits[e >> 5], 1u << (e & 31));
+    }
+    if (cta0) {
+        for (int i = tid; i < T * H / 16; i += kThreads)
+            reinterpret_cast<int4 *>(ws + L.xq)[i] = reinterpret_cast<const int4 *>(s_xq)[i];
+        for (int a = tid; a < A; a += kThreads) {
+            reinterpret_cast<int32_t *>(ws + L.ids)[a] = s_ids[a];
+            reinterpret_cast<float *>(ws + L.w)[a] = s_wt[a];
+        }
+    }
+    __syncthreads();
+    if (warp == 0) {
+        const int nwords = (E + 31) / 32;
+        const uint32_t word = lane < nwords ? s_bits[lane] : 0u;
+        int csum = 0;
+        for (uint32_t w = word; w; w &= w - 1) csum += s_cnt[lane * 32 + __ffs(w) - 1];
+        int jinc = __popc(word), cinc = csum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int a = __shfl_up_sync(kFullMask, jinc, o), b = __shfl_up_sync(kFullMask, cinc, o);
+            if (lane >= o) {
+                jinc += a;
+                cinc += b;
+            }
+        }
+        int jb = jinc - __popc(word), cb = cinc - csum;
+        s_wbase[lane] = cb;
+        for (uint32_t w = word; w; w &= w - 1) {
+            const int e = lane * 32 + __ffs(w) - 1;
+            const int cnt = s_cnt[e];
+            JobX &J = s_jobs[jb++];
+            J.expert = e;
+            J.slot0 = cb;
+            J.n = cnt;
+            J.shared = 0;
+            s_off[e] = cb;
+            cb += cnt;
+        }
+        const int n_routed = __shfl_sync(kFullMask, jinc, 31);
+        if (lane == 0) {
+            if (P.shared) {
+                JobX &J = s_jobs[n_routed];
+                J.expert = E;
+                J.slot0 = A;
+                J.n = T;
+                J.shared = 1;
+            }
+            s_misc[0] = n_routed + (P.shared ? 1 : 0);
+        }
+    }
+    __syncthreads();
+    const int U = s_misc[0];
+    for (int a = tid; a < A; a += kThreads) {
+        const int e = s_ids[a];
+        int rank = 0;
+        for (int b = 0; b < a; b++) rank += s_ids[b] == e;
+        const int slot = s_off[e] + rank;
+        s_stok[slot] = a / k;
+        s_sw[slot] = s_wt[a];
+        if (cta0) {
+            reinterpret_cast<int32_t *>(ws + L.perm)[slot] = a;
+            reinterpret_cast<int32_t *>(ws + L.inv_perm)[a] = slot;
+        }
+    }
+    for (int t = tid; t < T; t += kThreads) {
+        s_stok[A + t] = t;
+        s_sw[A + t] = 1.0f;
+    }
+    for (int u = tid; u < U; u += kThreads) {
+        JobX &J = s_jobs[u];
+        const ExpertDev &ex = P.experts[J.expert];
+        J.m[0] = ex.m[0];
+        J.m[1] = ex.m[1];
+        J.m[2] = ex.m[2];
+        J.stride[0] = ex.stride[0];
+        J.stride[1] = ex.stride[1];
+        J.stride[2] = ex.stride[2];
+        J.fmt = ex.fmt;
+    }
+    if (cta0) {
+        for (int e = tid; e < E; e += kThreads) {
+            reinterpret_cast<int32_t *>(ws + L.counts)[e] = s_cnt[e];
+            const uint32_t below = s_bits[e >> 5] & ((1u << (e & 31)) - 1u);
+            int off = s_wbase[e >> 5];
+            for (uint32_t w = below; w; w &= w - 1) off += s_cnt[(e & ~31) + __ffs(w) - 1];
+            reinterpret_cast<int32_t *>(ws + L.offsets)[e] = off;
+        }
+        if (tid == 0) reinterpret_cast<int32_t *>(ws + L.offsets)[E] = A;
+    }
+    __syncthreads();
+    if (cta0) {
+        for (int u = tid; u < U; u += kThreads) {
+            const JobX &J = s_jobs[u];
+            reinterpret_cast<Job *>(ws + L.jobs)[u] = Job{J.expert, J.slot0, J.n, J.shared};
+        }
+        if (tid == 0) *reinterpret_cast<int32_t *>(ws + L.njobs) = U;
+    }
+    // the prologue scratch in the stage ring is dead from here on
+
+    // ---- partition
+    const int G = gridDim.x, cta = blockIdx.x;
+    const int nb32 = F / 32;
+    const int n_blk = U * nb32;
+    const int my_blocks = n_blk / G + (cta < n_blk % G ? 1 : 0);
+    double gu_bytes = 0.0, row_bytes = 0.0;
+    for (int u = 0; u < U; u++) {
+        gu_bytes += 32.0 * nb32 * (double)(s_jobs[u].stride[0] + s_jobs[u].stride[1]);
+        row_bytes += (double)s_jobs[u].stride[2];
+    }
+    const double blk_bytes = n_blk ? gu_bytes / n_blk : 0.0;
+    const int i_lo = down_bound(cta, G, H, n_blk, blk_bytes, row_bytes);
+    const int i_hi = cta == G - 1 ? H : down_bound(cta + 1, G, H, n_blk, blk_bytes, row_bytes);
+    const int hb = P.hpad / 32;
+
+    if (warp == kCW) {
+        // ---------------------------------------------------------------- producer
+        if (lane == 0) {
+            const uint64_t pol = ptx::policy_evict_first();
+            int s = 0;
+            uint32_t ph = 0;
+            bool ok = true;
+            auto acquire = [&](int &st) -> bool {
+                if (!ptx::mbar_wait_bounded(&empty[s], ph ^ 1u, kWaitNs)) return false;
+                st = s;
+                if (++s == P.nstages) {
+                    s = 0;
+                    ph ^= 1u;
+                }
+                return true;
+            };
+            for (int mb = 0; mb < my_blocks && ok; mb++) {
+                const int blk = cta + mb * G;
+                const int ju = blk / nb32, b = blk % nb32;
+                const JobX &J = s_jobs[ju];
+                for (int half = 0; half < 2 && ok; half++) {
+                    const int r0 = 32 * b + 16 * half;
+                    const uint32_t b0 = 16u * J.stride[0], b1 = 16u * J.stride[1];
+                    int st;
+                    if (!(ok = acquire(st))) break;
+                    meta[st] = StageMeta{ST_GU, ju, r0, 16, 0, 0, 0, 0};
+                    uint8_t *dst = sm + (size_t)st * P.stage_bytes;
+                    ptx::mbar_arrive_expect_tx(&full[st], b0 + b1);
+                    ptx::bulk_g2s(dst, J.m[0] + (size_t)r0 * J.stride[0], b0, &full[st], pol);
+                    ptx::bulk_g2s(dst + b0, J.m[1] + (size_t)r0 * J.stride[1], b1, &full[st], pol);
+                }
+            }
+            for (int i = i_lo; i < i_hi && ok;) {
+                const int rows = min(kDownRows, i_hi - i);
+                int j = 0;
+                while (j < U && ok) {
+                    const int j0 = j;
+                    uint32_t bytes = 0;
+                    while (j < U) {
+                        const uint32_t b = (uint32_t)rows * s_jobs[j].stride[2];
+                        if (j > j0 && bytes + b > (uint32_t)P.stage_bytes) break;
+                        bytes += b;
+                        j++;
+                    }
+                    int st;
+                    if (!(ok = acquire(st))) break;
+                    meta[st] = StageMeta{ST_DOWN, i, rows, j0, j, j == U ? 1 : 0, 0, 0};
+                    uint8_t *dst = sm + (size_t)st * P.stage_bytes;
+                    ptx::mbar_arrive_expect_tx(&full[st], bytes);
+                    uint32_t off = 0;
+                    for (int jj = j0; jj < j; jj++) {
+                        const JobX &J = s_jobs[jj];
+                        const uint32_t b = (uint32_t)rows * J.stride[2];
+                        ptx::bulk_g2s(dst + off, J.m[2] + (size_t)i * J.stride[2], b, &full[st], pol);
+                        off += b;
+                    }
+                }
+                i += rows;
+            }
+            int st;
+            if (ok && acquire(st)) {
+                meta[st] = StageMeta{ST_END, 0, 0, 0, 0, 0, 0, 0};
+                ptx::mbar_arrive(&full[st]);
+            } else {
+                set_status(status, MOE_ERR_TIMEOUT);
+            }
+        }
+    } else {
+        // ---------------------------------------------------------------- consumers
+        const int ctid = tid;                 // 0..255
+        int s = 0;
+        uint32_t ph = 0;
+        bool gu_done = false, have_h = false, skip_down = false;
+        int done_blocks = 0;
+        int8_t *g_hq = reinterpret_cast<int8_t *>(ws + L.hq);
+        uint16_t *g_hd = reinterpret_cast<uint16_t *>(ws + L.hd);
+        uint16_t *g_hs = reinterpret_cast<uint16_t *>(ws + L.hs);
+        float *g_hsum = reinterpret_cast<float *>(ws + L.hsum);
+        float *g_h = reinterpret_cast<float *>(ws + L.h);
+        while (true) {
+            if (!ptx::mbar_wait_bounded(&full[s], ph, kWaitNs)) {
+                if (lane == 0) set_status(status, MOE_ERR_TIMEOUT);
+                break;
+            }
+            const StageMeta m = meta[s];
+            if (m.kind != ST_GU && !gu_done) {
+                // publish this CTA's Q8_1(h) blocks
+                gu_done = true;
+                ptx::named_barrier(1, kCW * 32);
+                if (ctid == 0 && done_blocks > 0) {
+                    __threadfence();
+                    atomicAdd(&ctr[1], (uint32_t)done_blocks);
+                }
+            }
+            if (m.kind == ST_END) break;
+            const uint8_t *stage = sm + (size_t)s * P.stage_bytes;
+            if (m.kind == ST_GU) {
+                const int ju = m.a, r0 = m.b;
+                const JobX &J = s_jobs[ju];
+                const int which = warp >> 2, rg = (warp & 3) * kRG;   // warps 0-3 gate, 4-7 up
+                for (int t0 = 0; t0 < J.n; t0 += NT) {
+                    const int n = min(NT, J.n - t0);
+                    int act[NT];
+#pragma unroll
+                    for (int t = 0; t < NT; t++) act[t] = t < n ? s_stok[J.slot0 + t0 + t] : 0;
+                    float acc[kRG][NT];
+#pragma unroll
+                    for (int r = 0; r < kRG; r++)
+#pragma unroll
+                        for (int t = 0; t < NT; t++) acc[r][t] = 0.f;
+                    const uint8_t *base = stage + (which ? 16u * J.stride[0] : 0u) +
+                                          (size_t)rg * J.stride[which];
+                    rows_dot<NT, kRG>(J.fmt, base, J.stride[which], kRG, H, s_xq, s_xd, s_xs, H,
+                                      act, n, acc);
+#pragma unroll
+                    for (int r = 0; r < kRG; r++)
+#pragma unroll
+                        for (int t = 0; t < NT; t++) {
+                            const float v = warp_sum(acc[r][t]);
+                            if (lane == 0 && t < n) s_gu[(which * 16 + rg + r) * 16 + t0 + t] = v;
+                        }
+                }
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(&empty[s]);
+                ptx::named_barrier(1, kCW * 32);
+                const int hrow0 = r0 & 31;   // 0 or 16 inside the block
+                for (int i = ctid; i < 16 * J.n; i += kCW * 32) {
+                    const int rr = i / J.n, t = i % J.n;
+                    s_h[(hrow0 + rr) * 16 + t] =
+                        silu_mul(s_gu[rr * 16 + t], s_gu[(16 + rr) * 16 + t]);
+                }
+                ptx::named_barrier(1, kCW * 32);
+                if (hrow0 == 16) {   // the block is complete: Q8_1 of its 32 rows, per slot
+                    const int b = r0 / 32;
+                    for (int t = warp; t < J.n; t += kCW) {
+                        const int slot = J.slot0 + t;
+                        const float v = s_h[lane * 16 + t];
+                        g_h[(size_t)slot * F + 32 * b + lane] = v;
+                        bool fin;
+                        uint16_t d16, s16;
+                        float dsum;
+                        const int q = q8_1_lane(v, fin, d16, s16, dsum);
+                        g_hq[(size_t)slot * P.hpad + 32 * b + lane] = (int8_t)q;
+                        if (lane == 0) {
+                            g_hd[(size_t)slot * hb + b] = d16;
+                            g_hs[(size_t)slot * hb + b] = s16;
+                            g_hsum[(size_t)slot * hb + b] = dsum;
+                            if (!fin) set_status(status, MOE_ERR_NONFINITE);
+                        }
+                        if (b == nb32 - 1) {   // zero the padded tail [F, hpad) of this slot
+                            for (int z = F + lane; z < P.hpad; z += 32) g_hq[(size_t)slot * P.hpad + z] = 0;
+                            for (int z = nb32 + lane; z < hb; z += 32) {
+                                g_hd[(size_t)slot * hb + z] = 0;
+                                g_hs[(size_t)slot * hb + z] = 0;
+                                g_hsum[(size_t)slot * hb + z] = 0.f;
+                            }
+                        }
+                    }
+                    done_blocks++;
+                    ptx::named_barrier(1, kCW * 32);   // s_h is rewritten by the next block
+                }
+            } else {   // ST_DOWN
+                if (!have_h) {
+                    if (ctid == 0) {
+                        const uint64_t t0 = ptx::globaltimer();
+                        int to = 0;
+                        while (ptx::ld_acquire_u32(&ctr[1]) < (uint32_t)n_blk) {
+                            if (ptx::globaltimer() - t0 > kWaitNs) {
+                                to = 1;
+                                break;
+                            }
+                            __nanosleep(32);
+                        }
+                        s_misc[2] = to;
+                        if (to) set_status(status, MOE_ERR_TIMEOUT);
+                    }
+                    ptx::named_barrier(1, kCW * 32);
+                    skip_down = s_misc[2] != 0;
+                    for (int i = ctid; i < P.slots * P.hpad / 16; i += kCW * 32)
+                        reinterpret_cast<int4 *>(s_hq)[i] = ptx::ld_cg_v4(g_hq + (size_t)i * 16);
+                    for (int i = ctid; i < P.slots * hb; i += kCW * 32) {
+                        s_hd[i] = half_bits_to_float(__ldcg(g_hd + i));
+                        s_hs[i] = __ldcg(g_hsum + i);
+                    }
+                    ptx::named_barrier(1, kCW * 32);
+                    have_h = true;
+                }
+                const int i0 = m.a, rows = m.b;
+                if (m.c == 0) {                 // first stage of a down unit: clear the sums
+                    for (int i = ctid; i < kDownRows * T; i += kCW * 32) s_acc[i] = 0.f;
+                    ptx::named_barrier(1, kCW * 32);
+                }
+                const int rw = warp * kRD;
+                if (!skip_down && rw < rows) {
+                    uint32_t off = 0;
+                    for (int ju = m.c; ju < m.d; ju++) {
+                        const JobX &J = s_jobs[ju];
+                        const int Kd = J.fmt == MOE_FMT_Q8_0 ? ((F + 31) / 32) * 32 : P.hpad;
+                        const uint8_t *base = stage + off + (size_t)rw * J.stride[2];
+                        off += (uint32_t)rows * J.stride[2];
+                        for (int t0 = 0; t0 < J.n; t0 += NT) {
+                            const int n = min(NT, J.n - t0);
+                            int act[NT];
+#pragma unroll
+                            for (int t = 0; t < NT; t++) act[t] = t < n ? J.slot0 + t0 + t : 0;
+                            float acc[kRD][NT];
+#pragma unroll
+                            for (int r = 0; r < kRD; r++)
+#pragma unroll
+                                for (int t = 0; t < NT; t++) acc[r][t] = 0.f;
+                            rows_dot<NT, kRD>(J.fmt, base, J.stride[2], min(kRD, rows - rw), Kd,
+                                              s_hq, s_hd, s_hs, P.hpad, act, n, acc);
+#pragma unroll
+                            for (int r = 0; r < kRD; r++)
+#pragma unroll
+                                for (int t = 0; t < NT; t++) {
+                                    const float v = warp_sum(acc[r][t]);
+                                    if (lane == 0 && t < n && rw + r < rows) {
+                                        const int slot = J.slot0 + t0 + t;
+                                        s_acc[(rw + r) * T + s_stok[slot]] += s_sw[slot] * v;
+                                    }
+                                }
+                        }
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(&empty[s]);
+                if (m.e) {                      // last stage of the unit: write the outputs
+                    ptx::named_barrier(1, kCW * 32);
+                    if (!skip_down)
+                        for (int i = ctid; i < rows * T; i += kCW * 32) {
+                            const int r = i / T, t = i % T;
+                            P.out[(size_t)t * H + i0 + r] = s_acc[r * T + t];
+                        }
+                    ptx::named_barrier(1, kCW * 32);
+                }
+            }
+            if (++s == P.nstages) {
+                s = 0;
+                ph ^= 1u;
+            }
+        }
+    }
+    __syncthreads();
+    if (tid == 0) {
+        __threadfence();
+        if (atomicAdd(&ctr[2], 1u) == gridDim.x - 1) {
+            ctr[1] = 0;
+            ctr[2] = 0;
+            __threadfence();
+        }
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_decode_fused(const FfnArgs &a, int E, int shared, const float *x,
+                                const float *logits, uint8_t *ws, const WsLayout &L,
+                                size_t sync_off, size_t blkcnt_off, bool pdl, cudaStream_t st,
+                                bool *taken) {
+    (void)sync_off;
+    (void)blkcnt_off;
+    *taken = false;
+    if (a.T > kDecodeMaxT || E > 1024 || a.T * a.k > kDecodeMaxT * kMaxK || a.F % 32) return cudaSuccess;
+    int dev = 0, nsm = 0, cap = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return err;
+    if ((err = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return err;
+    if ((err = cudaDeviceGetAttribute(&cap, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess)
+        return err;
+    const int max_s01 = a.max_stride01, max_s2 = a.max_stride2;
+    if (max_s01 <= 0 || max_s2 <= 0 || 2 * kUnitPairs * max_s01 > 96 * 1024 ||
+        kDownRows * max_s2 > 96 * 1024)
+        return cudaSuccess;   // rows too wide for the ring: not taken
+    DecParams P{};
+    P.experts = a.experts;
+    P.x = x;
+    P.logits = logits;
+    P.out = a.out;
+    P.ws = ws;
+    P.L = L;
+    P.T = a.T;
+    P.H = a.H;
+    P.F = a.F;
+    P.E = E;
+    P.k = a.k;
+    P.shared = shared;
+    P.hpad = a.hpad;
+    P.max_jobs = a.max_jobs;
+    P.slots = a.T * a.k + a.T;
+    auto al = [](int v, int q) { return (v + q - 1) / q * q; };
+    P.stage_bytes = al(std::max(2 * kUnitPairs * max_s01, kDownRows * max_s2), 1024);
+    const int slots = P.slots;
+    const int sizes[] = {
+        2 * 16 * 8,                                  // barriers (<= 16 stages)
+        16 * (int)sizeof(StageMeta),                 // stage meta
+        al(a.T * a.H, 128),                          // xq
+        al(a.T * (a.H / 32) * 4, 16),                // xd
+        al(a.T * (a.H / 32) * 4, 16),                // xs
+        al(a.max_jobs * (int)sizeof(JobX), 16),      // jobs
+        al(slots * 4, 16),                           // slot tokens
+        al(slots * 4, 16),                           // slot weights
+        al(slots * a.hpad, 128),                     // Q8_1(h) q
+        al(slots * (a.hpad / 32) * 4, 16),           // Q8_1(h) d
+        al(slots * (a.hpad / 32) * 4, 16),           // Q8_1(h) xd*sum(q)
+        2 * 16 * 16 * 4,                             // gate / up sums [2][16][16]
+        32 * 16 * 4,                                 // one block of h [32][16]
+        al(kDownRows * a.T * 4, 16),                 // down sums [16][T]
+        64};                                         // misc
+    int fixed = 0;
+    for (int v : sizes) fixed += v;
+    int nst = (cap - fixed - 1024) / P.stage_bytes;
+    if (nst > 16) nst = 16;
+    const int scratch = (2 * E + 64 + 2 * a.T * a.k) * 4;   // prologue scratch in the ring
+    if (nst < 2 || nst * P.stage_bytes < scratch) return cudaSuccess;
+    P.nstages = nst;
+    int o = nst * P.stage_bytes;
+    int *offs[] = {&P.o_bar, &P.o_meta, &P.o_xq, &P.o_xd, &P.o_xs, &P.o_jobs, &P.o_stok,
+                   &P.o_sw, &P.o_hq, &P.o_hd, &P.o_hs, &P.o_gu, &P.o_h, &P.o_acc, &P.o_misc};
+    for (int i = 0; i < 15; i++) {
+        *offs[i] = o;
+        o += sizes[i];
+    }
+    P.smem_bytes = o;
+    if (o > cap) return cudaSuccess;
+
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(nsm);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = (size_t)P.smem_bytes;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    if (a.T <= 1) {
+        if ((err = ensure_smem(k_decode_fused<1>, (size_t)P.smem_bytes)) != cudaSuccess) return err;
+        err = cudaLaunchKernelEx(&cfg, k_decode_fused<1>, P);
+    } else {
+        if ((err = ensure_smem(k_decode_fused<4>, (size_t)P.smem_bytes)) != cudaSuccess) return err;
+        err = cudaLaunchKernelEx(&cfg, k_decode_fused<4>, P);
+    }
+    if (err != cudaSuccess) return err;
+    note_launches(1);
+    *taken = true;
+    return cudaSuccess;
+}
+
+}  // namespace moe

@@ -19,6 +19,7 @@ struct moe_arena {
     int H, F, E, shared;      // shared: index of the shared expert (== E) or -1
     int n;                    // descriptors (E or E + 1)
     int fmt_mask;             // bit f set when some expert uses format f
+    int max_stride01, max_stride2;
     moe::ExpertDev *d_experts;
     std::vector<moe_expert_desc> descs;
 };
@@ -62,6 +63,8 @@ WsLayout ws_layout(const moe_arena *A, int T, int k, uint32_t flags) {
     L.max_jobs = std::min(E, T * k) + shared;
     L.n_chunks = (T + kChunk - 1) / kChunk;
     L.status = take(sizeof(uint32_t));
+    L.sync = take(4 * sizeof(uint32_t));                                  // fused-decode counters
+    L.blkcnt = take(sizeof(uint32_t) * (size_t)L.max_jobs * (F / 32));    // rows done per h block
     L.njobs = take(sizeof(int32_t));
     L.jobs = take(sizeof(Job) * (size_t)L.max_jobs);
     L.xq = take((size_t)T * H);
@@ -80,7 +83,8 @@ WsLayout ws_layout(const moe_arena *A, int T, int k, uint32_t flags) {
     L.hd = take((size_t)L.slots * (L.hpad / 32) * 2);
     L.hs = take((size_t)L.slots * (L.hpad / 32) * 2);
     L.hsum = take((size_t)L.slots * (L.hpad / 32) * 4);
-    L.h = (flags & MOE_F_KEEP_H) ? take((size_t)L.slots * F * 4) : 0;
+    L.h = take((size_t)L.slots * F * 4);
+    (void)flags;
     L.y = (flags & MOE_F_DETERMINISTIC) ? take((size_t)L.slots * H * 4) : 0;
     L.total = p;
     return L;
@@ -123,6 +127,7 @@ moe_status moe_arena_create(const void *d_arena, size_t arena_bytes, int hidden,
     const int n = n_experts + (shared_expert >= 0 ? 1 : 0);
     std::vector<ExpertDev> dev(n);
     int fmt_mask = 0;
+    uint64_t ms01 = 0, ms2 = 0;
     for (int e = 0; e < n; e++) {
         const moe_expert_desc &d = host_descs[e];
         if (d.fmt < 0 || d.fmt > 2 || d.reserved != 0) return MOE_ERR_INVALID_ARG;
@@ -141,6 +146,8 @@ moe_status moe_arena_create(const void *d_arena, size_t arena_bytes, int hidden,
         }
         dev[e].fmt = d.fmt;
         dev[e].pad = 0;
+        ms01 = std::max(ms01, std::max(d.stride[0], d.stride[1]));
+        ms2 = std::max(ms2, d.stride[2]);
         fmt_mask |= 1 << d.fmt;
     }
     moe_arena *A = new (std::nothrow) moe_arena();
@@ -153,6 +160,8 @@ moe_status moe_arena_create(const void *d_arena, size_t arena_bytes, int hidden,
     A->shared = shared_expert;
     A->n = n;
     A->fmt_mask = fmt_mask;
+    A->max_stride01 = (int)ms01;
+    A->max_stride2 = (int)ms2;
     A->descs.assign(host_descs, host_descs + n);
     if (cudaMalloc(&A->d_experts, sizeof(ExpertDev) * n) != cudaSuccess ||
         cudaMemcpy(A->d_experts, dev.data(), sizeof(ExpertDev) * n, cudaMemcpyHostToDevice) !=
@@ -302,6 +311,26 @@ moe_status moe_forward(const moe_arena *arena, const float *d_x, const float *d_
     Job *jobs = reinterpret_cast<Job *>(ws + L.jobs);
     int32_t *njobs = reinterpret_cast<int32_t *>(ws + L.njobs);
 
+    if (decode && T <= kDecodeMaxT) {
+        FfnArgs a{};
+        a.experts = arena->d_experts;
+        a.out = d_out;
+        a.status = status;
+        a.T = T;
+        a.k = k;
+        a.H = H;
+        a.F = arena->F;
+        a.hpad = L.hpad;
+        a.max_jobs = L.max_jobs;
+        a.fmt_mask = arena->fmt_mask;
+        a.max_stride01 = arena->max_stride01;
+        a.max_stride2 = arena->max_stride2;
+        bool taken = false;
+        cudaError_t e = launch_decode_fused(a, E, shared, d_x, d_logits, ws, L, L.sync, L.blkcnt,
+                                            true, st, &taken);
+        if (e != cudaSuccess) return MOE_ERR_CUDA;
+        if (taken) return MOE_OK;
+    }
     // a1-a3
     const bool small_route = T <= kDecodeMaxT && T * k <= kDecodeMaxT * kMaxK &&
                              ((size_t)T * E + E) * 4 <= 96 * 1024;
@@ -332,7 +361,7 @@ moe_status moe_forward(const moe_arena *arena, const float *d_x, const float *d_
     a.hd = reinterpret_cast<uint16_t *>(ws + L.hd);
     a.hs = reinterpret_cast<uint16_t *>(ws + L.hs);
     a.hsum = reinterpret_cast<float *>(ws + L.hsum);
-    a.h = (flags & MOE_F_KEEP_H) ? reinterpret_cast<float *>(ws + L.h) : nullptr;
+    a.h = reinterpret_cast<float *>(ws + L.h);
     a.y = (flags & MOE_F_DETERMINISTIC) ? reinterpret_cast<float *>(ws + L.y) : nullptr;
     a.out = d_out;
     a.status = status;
@@ -343,6 +372,8 @@ moe_status moe_forward(const moe_arena *arena, const float *d_x, const float *d_
     a.hpad = L.hpad;
     a.max_jobs = L.max_jobs;
     a.fmt_mask = arena->fmt_mask;
+    a.max_stride01 = arena->max_stride01;
+    a.max_stride2 = arena->max_stride2;
 
     // a4 + a5
     err = launch_gateup_gemv(a, st);

@@ -59,8 +59,8 @@ struct moe_arena_impl;
 
 // Offsets (bytes) of everything moe_forward keeps in its workspace.
 struct WsLayout {
-    size_t status, njobs, jobs, xq, xd, xs, xsum, ids, w, counts, offsets, perm, inv_perm,
-        chunk_counts, chunk_base, hq, hd, hs, hsum, h, y, total;
+    size_t status, sync, blkcnt, njobs, jobs, xq, xd, xs, xsum, ids, w, counts, offsets, perm,
+        inv_perm, chunk_counts, chunk_base, hq, hd, hs, hsum, h, y, total;
     int slots, hpad, max_jobs, n_chunks;
 };
 
@@ -139,12 +139,20 @@ struct FfnArgs {
     float *out;
     uint32_t *status;
     int T, k, H, F, hpad, max_jobs, fmt_mask;
+    int max_stride01, max_stride2;   // largest gate/up and down row strides in the arena
 };
 
 cudaError_t launch_gateup_gemv(const FfnArgs &a, cudaStream_t st);
 cudaError_t launch_down_decode(const FfnArgs &a, cudaStream_t st);
 cudaError_t launch_down_grouped(const FfnArgs &a, bool deterministic, cudaStream_t st);
 cudaError_t launch_combine(const FfnArgs &a, bool shared, cudaStream_t st);
+
+// The whole layer for small batches in one persistent kernel (k_decode.cu).  Sets *taken to
+// false, enqueueing nothing, when the shape does not fit its shared-memory plan.
+cudaError_t launch_decode_fused(const FfnArgs &a, int E, int shared, const float *x,
+                                const float *logits, uint8_t *ws, const WsLayout &L,
+                                size_t sync_off, size_t blkcnt_off, bool pdl, cudaStream_t st,
+                                bool *taken);
 
 cudaError_t launch_dequant(const uint8_t *m, int fmt, int rows, int nblocks, int stride,
                            float *out, cudaStream_t st);

@@ -224,8 +224,10 @@ def test_layer_prefill_full_size_sampled(torch, name):
     x, logits = inputs(w, 0)
     ids, _, _ = oracle.topk(logits, w.k)
     counts = np.bincount(ids.ravel(), minlength=w.n_experts)
-    if name == "mixed_prefill":   # the Zipf(1.3) skew the workload asks for
-        assert counts.max() > 1000 and (counts < 8).sum() > 100
+    if name == "mixed_prefill":
+        # Zipf(1.3) popularity sampled k at a time without replacement (Gumbel top-k): a few
+        # experts take > 1000 tokens, a long tail takes only a handful
+        assert (counts > 1000).sum() >= 3 and (counts < 8).sum() >= 5 and (counts < 16).sum() >= 50
     _check_layer(torch, w, 0, x, logits, tokens=_sample_tokens(w.tokens, ids))
 
 
@@ -298,3 +300,10 @@ def test_host_errors_enqueue_nothing(torch):
     torch.cuda.synchronize()
     assert (out == 7.0).all()
     L.close()
+
+
+def test_decode_large_expert_count_uses_grouped_kernels(torch):
+    # 2048 experts exceed the fused decode kernel's plan: the three-kernel decode path runs
+    w = synth.Workload("wideE", 70, 256, 256, 2048, 4, 3, True, 1, "normal", sigma=2.0)
+    x, logits = inputs(w, 0)
+    _check_layer(torch, w, 0, x, logits, keep_h=True)
