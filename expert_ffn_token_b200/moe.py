@@ -33,7 +33,7 @@ F_KEEP_H = 8
 EXPORTED = ["moe_arena_create", "moe_arena_destroy", "moe_workspace_size", "moe_quantize_act",
             "moe_route_workspace_size", "moe_route_topk", "moe_forward", "moe_ws_views",
             "moe_read_status", "moe_debug_dequant", "moe_status_string",
-            "moe_kernels_enqueued"]
+            "moe_kernels_enqueued", "moe_forward_noalloc"]
 
 
 class ExpertDesc(ctypes.Structure):
@@ -68,6 +68,7 @@ _lib.moe_forward.argtypes = [_P, _P, _P, _I, _I, _P, _P, _S, _U, _P]
 _lib.moe_ws_views.argtypes = [_P, _P, _I, _I, _U, ctypes.POINTER(WsView)]
 _lib.moe_read_status.argtypes = [_P, _P, _I, ctypes.POINTER(_I)]
 _lib.moe_debug_dequant.argtypes = [_P, _I, _I, _P, _P]
+_lib.moe_forward_noalloc.argtypes = [_P, _P, _P, _I, _I, _P, _P, _P]
 _lib.moe_kernels_enqueued.argtypes = []
 _lib.moe_kernels_enqueued.restype = ctypes.c_uint64
 
@@ -141,6 +142,13 @@ def forward(arena: int, d_x: int, d_logits: int, T: int, k: int, d_out: int, d_w
             ws_bytes: int, flags: int = 0, stream=None) -> None:
     _check(_lib.moe_forward(arena, d_x, d_logits, T, k, d_out, d_ws, ws_bytes, flags, stream),
            "moe_forward")
+
+
+def forward_noalloc(arena: int, d_x: int, d_logits: int, T: int, k: int, d_out: int,
+                    d_status=None, stream=None) -> None:
+    """moe_forward_noalloc: the layer for 1..16 tokens using the library's fixed scratch."""
+    _check(_lib.moe_forward_noalloc(arena, d_x, d_logits, T, k, d_out, d_status, stream),
+           "moe_forward_noalloc")
 
 
 def forward_status(arena, d_x, d_logits, T, k, d_out, d_ws, ws_bytes, flags=0, stream=None) -> int:

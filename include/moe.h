@@ -164,6 +164,21 @@ moe_status moe_read_status(uint32_t *d_status_word, void *stream, int clear,
 moe_status moe_debug_dequant(const moe_arena *arena, int expert, int which, float *d_out,
                              void *stream);
 
+/* moe_forward without any allocation, for batches of 1..16 tokens.  The pages describe no such
+ * call; it exists for callers that may not allocate device memory -- code running under CUDA
+ * graph capture, inference loops with a fixed memory budget, plug-ins whose host framework owns
+ * every allocation.  Instead of a caller workspace it uses a 4 MiB scratch array compiled into
+ * the library (every GPU that loads libmoe.so holds it until the process exits); shapes whose
+ * workspace (moe_workspace_size for T, k, flags 0) exceeds 4 MiB return MOE_ERR_UNSUPPORTED.
+ * It calls no cudaMalloc/cudaFree: it clears the scratch's status word and counters with
+ * cudaMemsetAsync, runs moe_forward on `stream`, and copies the device status word to d_status
+ * (device uint32, may be NULL).  The first call on each device looks up the scratch address;
+ * make that first call before any stream capture.  All calls share the one scratch area, which
+ * keeps the previous call's contents: calls that can overlap on the GPU (different streams,
+ * other threads) race and must be serialised by the caller.                                  */
+moe_status moe_forward_noalloc(const moe_arena *arena, const float *d_x, const float *d_logits,
+                               int T, int k, float *d_out, uint32_t *d_status, void *stream);
+
 /* Number of kernels this library has enqueued (or recorded into a CUDA graph under stream
  * capture) in this process since it was loaded.  Counting a captured forward gives the
  * kernels each replay of that graph launches. */
