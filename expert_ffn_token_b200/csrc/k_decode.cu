@@ -12,17 +12,18 @@
 //     x to Q8_1 in shared memory; one warp then builds counts, offsets, slots and the job list
 //     from an expert bitmap (popc prefix sums), and the chosen experts' descriptors are cached.
 //   partition: the U * F/32 blocks of 32 gate/up rows go round-robin to the CTAs, so every CTA
-//     owns whole Q8_1(h) blocks and quantizes them itself; the H down rows are cut into one
-//     contiguous range per CTA sized so that every CTA streams the same number of bytes.
+//     owns whole Q8_1(h) blocks and quantizes them itself; the H down rows (computed after the
+//     barrier by everyone) are cut into equal contiguous ranges.
 //   pipeline: one producer thread streams the CTA's rows into a ring of shared-memory stages
 //     with bulk async copies (TMA engine, mbarrier byte counts, L2 evict-first) as far ahead
-//     as the ring allows; 8 consumer warps compute from shared memory.
-//   gate/up: a unit is 16 rows of gate and 16 of up; each warp takes 4 rows, each lane a fixed
+//     as the ring allows; 16 consumer warps compute from shared memory.
+//   gate/up: a unit is 16 rows of gate and 16 of up; each warp takes 2 rows, each lane a fixed
 //     set of 16-byte quant chunks (activations loaded once per chunk, reused over the rows);
 //     h = silu(g) * u goes to shared memory and, once the 32-row block is complete, to Q8_1.
 //   down: after every CTA has published its blocks (bounded wait on one counter), all Q8_1(h)
-//     rows are staged in shared memory; warps run over every job's rows and add w * y into
-//     per-row sums; each output element is written once -- deterministic, no output atomics.
+//     rows are staged in shared memory; each warp keeps one or two output rows (16 lanes per
+//     row when a row has <= 16 chunks), runs over every job, weights each slot's product in the
+//     lanes and reduces once per row -- deterministic, each output element written once.
 // Every wait is bounded by %globaltimer and reports MOE_ERR_TIMEOUT instead of hanging.  The
 // down phase waits on the gate/up work of every CTA: the grid is one CTA per SM (all resident
 // together; a programmatically launched successor starts only once every CTA here has
@@ -35,12 +36,11 @@ namespace moe {
 
 namespace {
 
-constexpr int kCW = 8;                       // consumer warps
+constexpr int kCW = 16;                      // consumer warps
 constexpr int kThreads = (kCW + 1) * 32;     // + one producer warp
-constexpr int kRG = 4;                       // gate/up rows per warp per unit
+constexpr int kRG = 2;                       // gate/up rows per warp per unit
 constexpr int kUnitPairs = kRG * kCW / 2;    // 16 gate + 16 up rows per unit
-constexpr int kRD = 2;                       // down rows per warp per unit
-constexpr int kDownRows = kRD * kCW;         // 16 output rows per down unit
+constexpr int kDownRowsMax = 2 * kCW;        // down rows per unit: 1 or 2 per warp
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s: far beyond any legitimate wait
 
 enum { ST_END = 0, ST_GU = 1, ST_DOWN = 2 };
@@ -191,42 +191,77 @@ __device__ __forceinline__ float q80_chunk_dot(const uint8_t *blk, const ActChun
     return d * (a.dl * (float)acc);
 }
 
-// R rows (row r at base + r*stride, r < nrows) of K weights against n <= NT activation rows
-// (row t at q + act[t]*astride): lane-partial sums into acc[R][NT].  Each lane keeps its own
-// chunks p = lane, lane+32, ... and reuses their activations over the R rows.
-template <int NT, int R>
-__device__ __forceinline__ void rows_dot(int fmt, const uint8_t *base, uint32_t stride, int nrows,
-                                         int K, const int8_t *q, const float *d, const float *s,
-                                         int astride, const int *act, int n, float (&acc)[R][NT]) {
+// Format classes the kernel is specialised for: every expert Q4_K, every expert Q5_K, or any.
+enum { FK_Q4K = 0, FK_Q5K = 1, FK_ANY = 2 };
+
+// R packed rows of K weights (rows[r], nullptr = skip) against n <= NT activation rows (row t
+// at q + act[t]*astride).  The lanes of the warp form 32/lpr groups of lpr lanes; the caller
+// gives each group its own rows.  A lane takes chunks p = lane%lpr, +lpr, ...; lane-partial
+// sums go to acc[R][NT].
+template <int NT, int R, int FK>
+__device__ __forceinline__ void rows_dot(int fmt_rt, const uint8_t *const (&rows)[R], int K,
+                                         const int8_t *q, const float *d, const float *s,
+                                         int astride, const int *act, int n, int lpr,
+                                         float (&acc)[R][NT]) {
     const int lane = threadIdx.x & 31;
     const int nchunk = K / 32;
+    const int fmt = FK == FK_Q4K ? MOE_FMT_Q4_K : FK == FK_Q5K ? MOE_FMT_Q5_K : fmt_rt;
     const bool q80 = fmt == MOE_FMT_Q8_0, q5 = fmt == MOE_FMT_Q5_K;
     const int SBB = q5 ? kQ5KBytes : kQ4KBytes;
-    for (int p = lane; p < nchunk; p += 32) {
-        ActChunk a[NT];
-#pragma unroll
-        for (int t = 0; t < NT; t++)
-            if (t < n)
-                a[t] = load_act(q + (size_t)act[t] * astride, d + act[t] * (astride / 32),
-                                s + act[t] * (astride / 32), p, q80);
+    for (int p = lane % lpr; p < nchunk; p += lpr) {
         const int sb = p >> 3, j = p & 7;
         const float mf = (j & 1) ? 0.f : 1.f;
+        // one activation row: keep its chunk in registers across the rows; several: reload
+        // each token's chunk per row from shared memory (saves registers, costs a few loads)
+        ActChunk a0;
+        if (NT == 1) a0 = load_act(q + (size_t)act[0] * astride, d + act[0] * (astride / 32),
+                                   s + act[0] * (astride / 32), p, q80);
 #pragma unroll
         for (int r = 0; r < R; r++) {
-            if (r < nrows) {
-                const uint8_t *row = base + (size_t)r * stride;
-                if (q80) {
+            const uint8_t *row = rows[r];
+            if (!row) continue;
+            if (FK == FK_ANY && q80) {
 #pragma unroll
-                    for (int t = 0; t < NT; t++)
-                        if (t < n) acc[r][t] += q80_chunk_dot(row + (size_t)p * kQ80Bytes, a[t]);
-                } else {
-                    const WChunk w = q5 ? kq_chunk<true>(row + (size_t)sb * SBB, j)
-                                        : kq_chunk<false>(row + (size_t)sb * SBB, j);
+                for (int t = 0; t < NT; t++) {
+                    if (t < n) {
+                        const ActChunk a = NT == 1 ? a0
+                            : load_act(q + (size_t)act[t] * astride, d + act[t] * (astride / 32),
+                                       s + act[t] * (astride / 32), p, true);
+                        acc[r][t] += q80_chunk_dot(row + (size_t)p * kQ80Bytes, a);
+                    }
+                }
+            } else {
+                const WChunk w = (FK == FK_Q5K || (FK == FK_ANY && q5))
+                                     ? kq_chunk<true>(row + (size_t)sb * SBB, j)
+                                     : kq_chunk<false>(row + (size_t)sb * SBB, j);
 #pragma unroll
-                    for (int t = 0; t < NT; t++)
-                        if (t < n) acc[r][t] += kq_chunk_dot(w, a[t], mf);
+                for (int t = 0; t < NT; t++) {
+                    if (t < n) {
+                        const ActChunk a = NT == 1 ? a0
+                            : load_act(q + (size_t)act[t] * astride, d + act[t] * (astride / 32),
+                                       s + act[t] * (astride / 32), p, false);
+                        acc[r][t] += kq_chunk_dot(w, a, mf);
+                    }
                 }
             }
+        }
+    }
+}
+
+// Q8_1 of one block of x held by 8 lanes, into shared memory (and, on CTA 0, the workspace).
+__device__ __noinline__ void quant_x_block(float4 v, bool act, int sub, int b, int8_t *s_xq,
+                                           float *s_xd, float *s_xs, uint16_t *g_xd,
+                                           uint16_t *g_xs, float *g_xsum, uint32_t *status) {
+    uint16_t d16 = 0, s16 = 0;
+    float dsum = 0.f;
+    q8_1_block8(v, act, sub, s_xq + b * 32, &d16, &s16, &dsum, status);
+    if (act && sub == 0) {
+        s_xd[b] = half_bits_to_float(d16);
+        s_xs[b] = dsum;
+        if (g_xd) {
+            g_xd[b] = d16;
+            g_xs[b] = s16;
+            g_xsum[b] = dsum;
         }
     }
 }
@@ -242,7 +277,7 @@ __device__ __forceinline__ float key_value(uint32_t k) {
 // One warp: top-k of a logit row held in registers (VPL values per lane, value e at lane e%32,
 // slot e/32).  Descending logit, ties to the lower id; weights = softmax over the chosen k.
 template <int VPL>
-__device__ __forceinline__ void warp_topk_reg(const float *row, int E, int k, int *ids_out,
+__device__ __noinline__ void warp_topk_reg(const float *row, int E, int k, int *ids_out,
                                               float *w_out, uint32_t *status) {
     const int lane = threadIdx.x & 31;
     uint32_t key[VPL];
@@ -298,8 +333,8 @@ __device__ __forceinline__ void warp_topk_reg(const float *row, int E, int k, in
 }
 
 // Q8_1 of 32 values held one per lane; lane 0 gets d16, s16, dsum.
-__device__ __forceinline__ int q8_1_lane(float v, bool &fin, uint16_t &d16, uint16_t &s16,
-                                         float &dsum) {
+__device__ __noinline__ int q8_1_lane(float v, bool &fin, uint16_t &d16, uint16_t &s16,
+                                      float &dsum) {
     fin = __all_sync(kFullMask, isfinite(v));
     float a = fabsf(v);
 #pragma unroll
@@ -323,83 +358,67 @@ __device__ __forceinline__ int q8_1_lane(float v, bool &fin, uint16_t &d16, uint
     return qi;
 }
 
-// Down-row boundary of CTA c: rows are shared out in proportion to the bytes each CTA still has
-// room for after its gate/up blocks, so that every CTA streams about the same total.
-__device__ __forceinline__ int down_bound(int c, int G, int H, int n_blk, double blk_bytes,
-                                          double row_bytes) {
-    if (c >= G) return H;
-    const int q = n_blk / G, r = n_blk % G;
-    const double total = blk_bytes * n_blk + row_bytes * H;
-    const double target = total / G;
-    const double cap_hi = fmax(0.0, target - (q + 1) * blk_bytes);   // CTAs c < r own q+1 blocks
-    const double cap_lo = fmax(0.0, target - q * blk_bytes);
-    const double ctot = r * cap_hi + (G - r) * cap_lo;
-    if (ctot <= 0.0) return (int)((long long)H * c / G);
-    const double cc = fmin((double)c, (double)r) * cap_hi + fmax(0.0, (double)(c - r)) * cap_lo;
-    return (int)floor(H * (cc / ctot));
-}
+// What a CTA shares between its phases: shared-memory and workspace views, sizes, its share of
+// the work.  Built once by the kernel and passed to the (inlined) phase functions below.
+struct Ctx {
+    int8_t *s_xq;
+    float *s_xd, *s_xs;
+    JobX *s_jobs;
+    int *s_stok;
+    float *s_sw;
+    int8_t *s_hq;
+    float *s_hd, *s_hs, *s_part, *s_h;
+    int *s_misc;             // [0] jobs [2] timeout
+    uint64_t *full, *empty;
+    StageMeta *meta;
+    uint8_t *ring;
+    uint8_t *ws;
+    uint32_t *status, *ctr;  // ctr: [1] blocks published [2] CTAs finished
+    int T, H, F, E, k, U, nb32, n_blk, my_blocks, i_lo, i_hi, hb, down_lpr;
+    bool cta0;
+};
 
-template <int NT>
-__global__ void __launch_bounds__(kThreads, 1) k_decode_fused(const DecParams P) {
-    extern __shared__ __align__(128) uint8_t sm[];
+// a1-a3 for the whole batch (every CTA; CTA 0 also stores the intermediates).
+template <int VPL>
+__device__ __forceinline__ void prologue(const DecParams &P, Ctx &C, uint8_t *sm) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const WsLayout &L = P.L;
     uint8_t *ws = P.ws;
-    uint32_t *status = reinterpret_cast<uint32_t *>(ws + L.status);
-    uint32_t *ctr = reinterpret_cast<uint32_t *>(ws + L.sync);   // [1] blocks_done [2] finished
-    const bool cta0 = blockIdx.x == 0;
-    const int T = P.T, H = P.H, F = P.F, E = P.E, k = P.k;
-    const int nbH = H / 32;
-
-    uint64_t *full = reinterpret_cast<uint64_t *>(sm + P.o_bar);
-    uint64_t *empty = full + P.nstages;
-    StageMeta *meta = reinterpret_cast<StageMeta *>(sm + P.o_meta);
-    int8_t *s_xq = reinterpret_cast<int8_t *>(sm + P.o_xq);
-    float *s_xd = reinterpret_cast<float *>(sm + P.o_xd);
-    float *s_xs = reinterpret_cast<float *>(sm + P.o_xs);
-    JobX *s_jobs = reinterpret_cast<JobX *>(sm + P.o_jobs);
-    int *s_stok = reinterpret_cast<int *>(sm + P.o_stok);
-    float *s_sw = reinterpret_cast<float *>(sm + P.o_sw);
-    int8_t *s_hq = reinterpret_cast<int8_t *>(sm + P.o_hq);
-    float *s_hd = reinterpret_cast<float *>(sm + P.o_hd);
-    float *s_hs = reinterpret_cast<float *>(sm + P.o_hs);
-    float *s_gu = reinterpret_cast<float *>(sm + P.o_gu);    // [2][16][16] gate / up sums
-    float *s_h = reinterpret_cast<float *>(sm + P.o_h);      // [32][16] one block of h
-    float *s_acc = reinterpret_cast<float *>(sm + P.o_acc);  // [16][T] down sums of a unit
-    int *s_misc = reinterpret_cast<int *>(sm + P.o_misc);    // [0] jobs [2] timeout
-    // prologue scratch inside the (still unused) stage ring
+    const int T = P.T, H = P.H, E = P.E, k = P.k;
+    const bool cta0 = C.cta0;
+    uint32_t *status = C.status;
+    // scratch in the (still unused) stage ring
     int *s_cnt = reinterpret_cast<int *>(sm);                // [E]
     int *s_off = s_cnt + E;                                  // [E]
     uint32_t *s_bits = reinterpret_cast<uint32_t *>(s_off + E);   // [32]
     int *s_wbase = reinterpret_cast<int *>(s_bits + 32);     // [32]
     int *s_ids = s_wbase + 32;                               // [T*k]
     float *s_wt = reinterpret_cast<float *>(s_ids + T * k);  // [T*k]
-
-    ptx::grid_dependency_wait();
-    ptx::launch_dependents();
-
-    if (tid == 0) {
-        for (int s = 0; s < P.nstages; s++) {
-            ptx::mbar_init(&full[s], 1);
-            ptx::mbar_init(&empty[s], kCW);
-        }
-        ptx::fence_barrier_init();
-        s_misc[2] = 0;
-    }
+    ExpertDev *s_ex = reinterpret_cast<ExpertDev *>(
+        sm + (((2 * E + 64 + 2 * T * k) * 4 + 15) / 16) * 16);   // [E + shared] descriptors
+#pragma unroll 1
     for (int e = tid; e < E; e += kThreads) s_cnt[e] = 0;
     if (tid < 32) s_bits[tid] = 0;
+    {   // the descriptor table, fetched while the experts are being chosen
+        const int nd = (E + P.shared) * (int)(sizeof(ExpertDev) / 8);
+        const unsigned long long *src = reinterpret_cast<const unsigned long long *>(P.experts);
+        unsigned long long *dst = reinterpret_cast<unsigned long long *>(s_ex);
+#pragma unroll 1
+        for (int i = tid; i < nd; i += kThreads) dst[i] = __ldg(src + i);
+    }
     // ---- a2 on warps 0..T-1 (T <= 4), a1 on the rest, at the same time
     const int topk_warps = T <= 4 ? T : 0;
+    uint16_t *g_xd = cta0 ? reinterpret_cast<uint16_t *>(ws + L.xd) : nullptr;
+    uint16_t *g_xs = reinterpret_cast<uint16_t *>(ws + L.xs);
+    float *g_xsum = reinterpret_cast<float *>(ws + L.xsum);
+    uint32_t *st = cta0 ? status : nullptr;
     if (warp < topk_warps) {
-        const float *row = P.logits + (size_t)warp * E;
-        uint32_t *st = cta0 ? status : nullptr;
-        if (E <= 256) warp_topk_reg<8>(row, E, k, s_ids + warp * k, s_wt + warp * k, st);
-        else if (E <= 512) warp_topk_reg<16>(row, E, k, s_ids + warp * k, s_wt + warp * k, st);
-        else warp_topk_reg<32>(row, E, k, s_ids + warp * k, s_wt + warp * k, st);
+        warp_topk_reg<VPL>(P.logits + (size_t)warp * E, E, k, s_ids + warp * k, s_wt + warp * k, st);
     } else {
-        const int nxb = T * nbH;
+        const int nxb = T * (H / 32);
         const int qt = tid - topk_warps * 32, nq = kThreads - topk_warps * 32;
         const int groups = nq / 8, g0 = qt >> 3, sub = qt & 7;
+#pragma unroll 1
         for (int b0 = 0; b0 < nxb; b0 += groups * 4) {
             float4 v[4];
 #pragma unroll
@@ -412,53 +431,43 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_fused(const DecParams P)
             for (int u = 0; u < 4; u++) {
                 const int blk = b0 + g0 + u * groups;
                 const bool act = blk < nxb;
-                const int b = act ? blk : 0;
-                uint16_t d16 = 0, s16 = 0;
-                float dsum = 0.f;
-                q8_1_block8(v[u], act, sub, s_xq + b * 32, &d16, &s16, &dsum, cta0 ? status : nullptr);
-                if (act && sub == 0) {
-                    s_xd[b] = half_bits_to_float(d16);
-                    s_xs[b] = dsum;
-                    if (cta0) {
-                        reinterpret_cast<uint16_t *>(ws + L.xd)[b] = d16;
-                        reinterpret_cast<uint16_t *>(ws + L.xs)[b] = s16;
-                        reinterpret_cast<float *>(ws + L.xsum)[b] = dsum;
-                    }
-                }
+                quant_x_block(v[u], act, sub, act ? blk : 0, C.s_xq, C.s_xd, C.s_xs, g_xd, g_xs,
+                              g_xsum, st);
             }
         }
     }
     if (topk_warps == 0) {       // larger batches: selection after quantization
         __syncthreads();
-        for (int t = warp; t < T; t += kCW + 1) {
-            const float *row = P.logits + (size_t)t * E;
-            uint32_t *st = cta0 ? status : nullptr;
-            if (E <= 256) warp_topk_reg<8>(row, E, k, s_ids + t * k, s_wt + t * k, st);
-            else if (E <= 512) warp_topk_reg<16>(row, E, k, s_ids + t * k, s_wt + t * k, st);
-            else warp_topk_reg<32>(row, E, k, s_ids + t * k, s_wt + t * k, st);
-        }
+#pragma unroll 1
+        for (int t = warp; t < T; t += kCW + 1)
+            warp_topk_reg<VPL>(P.logits + (size_t)t * E, E, k, s_ids + t * k, s_wt + t * k, st);
     }
     __syncthreads();
     // ---- a3: counts and an expert bitmap, then one warp builds offsets and jobs
     const int A = T * k;
+#pragma unroll 1
     for (int a = tid; a < A; a += kThreads) {
         const int e = s_ids[a];
         atomicAdd(&s_cnt[e], 1);
         atomicOr(&s_bits[e >> 5], 1u << (e & 31));
     }
     if (cta0) {
+#pragma unroll 1
         for (int i = tid; i < T * H / 16; i += kThreads)
-            reinterpret_cast<int4 *>(ws + L.xq)[i] = reinterpret_cast<const int4 *>(s_xq)[i];
+            reinterpret_cast<int4 *>(ws + L.xq)[i] = reinterpret_cast<const int4 *>(C.s_xq)[i];
+#pragma unroll 1
         for (int a = tid; a < A; a += kThreads) {
             reinterpret_cast<int32_t *>(ws + L.ids)[a] = s_ids[a];
             reinterpret_cast<float *>(ws + L.w)[a] = s_wt[a];
         }
     }
     __syncthreads();
+    JobX *s_jobs = C.s_jobs;
     if (warp == 0) {
         const int nwords = (E + 31) / 32;
         const uint32_t word = lane < nwords ? s_bits[lane] : 0u;
         int csum = 0;
+#pragma unroll 1
         for (uint32_t w = word; w; w &= w - 1) csum += s_cnt[lane * 32 + __ffs(w) - 1];
         int jinc = __popc(word), cinc = csum;
 #pragma unroll
@@ -471,6 +480,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_fused(const DecParams P)
         }
         int jb = jinc - __popc(word), cb = cinc - csum;
         s_wbase[lane] = cb;
+#pragma unroll 1
         for (uint32_t w = word; w; w &= w - 1) {
             const int e = lane * 32 + __ffs(w) - 1;
             const int cnt = s_cnt[e];
@@ -491,30 +501,34 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_fused(const DecParams P)
                 J.n = T;
                 J.shared = 1;
             }
-            s_misc[0] = n_routed + (P.shared ? 1 : 0);
+            C.s_misc[0] = n_routed + (P.shared ? 1 : 0);
         }
     }
     __syncthreads();
-    const int U = s_misc[0];
+    const int U = C.s_misc[0];
+#pragma unroll 1
     for (int a = tid; a < A; a += kThreads) {
         const int e = s_ids[a];
         int rank = 0;
+#pragma unroll 1
         for (int b = 0; b < a; b++) rank += s_ids[b] == e;
         const int slot = s_off[e] + rank;
-        s_stok[slot] = a / k;
-        s_sw[slot] = s_wt[a];
+        C.s_stok[slot] = a / k;
+        C.s_sw[slot] = s_wt[a];
         if (cta0) {
             reinterpret_cast<int32_t *>(ws + L.perm)[slot] = a;
             reinterpret_cast<int32_t *>(ws + L.inv_perm)[a] = slot;
         }
     }
+#pragma unroll 1
     for (int t = tid; t < T; t += kThreads) {
-        s_stok[A + t] = t;
-        s_sw[A + t] = 1.0f;
+        C.s_stok[A + t] = t;
+        C.s_sw[A + t] = 1.0f;
     }
+#pragma unroll 1
     for (int u = tid; u < U; u += kThreads) {
         JobX &J = s_jobs[u];
-        const ExpertDev &ex = P.experts[J.expert];
+        const ExpertDev &ex = s_ex[J.expert];
         J.m[0] = ex.m[0];
         J.m[1] = ex.m[1];
         J.m[2] = ex.m[2];
@@ -524,10 +538,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_fused(const DecParams P)
         J.fmt = ex.fmt;
     }
     if (cta0) {
+#pragma unroll 1
         for (int e = tid; e < E; e += kThreads) {
             reinterpret_cast<int32_t *>(ws + L.counts)[e] = s_cnt[e];
             const uint32_t below = s_bits[e >> 5] & ((1u << (e & 31)) - 1u);
             int off = s_wbase[e >> 5];
+#pragma unroll 1
             for (uint32_t w = below; w; w &= w - 1) off += s_cnt[(e & ~31) + __ffs(w) - 1];
             reinterpret_cast<int32_t *>(ws + L.offsets)[e] = off;
         }
@@ -535,281 +551,434 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_fused(const DecParams P)
     }
     __syncthreads();
     if (cta0) {
+#pragma unroll 1
         for (int u = tid; u < U; u += kThreads) {
             const JobX &J = s_jobs[u];
             reinterpret_cast<Job *>(ws + L.jobs)[u] = Job{J.expert, J.slot0, J.n, J.shared};
         }
         if (tid == 0) *reinterpret_cast<int32_t *>(ws + L.njobs) = U;
     }
-    // the prologue scratch in the stage ring is dead from here on
+}
 
-    // ---- partition
-    const int G = gridDim.x, cta = blockIdx.x;
-    const int nb32 = F / 32;
-    const int n_blk = U * nb32;
-    const int my_blocks = n_blk / G + (cta < n_blk % G ? 1 : 0);
-    double gu_bytes = 0.0, row_bytes = 0.0;
-    for (int u = 0; u < U; u++) {
-        gu_bytes += 32.0 * nb32 * (double)(s_jobs[u].stride[0] + s_jobs[u].stride[1]);
-        row_bytes += (double)s_jobs[u].stride[2];
+// Stage ring bookkeeping of the producer.
+struct Ring {
+    int s;
+    uint32_t ph;
+};
+
+__device__ __forceinline__ bool ring_acquire(const DecParams &P, const Ctx &C, Ring &R, int &st) {
+    if (!ptx::mbar_wait_bounded(&C.empty[R.s], R.ph ^ 1u, kWaitNs)) return false;
+    st = R.s;
+    if (++R.s == P.nstages) {
+        R.s = 0;
+        R.ph ^= 1u;
     }
-    const double blk_bytes = n_blk ? gu_bytes / n_blk : 0.0;
-    const int i_lo = down_bound(cta, G, H, n_blk, blk_bytes, row_bytes);
-    const int i_hi = cta == G - 1 ? H : down_bound(cta + 1, G, H, n_blk, blk_bytes, row_bytes);
-    const int hb = P.hpad / 32;
+    return true;
+}
 
-    if (warp == kCW) {
-        // ---------------------------------------------------------------- producer
-        if (lane == 0) {
-            const uint64_t pol = ptx::policy_evict_first();
-            int s = 0;
-            uint32_t ph = 0;
-            bool ok = true;
-            auto acquire = [&](int &st) -> bool {
-                if (!ptx::mbar_wait_bounded(&empty[s], ph ^ 1u, kWaitNs)) return false;
-                st = s;
-                if (++s == P.nstages) {
-                    s = 0;
-                    ph ^= 1u;
-                }
-                return true;
-            };
-            for (int mb = 0; mb < my_blocks && ok; mb++) {
-                const int blk = cta + mb * G;
-                const int ju = blk / nb32, b = blk % nb32;
-                const JobX &J = s_jobs[ju];
-                for (int half = 0; half < 2 && ok; half++) {
-                    const int r0 = 32 * b + 16 * half;
-                    const uint32_t b0 = 16u * J.stride[0], b1 = 16u * J.stride[1];
-                    int st;
-                    if (!(ok = acquire(st))) break;
-                    meta[st] = StageMeta{ST_GU, ju, r0, 16, 0, 0, 0, 0};
-                    uint8_t *dst = sm + (size_t)st * P.stage_bytes;
-                    ptx::mbar_arrive_expect_tx(&full[st], b0 + b1);
-                    ptx::bulk_g2s(dst, J.m[0] + (size_t)r0 * J.stride[0], b0, &full[st], pol);
-                    ptx::bulk_g2s(dst + b0, J.m[1] + (size_t)r0 * J.stride[1], b1, &full[st], pol);
-                }
-            }
-            for (int i = i_lo; i < i_hi && ok;) {
-                const int rows = min(kDownRows, i_hi - i);
-                int j = 0;
-                while (j < U && ok) {
-                    const int j0 = j;
-                    uint32_t bytes = 0;
-                    while (j < U) {
-                        const uint32_t b = (uint32_t)rows * s_jobs[j].stride[2];
-                        if (j > j0 && bytes + b > (uint32_t)P.stage_bytes) break;
-                        bytes += b;
-                        j++;
-                    }
-                    int st;
-                    if (!(ok = acquire(st))) break;
-                    meta[st] = StageMeta{ST_DOWN, i, rows, j0, j, j == U ? 1 : 0, 0, 0};
-                    uint8_t *dst = sm + (size_t)st * P.stage_bytes;
-                    ptx::mbar_arrive_expect_tx(&full[st], bytes);
-                    uint32_t off = 0;
-                    for (int jj = j0; jj < j; jj++) {
-                        const JobX &J = s_jobs[jj];
-                        const uint32_t b = (uint32_t)rows * J.stride[2];
-                        ptx::bulk_g2s(dst + off, J.m[2] + (size_t)i * J.stride[2], b, &full[st], pol);
-                        off += b;
-                    }
-                }
-                i += rows;
+// One thread: stream this CTA's gate/up blocks, then its down rows, into the ring.
+__device__ __forceinline__ void producer(const DecParams &P, const Ctx &C) {
+    const uint64_t pol = ptx::policy_evict_first();
+    Ring R{0, 0u};
+    bool ok = true;
+    const int G = gridDim.x, cta = blockIdx.x;
+    const JobX *s_jobs = C.s_jobs;
+#pragma unroll 1
+    for (int mb = 0; mb < C.my_blocks && ok; mb++) {
+        const int blk = cta + mb * G;
+        const int ju = blk / C.nb32, b = blk % C.nb32;
+        const JobX &J = s_jobs[ju];
+#pragma unroll 1
+        for (int half = 0; half < 2 && ok; half++) {
+            const int r0 = 32 * b + 16 * half;
+            const uint32_t b0 = 16u * J.stride[0], b1 = 16u * J.stride[1];
+            int st;
+            if (!(ok = ring_acquire(P, C, R, st))) break;
+            C.meta[st] = StageMeta{ST_GU, ju, r0, 16, 0, 0, 0, 0};
+            uint8_t *dst = C.ring + (size_t)st * P.stage_bytes;
+            ptx::mbar_arrive_expect_tx(&C.full[st], b0 + b1);
+            ptx::bulk_g2s(dst, J.m[0] + (size_t)r0 * J.stride[0], b0, &C.full[st], pol);
+            ptx::bulk_g2s(dst + b0, J.m[1] + (size_t)r0 * J.stride[1], b1, &C.full[st], pol);
+        }
+    }
+    const int down_rows = 32;
+#pragma unroll 1
+    for (int i = C.i_lo; i < C.i_hi && ok;) {
+        const int rows = min(down_rows, C.i_hi - i);
+        int j = 0;
+#pragma unroll 1
+        while (j < C.U && ok) {
+            const int j0 = j;
+            uint32_t bytes = 0;
+#pragma unroll 1
+            while (j < C.U) {
+                const uint32_t b = (uint32_t)rows * s_jobs[j].stride[2];
+                if (j > j0 && bytes + b > (uint32_t)P.stage_bytes) break;
+                bytes += b;
+                j++;
             }
             int st;
-            if (ok && acquire(st)) {
-                meta[st] = StageMeta{ST_END, 0, 0, 0, 0, 0, 0, 0};
-                ptx::mbar_arrive(&full[st]);
-            } else {
-                set_status(status, MOE_ERR_TIMEOUT);
+            if (!(ok = ring_acquire(P, C, R, st))) break;
+            C.meta[st] = StageMeta{ST_DOWN, i, rows, j0, j, j == C.U ? 1 : 0, 0, 0};
+            uint8_t *dst = C.ring + (size_t)st * P.stage_bytes;
+            ptx::mbar_arrive_expect_tx(&C.full[st], bytes);
+            uint32_t off = 0;
+#pragma unroll 1
+            for (int jj = j0; jj < j; jj++) {
+                const JobX &J = s_jobs[jj];
+                const uint32_t b = (uint32_t)rows * J.stride[2];
+                ptx::bulk_g2s(dst + off, J.m[2] + (size_t)i * J.stride[2], b, &C.full[st], pol);
+                off += b;
             }
         }
+        i += rows;
+    }
+    int st;
+    if (ok && ring_acquire(P, C, R, st)) {
+        C.meta[st] = StageMeta{ST_END, 0, 0, 0, 0, 0, 0, 0};
+        ptx::mbar_arrive(&C.full[st]);
     } else {
-        // ---------------------------------------------------------------- consumers
-        const int ctid = tid;                 // 0..255
-        int s = 0;
-        uint32_t ph = 0;
-        bool gu_done = false, have_h = false, skip_down = false;
-        int done_blocks = 0;
-        int8_t *g_hq = reinterpret_cast<int8_t *>(ws + L.hq);
-        uint16_t *g_hd = reinterpret_cast<uint16_t *>(ws + L.hd);
-        uint16_t *g_hs = reinterpret_cast<uint16_t *>(ws + L.hs);
-        float *g_hsum = reinterpret_cast<float *>(ws + L.hsum);
-        float *g_h = reinterpret_cast<float *>(ws + L.h);
-        while (true) {
-            if (!ptx::mbar_wait_bounded(&full[s], ph, kWaitNs)) {
-                if (lane == 0) set_status(status, MOE_ERR_TIMEOUT);
+        set_status(C.status, MOE_ERR_TIMEOUT);
+    }
+}
+
+// Q8_1 of a completed 32-row block of h (s_h [32][16]) for every slot of job J.
+__device__ __forceinline__ void quantize_h_block(const DecParams &P, const Ctx &C, const JobX &J, int b) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const WsLayout &L = P.L;
+    int8_t *g_hq = reinterpret_cast<int8_t *>(P.ws + L.hq);
+    uint16_t *g_hd = reinterpret_cast<uint16_t *>(P.ws + L.hd);
+    uint16_t *g_hs = reinterpret_cast<uint16_t *>(P.ws + L.hs);
+    float *g_hsum = reinterpret_cast<float *>(P.ws + L.hsum);
+    float *g_h = reinterpret_cast<float *>(P.ws + L.h);
+    const int F = C.F, hb = C.hb, nb32 = C.nb32;
+#pragma unroll 1
+    for (int t = warp; t < J.n; t += kCW) {
+        const int slot = J.slot0 + t;
+        const float v = C.s_h[lane * 16 + t];
+        g_h[(size_t)slot * F + 32 * b + lane] = v;
+        bool fin;
+        uint16_t d16, s16;
+        float dsum;
+        const int q = q8_1_lane(v, fin, d16, s16, dsum);
+        g_hq[(size_t)slot * P.hpad + 32 * b + lane] = (int8_t)q;
+        if (lane == 0) {
+            g_hd[(size_t)slot * hb + b] = d16;
+            g_hs[(size_t)slot * hb + b] = s16;
+            g_hsum[(size_t)slot * hb + b] = dsum;
+            if (!fin) set_status(C.status, MOE_ERR_NONFINITE);
+        }
+        if (b == nb32 - 1) {   // zero the padded tail [F, hpad) of this slot
+#pragma unroll 1
+            for (int z = F + lane; z < P.hpad; z += 32) g_hq[(size_t)slot * P.hpad + z] = 0;
+#pragma unroll 1
+            for (int z = nb32 + lane; z < hb; z += 32) {
+                g_hd[(size_t)slot * hb + z] = 0;
+                g_hs[(size_t)slot * hb + z] = 0;
+                g_hsum[(size_t)slot * hb + z] = 0.f;
+            }
+        }
+    }
+}
+
+// After this CTA's gate/up work: wait (bounded) until every block of h is published, then stage
+// every slot's Q8_1(h) in shared memory.  Returns false on timeout.
+__device__ __forceinline__ bool wait_and_stage_h(const DecParams &P, const Ctx &C) {
+    const int ctid = threadIdx.x;
+    const WsLayout &L = P.L;
+    if (ctid == 0) {
+        const uint64_t t0 = ptx::globaltimer();
+        int to = 0;
+#pragma unroll 1
+        while (ptx::ld_acquire_u32(&C.ctr[1]) < (uint32_t)C.n_blk) {
+            if (ptx::globaltimer() - t0 > kWaitNs) {
+                to = 1;
                 break;
             }
-            const StageMeta m = meta[s];
-            if (m.kind != ST_GU && !gu_done) {
-                // publish this CTA's Q8_1(h) blocks
-                gu_done = true;
-                ptx::named_barrier(1, kCW * 32);
-                if (ctid == 0 && done_blocks > 0) {
-                    __threadfence();
-                    atomicAdd(&ctr[1], (uint32_t)done_blocks);
-                }
-            }
-            if (m.kind == ST_END) break;
-            const uint8_t *stage = sm + (size_t)s * P.stage_bytes;
-            if (m.kind == ST_GU) {
-                const int ju = m.a, r0 = m.b;
-                const JobX &J = s_jobs[ju];
-                const int which = warp >> 2, rg = (warp & 3) * kRG;   // warps 0-3 gate, 4-7 up
-                for (int t0 = 0; t0 < J.n; t0 += NT) {
-                    const int n = min(NT, J.n - t0);
-                    int act[NT];
-#pragma unroll
-                    for (int t = 0; t < NT; t++) act[t] = t < n ? s_stok[J.slot0 + t0 + t] : 0;
-                    float acc[kRG][NT];
-#pragma unroll
-                    for (int r = 0; r < kRG; r++)
-#pragma unroll
-                        for (int t = 0; t < NT; t++) acc[r][t] = 0.f;
-                    const uint8_t *base = stage + (which ? 16u * J.stride[0] : 0u) +
-                                          (size_t)rg * J.stride[which];
-                    rows_dot<NT, kRG>(J.fmt, base, J.stride[which], kRG, H, s_xq, s_xd, s_xs, H,
-                                      act, n, acc);
-#pragma unroll
-                    for (int r = 0; r < kRG; r++)
-#pragma unroll
-                        for (int t = 0; t < NT; t++) {
-                            const float v = warp_sum(acc[r][t]);
-                            if (lane == 0 && t < n) s_gu[(which * 16 + rg + r) * 16 + t0 + t] = v;
-                        }
-                }
-                __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(&empty[s]);
-                ptx::named_barrier(1, kCW * 32);
-                const int hrow0 = r0 & 31;   // 0 or 16 inside the block
-                for (int i = ctid; i < 16 * J.n; i += kCW * 32) {
-                    const int rr = i / J.n, t = i % J.n;
-                    s_h[(hrow0 + rr) * 16 + t] =
-                        silu_mul(s_gu[rr * 16 + t], s_gu[(16 + rr) * 16 + t]);
-                }
-                ptx::named_barrier(1, kCW * 32);
-                if (hrow0 == 16) {   // the block is complete: Q8_1 of its 32 rows, per slot
-                    const int b = r0 / 32;
-                    for (int t = warp; t < J.n; t += kCW) {
-                        const int slot = J.slot0 + t;
-                        const float v = s_h[lane * 16 + t];
-                        g_h[(size_t)slot * F + 32 * b + lane] = v;
-                        bool fin;
-                        uint16_t d16, s16;
-                        float dsum;
-                        const int q = q8_1_lane(v, fin, d16, s16, dsum);
-                        g_hq[(size_t)slot * P.hpad + 32 * b + lane] = (int8_t)q;
-                        if (lane == 0) {
-                            g_hd[(size_t)slot * hb + b] = d16;
-                            g_hs[(size_t)slot * hb + b] = s16;
-                            g_hsum[(size_t)slot * hb + b] = dsum;
-                            if (!fin) set_status(status, MOE_ERR_NONFINITE);
-                        }
-                        if (b == nb32 - 1) {   // zero the padded tail [F, hpad) of this slot
-                            for (int z = F + lane; z < P.hpad; z += 32) g_hq[(size_t)slot * P.hpad + z] = 0;
-                            for (int z = nb32 + lane; z < hb; z += 32) {
-                                g_hd[(size_t)slot * hb + z] = 0;
-                                g_hs[(size_t)slot * hb + z] = 0;
-                                g_hsum[(size_t)slot * hb + z] = 0.f;
-                            }
-                        }
-                    }
-                    done_blocks++;
-                    ptx::named_barrier(1, kCW * 32);   // s_h is rewritten by the next block
-                }
-            } else {   // ST_DOWN
-                if (!have_h) {
-                    if (ctid == 0) {
-                        const uint64_t t0 = ptx::globaltimer();
-                        int to = 0;
-                        while (ptx::ld_acquire_u32(&ctr[1]) < (uint32_t)n_blk) {
-                            if (ptx::globaltimer() - t0 > kWaitNs) {
-                                to = 1;
-                                break;
-                            }
-                            __nanosleep(32);
-                        }
-                        s_misc[2] = to;
-                        if (to) set_status(status, MOE_ERR_TIMEOUT);
-                    }
-                    ptx::named_barrier(1, kCW * 32);
-                    skip_down = s_misc[2] != 0;
-                    for (int i = ctid; i < P.slots * P.hpad / 16; i += kCW * 32)
-                        reinterpret_cast<int4 *>(s_hq)[i] = ptx::ld_cg_v4(g_hq + (size_t)i * 16);
-                    for (int i = ctid; i < P.slots * hb; i += kCW * 32) {
-                        s_hd[i] = half_bits_to_float(__ldcg(g_hd + i));
-                        s_hs[i] = __ldcg(g_hsum + i);
-                    }
-                    ptx::named_barrier(1, kCW * 32);
-                    have_h = true;
-                }
-                const int i0 = m.a, rows = m.b;
-                if (m.c == 0) {                 // first stage of a down unit: clear the sums
-                    for (int i = ctid; i < kDownRows * T; i += kCW * 32) s_acc[i] = 0.f;
-                    ptx::named_barrier(1, kCW * 32);
-                }
-                const int rw = warp * kRD;
-                if (!skip_down && rw < rows) {
-                    uint32_t off = 0;
-                    for (int ju = m.c; ju < m.d; ju++) {
-                        const JobX &J = s_jobs[ju];
-                        const int Kd = J.fmt == MOE_FMT_Q8_0 ? ((F + 31) / 32) * 32 : P.hpad;
-                        const uint8_t *base = stage + off + (size_t)rw * J.stride[2];
-                        off += (uint32_t)rows * J.stride[2];
-                        for (int t0 = 0; t0 < J.n; t0 += NT) {
-                            const int n = min(NT, J.n - t0);
-                            int act[NT];
-#pragma unroll
-                            for (int t = 0; t < NT; t++) act[t] = t < n ? J.slot0 + t0 + t : 0;
-                            float acc[kRD][NT];
-#pragma unroll
-                            for (int r = 0; r < kRD; r++)
-#pragma unroll
-                                for (int t = 0; t < NT; t++) acc[r][t] = 0.f;
-                            rows_dot<NT, kRD>(J.fmt, base, J.stride[2], min(kRD, rows - rw), Kd,
-                                              s_hq, s_hd, s_hs, P.hpad, act, n, acc);
-#pragma unroll
-                            for (int r = 0; r < kRD; r++)
-#pragma unroll
-                                for (int t = 0; t < NT; t++) {
-                                    const float v = warp_sum(acc[r][t]);
-                                    if (lane == 0 && t < n && rw + r < rows) {
-                                        const int slot = J.slot0 + t0 + t;
-                                        s_acc[(rw + r) * T + s_stok[slot]] += s_sw[slot] * v;
-                                    }
-                                }
-                        }
-                    }
-                }
-                __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(&empty[s]);
-                if (m.e) {                      // last stage of the unit: write the outputs
-                    ptx::named_barrier(1, kCW * 32);
-                    if (!skip_down)
-                        for (int i = ctid; i < rows * T; i += kCW * 32) {
-                            const int r = i / T, t = i % T;
-                            P.out[(size_t)t * H + i0 + r] = s_acc[r * T + t];
-                        }
-                    ptx::named_barrier(1, kCW * 32);
-                }
-            }
-            if (++s == P.nstages) {
-                s = 0;
-                ph ^= 1u;
+            __nanosleep(32);
+        }
+        C.s_misc[2] = to;
+        if (to) set_status(C.status, MOE_ERR_TIMEOUT);
+    }
+    ptx::named_barrier(1, kCW * 32);
+    const int8_t *g_hq = reinterpret_cast<const int8_t *>(P.ws + L.hq);
+    const uint16_t *g_hd = reinterpret_cast<const uint16_t *>(P.ws + L.hd);
+    const float *g_hsum = reinterpret_cast<const float *>(P.ws + L.hsum);
+#pragma unroll 1
+    for (int i = ctid; i < P.slots * P.hpad / 16; i += kCW * 32)
+        reinterpret_cast<int4 *>(C.s_hq)[i] = ptx::ld_cg_v4(g_hq + (size_t)i * 16);
+#pragma unroll 1
+    for (int i = ctid; i < P.slots * C.hb; i += kCW * 32) {
+        C.s_hd[i] = half_bits_to_float(__ldcg(g_hd + i));
+        C.s_hs[i] = __ldcg(g_hsum + i);
+    }
+    ptx::named_barrier(1, kCW * 32);
+    return C.s_misc[2] == 0;
+}
+
+// Sum a down unit's per-warp partials in a fixed order and write the outputs.
+template <int TT>
+__device__ __forceinline__ void finish_down_unit(const DecParams &P, const Ctx &C, int i0, int rows) {
+    const int ctid = threadIdx.x;
+#pragma unroll 1
+    for (int i = ctid; i < rows * C.T; i += kCW * 32) {
+        const int r = i / C.T, t = i % C.T;
+        float v = 0.f;
+#pragma unroll 1
+        for (int w = 0; w < kCW; w++)
+            v += C.s_part[((size_t)w * 2 * 32 + r) * TT + t] +
+                 C.s_part[((size_t)w * 2 * 32 + 32 + r) * TT + t];
+        P.out[(size_t)t * C.H + i0 + r] = v;
+    }
+}
+
+// The 16 consumer warps: gate/up units, then down units, from the ring.
+template <int NT, int TT, int FK>
+__device__ __forceinline__ void consumer(const DecParams &P, const Ctx &C) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int H = C.H, F = C.F;
+    int s = 0;
+    uint32_t ph = 0;
+    bool gu_done = false, have_h = false, skip_down = false;
+    int done_blocks = 0;
+#pragma unroll 1
+    while (true) {
+        if (!ptx::mbar_wait_bounded(&C.full[s], ph, kWaitNs)) {
+            if (lane == 0) set_status(C.status, MOE_ERR_TIMEOUT);
+            break;
+        }
+        const StageMeta m = C.meta[s];
+        if (m.kind != ST_GU && !gu_done) {
+            // publish this CTA's Q8_1(h) blocks
+            gu_done = true;
+            ptx::named_barrier(1, kCW * 32);
+            if (threadIdx.x == 0 && done_blocks > 0) {
+                __threadfence();
+                atomicAdd(&C.ctr[1], (uint32_t)done_blocks);
             }
         }
+        if (m.kind == ST_END) break;
+        const uint8_t *stage = C.ring + (size_t)s * P.stage_bytes;
+        if (m.kind == ST_GU) {
+            // warp w computes gate row r0+w and up row r0+w for every token of the job
+            const int ju = m.a, r0 = m.b;
+            const JobX &J = C.s_jobs[ju];
+            const int hrow0 = r0 & 31;   // 0 or 16 inside the block
+            const uint8_t *const rp[2] = {stage + (size_t)warp * J.stride[0],
+                                          stage + 16u * J.stride[0] + (size_t)warp * J.stride[1]};
+#pragma unroll 1
+            for (int t0 = 0; t0 < J.n; t0 += NT) {
+                const int n = min(NT, J.n - t0);
+                int act[NT];
+#pragma unroll
+                for (int t = 0; t < NT; t++) act[t] = t < n ? C.s_stok[J.slot0 + t0 + t] : 0;
+                float acc[2][NT];
+#pragma unroll
+                for (int t = 0; t < NT; t++) acc[0][t] = acc[1][t] = 0.f;
+                rows_dot<NT, 2, FK>(J.fmt, rp, H, C.s_xq, C.s_xd, C.s_xs, H, act, n, 32, acc);
+#pragma unroll
+                for (int t = 0; t < NT; t++) {
+                    const float g = warp_sum(acc[0][t]), u = warp_sum(acc[1][t]);
+                    if (lane == 0 && t < n) C.s_h[(hrow0 + warp) * 16 + t0 + t] = silu_mul(g, u);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&C.empty[s]);
+            if (hrow0 == 16) {   // the block is complete: Q8_1 of its 32 rows, per slot
+                ptx::named_barrier(1, kCW * 32);
+                quantize_h_block(P, C, J, r0 / 32);
+                done_blocks++;
+                ptx::named_barrier(1, kCW * 32);   // s_h is rewritten by the next block
+            }
+        } else {   // ST_DOWN
+            if (!have_h) {
+                skip_down = !wait_and_stage_h(P, C);
+                have_h = true;
+            }
+            const int i0 = m.a, rows = m.b;
+            const int lpr = C.down_lpr, sr = lane / lpr;
+            float *part = C.s_part + (size_t)warp * 2 * 32 * TT;   // this warp's [2][32][TT]
+            if (m.c == 0) {   // first stage of a down unit: clear this warp's partials
+#pragma unroll 1
+                for (int i = lane; i < 2 * 32 * TT; i += 32) part[i] = 0.f;
+                __syncwarp();
+            }
+            // items (job, row) of this stage, job-major; a lane group takes one item
+            const int nj = m.d - m.c, nitems = nj * rows;
+            const int per_pass = kCW * (32 / lpr);
+#pragma unroll 1
+            for (int base_i = warp * (32 / lpr); base_i < nitems && !skip_down; base_i += per_pass) {
+                const int it = base_i + sr;
+                const bool valid = it < nitems;
+                const int jl = valid ? it / rows : 0, r = valid ? it % rows : 0;
+                const JobX &J = C.s_jobs[m.c + jl];
+                uint32_t joff;
+                if (FK != FK_ANY) {
+                    joff = (uint32_t)jl * rows * J.stride[2];
+                } else {
+                    joff = 0;
+#pragma unroll 1
+                    for (int jj = m.c; jj < m.c + jl; jj++) joff += (uint32_t)rows * C.s_jobs[jj].stride[2];
+                }
+                const int Kd = (FK == FK_ANY && J.fmt == MOE_FMT_Q8_0) ? ((F + 31) / 32) * 32 : P.hpad;
+                const uint8_t *const rp[1] = {valid ? stage + joff + (size_t)r * J.stride[2] : nullptr};
+                const int jn = valid ? J.n : 0;
+                int nmax = jn;
+                if (lpr == 16) nmax = max(nmax, __shfl_xor_sync(kFullMask, nmax, 16));
+#pragma unroll 1
+                for (int t0 = 0; t0 < nmax; t0 += NT) {
+                    const int n = max(0, min(NT, jn - t0));
+                    int act[NT];
+#pragma unroll
+                    for (int t = 0; t < NT; t++) act[t] = t < n ? J.slot0 + t0 + t : 0;
+                    float acc[1][NT];
+#pragma unroll
+                    for (int t = 0; t < NT; t++) acc[0][t] = 0.f;
+                    rows_dot<NT, 1, FK>(J.fmt, rp, Kd, C.s_hq, C.s_hd, C.s_hs, P.hpad, act, n, lpr, acc);
+#pragma unroll
+                    for (int t = 0; t < NT; t++) {
+                        float v = acc[0][t];
+                        if (lpr == 32) v += __shfl_xor_sync(kFullMask, v, 16);
+                        v += __shfl_xor_sync(kFullMask, v, 8);
+                        v += __shfl_xor_sync(kFullMask, v, 4);
+                        v += __shfl_xor_sync(kFullMask, v, 2);
+                        v += __shfl_xor_sync(kFullMask, v, 1);
+                        acc[0][t] = v;
+                    }
+                    // the lane groups write their own halves of the partials in turn
+                    if (lane % lpr == 0) {
+                        float *pr = part + (sr * 32 + r) * TT;
+#pragma unroll
+                        for (int t = 0; t < NT; t++) {
+                            if (t < n) {
+                                const int slot = J.slot0 + t0 + t;
+                                pr[C.s_stok[slot]] += C.s_sw[slot] * acc[0][t];
+                            }
+                        }
+                    }
+                    __syncwarp();
+                }
+            }
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&C.empty[s]);
+            if (m.e) {   // last stage of the unit: sum the partials in warp order, write
+                ptx::named_barrier(1, kCW * 32);
+                if (!skip_down) finish_down_unit<TT>(P, C, i0, rows);
+                ptx::named_barrier(1, kCW * 32);
+            }
+        }
+        if (++s == P.nstages) {
+            s = 0;
+            ph ^= 1u;
+        }
+    }
+}
+
+// NT: activation rows per pass of rows_dot; TT: largest token count the down sums hold;
+// FK: format class of the arena; VPL: router logits per lane (E <= 32 * VPL).
+template <int NT, int TT, int FK, int VPL>
+__global__ void __launch_bounds__(kThreads, 1) k_decode_fused(const DecParams P) {
+    extern __shared__ __align__(128) uint8_t sm[];
+    const int tid = threadIdx.x, warp = tid >> 5;
+    Ctx C;
+    C.s_xq = reinterpret_cast<int8_t *>(sm + P.o_xq);
+    C.s_xd = reinterpret_cast<float *>(sm + P.o_xd);
+    C.s_xs = reinterpret_cast<float *>(sm + P.o_xs);
+    C.s_jobs = reinterpret_cast<JobX *>(sm + P.o_jobs);
+    C.s_stok = reinterpret_cast<int *>(sm + P.o_stok);
+    C.s_sw = reinterpret_cast<float *>(sm + P.o_sw);
+    C.s_hq = reinterpret_cast<int8_t *>(sm + P.o_hq);
+    C.s_hd = reinterpret_cast<float *>(sm + P.o_hd);
+    C.s_hs = reinterpret_cast<float *>(sm + P.o_hs);
+    C.s_part = reinterpret_cast<float *>(sm + P.o_gu);
+    C.s_h = reinterpret_cast<float *>(sm + P.o_h);
+    C.s_misc = reinterpret_cast<int *>(sm + P.o_misc);
+    C.full = reinterpret_cast<uint64_t *>(sm + P.o_bar);
+    C.empty = C.full + P.nstages;
+    C.meta = reinterpret_cast<StageMeta *>(sm + P.o_meta);
+    C.ring = sm;
+    C.ws = P.ws;
+    C.status = reinterpret_cast<uint32_t *>(P.ws + P.L.status);
+    C.ctr = reinterpret_cast<uint32_t *>(P.ws + P.L.sync);
+    C.T = P.T;
+    C.H = P.H;
+    C.F = P.F;
+    C.E = P.E;
+    C.k = P.k;
+    C.cta0 = blockIdx.x == 0;
+    C.hb = P.hpad / 32;
+    C.nb32 = P.F / 32;
+
+    ptx::grid_dependency_wait();
+    ptx::launch_dependents();
+    if (tid == 0) {
+#pragma unroll 1
+        for (int s = 0; s < P.nstages; s++) {
+            ptx::mbar_init(&C.full[s], 1);
+            ptx::mbar_init(&C.empty[s], kCW);
+        }
+        ptx::fence_barrier_init();
+        C.s_misc[2] = 0;
+    }
+    prologue<VPL>(P, C, sm);
+    // the prologue scratch in the stage ring is dead from here on
+    const int G = gridDim.x, cta = blockIdx.x;
+    C.U = C.s_misc[0];
+    C.n_blk = C.U * C.nb32;
+    C.my_blocks = C.n_blk / G + (cta < C.n_blk % G ? 1 : 0);
+    // down rows: computed after the barrier by every CTA, so split evenly
+    C.i_lo = (int)((long long)P.H * cta / G);
+    C.i_hi = (int)((long long)P.H * (cta + 1) / G);
+    // down: rows with <= 16 chunks are handled by 16-lane groups (two items per warp)
+    int kmax_down = 0;
+#pragma unroll 1
+    for (int u = 0; u < C.U; u++)
+        kmax_down = max(kmax_down, C.s_jobs[u].fmt == MOE_FMT_Q8_0 ? (P.F + 31) / 32 : P.hpad / 32);
+    C.down_lpr = kmax_down <= 16 ? 16 : 32;
+
+    if (warp == kCW) {
+        if ((tid & 31) == 0) producer(P, C);
+    } else {
+        consumer<NT, TT, FK>(P, C);
     }
     __syncthreads();
     if (tid == 0) {
         __threadfence();
-        if (atomicAdd(&ctr[2], 1u) == gridDim.x - 1) {
-            ctr[1] = 0;
-            ctr[2] = 0;
+        if (atomicAdd(&C.ctr[2], 1u) == gridDim.x - 1) {
+            C.ctr[1] = 0;
+            C.ctr[2] = 0;
             __threadfence();
         }
     }
+}
+
+template <int NT, int TT, int FK, int VPL>
+cudaError_t launch_one(const cudaLaunchConfig_t &cfg, const DecParams &P) {
+    cudaError_t err = ensure_smem(k_decode_fused<NT, TT, FK, VPL>, (size_t)P.smem_bytes);
+    if (err != cudaSuccess) return err;
+    return cudaLaunchKernelEx(&cfg, k_decode_fused<NT, TT, FK, VPL>, P);
+}
+
+template <int NT, int TT, int FK>
+cudaError_t launch_vpl(const cudaLaunchConfig_t &cfg, const DecParams &P, int E) {
+    if (E <= 256) return launch_one<NT, TT, FK, 8>(cfg, P);
+    if (E <= 512) return launch_one<NT, TT, FK, 16>(cfg, P);
+    return launch_one<NT, TT, FK, 32>(cfg, P);
+}
+
+template <int NT, int TT>
+cudaError_t launch_fk(const cudaLaunchConfig_t &cfg, const DecParams &P, int fk, int E) {
+    if (fk == FK_Q4K) return launch_vpl<NT, TT, FK_Q4K>(cfg, P, E);
+    if (fk == FK_Q5K) return launch_vpl<NT, TT, FK_Q5K>(cfg, P, E);
+    return launch_vpl<NT, TT, FK_ANY>(cfg, P, E);
+}
+
+// Instantiations: batch class (1, <= 4, <= 16 tokens) x format class x top-k width; the
+// largest batch class exists only for the any-format kernel, to bound the code size.
+cudaError_t launch_variant(const cudaLaunchConfig_t &cfg, const DecParams &P, int T, int fk, int E) {
+    if (T <= 1) return launch_fk<1, 1>(cfg, P, fk, E);
+    if (T <= 4) return launch_fk<4, 4>(cfg, P, fk, E);
+    return launch_vpl<4, 16, FK_ANY>(cfg, P, E);
 }
 
 }  // namespace
@@ -830,7 +999,7 @@ cudaError_t launch_decode_fused(const FfnArgs &a, int E, int shared, const float
         return err;
     const int max_s01 = a.max_stride01, max_s2 = a.max_stride2;
     if (max_s01 <= 0 || max_s2 <= 0 || 2 * kUnitPairs * max_s01 > 96 * 1024 ||
-        kDownRows * max_s2 > 96 * 1024)
+        kDownRowsMax * max_s2 > 96 * 1024)
         return cudaSuccess;   // rows too wide for the ring: not taken
     DecParams P{};
     P.experts = a.experts;
@@ -849,7 +1018,10 @@ cudaError_t launch_decode_fused(const FfnArgs &a, int E, int shared, const float
     P.max_jobs = a.max_jobs;
     P.slots = a.T * a.k + a.T;
     auto al = [](int v, int q) { return (v + q - 1) / q * q; };
-    P.stage_bytes = al(std::max(2 * kUnitPairs * max_s01, kDownRows * max_s2), 1024);
+    const int tt = a.T <= 1 ? 1 : a.T <= 4 ? 4 : 16;
+    const int fk = a.fmt_mask == (1 << MOE_FMT_Q4_K) ? FK_Q4K
+                   : a.fmt_mask == (1 << MOE_FMT_Q5_K) ? FK_Q5K : FK_ANY;
+    P.stage_bytes = al(std::max(2 * kUnitPairs * max_s01, kDownRowsMax * max_s2), 1024);
     const int slots = P.slots;
     const int sizes[] = {
         2 * 16 * 8,                                  // barriers (<= 16 stages)
@@ -863,15 +1035,16 @@ cudaError_t launch_decode_fused(const FfnArgs &a, int E, int shared, const float
         al(slots * a.hpad, 128),                     // Q8_1(h) q
         al(slots * (a.hpad / 32) * 4, 16),           // Q8_1(h) d
         al(slots * (a.hpad / 32) * 4, 16),           // Q8_1(h) xd*sum(q)
-        2 * 16 * 16 * 4,                             // gate / up sums [2][16][16]
+        kCW * 2 * 32 * tt * 4,                       // down partials [kCW][2][32][TT]
         32 * 16 * 4,                                 // one block of h [32][16]
-        al(kDownRows * a.T * 4, 16),                 // down sums [16][T]
+        16,                                          // (unused)
         64};                                         // misc
     int fixed = 0;
     for (int v : sizes) fixed += v;
     int nst = (cap - fixed - 1024) / P.stage_bytes;
     if (nst > 16) nst = 16;
-    const int scratch = (2 * E + 64 + 2 * a.T * a.k) * 4;   // prologue scratch in the ring
+    const int scratch = al((2 * E + 64 + 2 * a.T * a.k) * 4, 16) +
+                        (E + shared) * (int)sizeof(ExpertDev);   // prologue scratch in the ring
     if (nst < 2 || nst * P.stage_bytes < scratch) return cudaSuccess;
     P.nstages = nst;
     int o = nst * P.stage_bytes;
@@ -894,13 +1067,7 @@ cudaError_t launch_decode_fused(const FfnArgs &a, int E, int shared, const float
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
-    if (a.T <= 1) {
-        if ((err = ensure_smem(k_decode_fused<1>, (size_t)P.smem_bytes)) != cudaSuccess) return err;
-        err = cudaLaunchKernelEx(&cfg, k_decode_fused<1>, P);
-    } else {
-        if ((err = ensure_smem(k_decode_fused<4>, (size_t)P.smem_bytes)) != cudaSuccess) return err;
-        err = cudaLaunchKernelEx(&cfg, k_decode_fused<4>, P);
-    }
+    err = launch_variant(cfg, P, a.T, fk, E);
     if (err != cudaSuccess) return err;
     note_launches(1);
     *taken = true;
