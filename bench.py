@@ -97,17 +97,18 @@ class Clocks:
                 "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
 
 
-def traffic_for(kernel: str, src_files):
-    """dram bytes per launch from the committed ncu summary, if the kernel source is unchanged."""
+def traffic_for(kernel: str, workload: str):
+    """dram bytes per launch from the committed ncu summary (profiles/traffic.json), or None when
+    that capture was of another workload or the kernel's sources changed since it was taken."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         d = json.load(f).get(kernel)
-    if not d:
+    if not d or d.get("workload", "decode") != workload:
         return None
     h = hashlib.sha256()
-    for s in src_files:
+    for s in d.get("source_files", []):
         with open(os.path.join(ROOT, s), "rb") as f:
             h.update(f.read())
     return d["bytes_per_launch"] if d.get("source_sha256") == h.hexdigest() else None
@@ -285,9 +286,11 @@ def run_ours(args, rank, world):
         "expert_gbs": step_bytes / (ms_step / 1e3) / 1e9,
         "int8_tops": step_ops / (ms_step / 1e3) / 1e12,
         "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm, "unit": "GB/s",
-                     "frac": achieved_gbs / hbm, "traffic": None,
-                     "kernel": "moe_forward (one layer)", "peak_source": src,
-                     "bytes_per_launch": bytes_per_launch},
+                     "frac": achieved_gbs / hbm,
+                     "traffic": traffic_for("k_decode_fused", args.workload) if decode else None,
+                     "kernel": "k_decode_fused (one launch per layer)" if decode else
+                               "moe_forward (one layer)",
+                     "peak_source": src, "bytes_per_launch": bytes_per_launch},
         "e2e": {"value": world * tok_per_step * K2 / (ms_e2e / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(xs.nbytes + lgs.nbytes),
                 "d2h_bytes_per_step": int(out_h.numel() * 4)},
