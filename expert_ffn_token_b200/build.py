@@ -26,8 +26,9 @@ ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",
          "--expt-relaxed-constexpr", f"-I{INCLUDE}", f"-I{CSRC}"]
 
-LIB_SOURCES = ["k_route.cu", "k_ffn.cu", "k_decode.cu", "moe_api.cu", "moe_noalloc.cu"]
-OPTIONAL_SOURCES = ["k_gemm_tc.cu"]
+LIB_SOURCES = ["k_route.cu", "k_ffn.cu", "k_decode.cu", "k_gemm_tc.cu", "moe_api.cu",
+               "moe_noalloc.cu"]
+OPTIONAL_SOURCES: list[str] = []
 SYNTH_SOURCES = ["synth_fill.cu"]
 
 

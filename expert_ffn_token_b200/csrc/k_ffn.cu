@@ -116,12 +116,18 @@ __global__ void k_hpad_zero(int8_t *hq, uint16_t *hd, uint16_t *hs, float *hsum,
     }
 }
 
-cudaError_t launch_gateup_gemv(const FfnArgs &a, cudaStream_t st) {
+cudaError_t launch_hpad_zero(const FfnArgs &a, cudaStream_t st) {
     const int slots = a.T * a.k + a.T;   // upper bound, padded tail only
     if (a.hpad > a.F) {
         k_hpad_zero<<<64, 256, 0, st>>>(a.hq, a.hd, a.hs, a.hsum, slots, a.F, a.hpad);
         note_launches(1);
     }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gateup_gemv(const FfnArgs &a, cudaStream_t st) {
+    cudaError_t err0 = launch_hpad_zero(a, st);
+    if (err0 != cudaSuccess) return err0;
     constexpr int NT = 4;
     const size_t smem = (size_t)NT * a.H + 2 * sizeof(float) * NT * (a.H / 32) +
                         sizeof(float) * 32 * NT;

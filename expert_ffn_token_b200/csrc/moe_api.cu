@@ -21,6 +21,8 @@ struct moe_arena {
     int fmt_mask;             // bit f set when some expert uses format f
     int max_stride01, max_stride2;
     moe::ExpertDev *d_experts;
+    void *d_wmaps;            // tensor maps of the packed matrices (tensor-core path) or null
+    bool tc_ok;               // large batches may run on the tensor cores
     std::vector<moe_expert_desc> descs;
 };
 
@@ -48,7 +50,7 @@ static size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 static bool aligned(const void *p, size_t a) { return ((uintptr_t)p & (a - 1)) == 0; }
 
-WsLayout ws_layout(const moe_arena *A, int T, int k, uint32_t flags) {
+WsLayout ws_layout(const moe_arena *A, int T, int k, uint32_t flags, bool allow_tc) {
     WsLayout L{};
     size_t p = 0;
     auto take = [&](size_t bytes) {
@@ -86,6 +88,20 @@ WsLayout ws_layout(const moe_arena *A, int T, int k, uint32_t flags) {
     L.h = take((size_t)L.slots * F * 4);
     (void)flags;
     L.y = (flags & MOE_F_DETERMINISTIC) ? take((size_t)L.slots * H * 4) : 0;
+    // the tensor-core operands come last, so that a workspace without them keeps every other
+    // offset (moe_forward then runs the CUDA-core grouped kernels)
+    L.tc = allow_tc && A->tc_ok && ((flags & MOE_F_FORCE_PREFILL) || T > kDecodeMaxT) &&
+           !(flags & MOE_F_FORCE_DECODE);
+    if (L.tc) {
+        L.xg = take((size_t)L.slots * H * 2);
+        L.xgd = take((size_t)L.slots * (H / 32) * 4);
+        L.xgsh = take((size_t)L.slots * (H / 32) * 4);
+        L.xgsl = take((size_t)L.slots * (H / 32) * 4);
+        L.hg = take((size_t)L.slots * L.hpad * 2);
+        L.hgd = take((size_t)L.slots * (L.hpad / 32) * 4);
+        L.hgsh = take((size_t)L.slots * (L.hpad / 32) * 4);
+        L.hgsl = take((size_t)L.slots * (L.hpad / 32) * 4);
+    }
     L.total = p;
     return L;
 }
@@ -163,12 +179,34 @@ moe_status moe_arena_create(const void *d_arena, size_t arena_bytes, int hidden,
     A->max_stride01 = (int)ms01;
     A->max_stride2 = (int)ms2;
     A->descs.assign(host_descs, host_descs + n);
+    A->d_wmaps = nullptr;
+    A->tc_ok = false;
     if (cudaMalloc(&A->d_experts, sizeof(ExpertDev) * n) != cudaSuccess ||
         cudaMemcpy(A->d_experts, dev.data(), sizeof(ExpertDev) * n, cudaMemcpyHostToDevice) !=
             cudaSuccess) {
         cudaFree(A->d_experts);
         delete A;
         return MOE_ERR_CUDA;
+    }
+    // tensor-core path: weight tensor maps, and a shared-memory plan that fits this device
+    {
+        std::vector<uint8_t> maps;
+        int dev_id = 0, optin = 0;
+        const bool fits = cudaGetDevice(&dev_id) == cudaSuccess &&
+                          cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin,
+                                                 dev_id) == cudaSuccess &&
+                          tc_smem_bytes(fmt_mask) <= (size_t)optin;
+        if (fits && tc_build_weight_maps(A->base, host_descs, n, hidden, ffn, maps)) {
+            if (cudaMalloc(&A->d_wmaps, maps.size()) != cudaSuccess ||
+                cudaMemcpy(A->d_wmaps, maps.data(), maps.size(), cudaMemcpyHostToDevice) !=
+                    cudaSuccess) {
+                cudaFree(A->d_wmaps);
+                cudaFree(A->d_experts);
+                delete A;
+                return MOE_ERR_CUDA;
+            }
+            A->tc_ok = true;
+        }
     }
     *out = A;
     return MOE_OK;
@@ -177,6 +215,7 @@ moe_status moe_arena_create(const void *d_arena, size_t arena_bytes, int hidden,
 void moe_arena_destroy(moe_arena *arena) {
     if (!arena) return;
     cudaFree(arena->d_experts);
+    cudaFree(arena->d_wmaps);
     delete arena;
 }
 
@@ -288,7 +327,8 @@ moe_status moe_forward(const moe_arena *arena, const float *d_x, const float *d_
     if ((flags & MOE_F_FORCE_DECODE) && (flags & MOE_F_FORCE_PREFILL)) return MOE_ERR_INVALID_ARG;
     if (!aligned(d_x, 16) || !aligned(d_out, 16) || !aligned(d_logits, 4) || !aligned(d_ws, 256))
         return MOE_ERR_ALIGNMENT;
-    const WsLayout L = ws_layout(arena, T, k, flags);
+    WsLayout L = ws_layout(arena, T, k, flags);
+    if (ws_bytes < L.total && L.tc) L = ws_layout(arena, T, k, flags, false);
     if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
     cudaStream_t st = (cudaStream_t)stream;
     uint8_t *ws = static_cast<uint8_t *>(d_ws);
@@ -375,6 +415,41 @@ moe_status moe_forward(const moe_arena *arena, const float *d_x, const float *d_
     a.max_stride01 = arena->max_stride01;
     a.max_stride2 = arena->max_stride2;
 
+    if (L.tc && !(decode && T <= kDecodeMaxT)) {
+        // a4-a7 on the tensor cores
+        TcPhaseArgs p{};
+        p.ffn = a;
+        p.wmaps = arena->d_wmaps;
+        p.slots = L.slots;
+        p.keep_h = (flags & MOE_F_KEEP_H) ? 1 : 0;
+        p.xg = reinterpret_cast<__half *>(ws + L.xg);
+        p.xgd = reinterpret_cast<float *>(ws + L.xgd);
+        p.xgsh = reinterpret_cast<float *>(ws + L.xgsh);
+        p.xgsl = reinterpret_cast<float *>(ws + L.xgsl);
+        p.hg = reinterpret_cast<__half *>(ws + L.hg);
+        p.hgd = reinterpret_cast<float *>(ws + L.hgd);
+        p.hgsh = reinterpret_cast<float *>(ws + L.hgsh);
+        p.hgsl = reinterpret_cast<float *>(ws + L.hgsl);
+        const int used = T * k + (shared ? T : 0);
+        err = launch_act_gather(xq, xd, xsum, perm, T, k, H, used, p.xg, p.xgd, p.xgsh, p.xgsl,
+                                st);
+        if (err == cudaSuccess)
+            err = launch_hg_tail_zero(p.hg, p.hgd, p.hgsh, p.hgsl, L.slots, arena->F, L.hpad, st);
+        if (err == cudaSuccess && p.keep_h) err = launch_hpad_zero(a, st);
+        if (err == cudaSuccess) {
+            p.phase = 0;
+            err = launch_gemm_tc(p, st);
+        }
+        if (err == cudaSuccess && !(flags & MOE_F_DETERMINISTIC))
+            err = cudaMemsetAsync(d_out, 0, (size_t)T * H * sizeof(float), st);
+        if (err == cudaSuccess) {
+            p.phase = 1;
+            err = launch_gemm_tc(p, st);
+        }
+        if (err == cudaSuccess && (flags & MOE_F_DETERMINISTIC))
+            err = launch_combine(a, shared != 0, st);
+        return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    }
     // a4 + a5
     err = launch_gateup_gemv(a, st);
     if (err != cudaSuccess) return MOE_ERR_CUDA;

@@ -14,6 +14,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <vector>
+
 #include "moe.h"
 
 #if defined(__CUDA_ARCH__) && (__CUDA_ARCH__ < 1000)
@@ -57,12 +59,19 @@ struct Job {
 
 struct moe_arena_impl;
 
+
 // Offsets (bytes) of everything moe_forward keeps in its workspace.
 struct WsLayout {
     size_t status, sync, blkcnt, njobs, jobs, xq, xd, xs, xsum, ids, w, counts, offsets, perm,
         inv_perm, chunk_counts, chunk_base, hq, hd, hs, hsum, h, y, total;
-    int slots, hpad, max_jobs, n_chunks;
+    // tensor-core path: slot-ordered fp16 operands and fp32 scales (absent when tc == 0)
+    size_t xg, xgd, xgsh, xgsl, hg, hgd, hgsh, hgsl;
+    int slots, hpad, max_jobs, n_chunks, tc;
 };
+
+// Workspace layout of one moe_forward call (moe_api.cu).  Without allow_tc the tensor-core
+// operands are left out.
+WsLayout ws_layout(const moe_arena *A, int T, int k, uint32_t flags, bool allow_tc = true);
 
 // ------------------------------------------------------------------ device helpers
 
@@ -153,6 +162,34 @@ cudaError_t launch_decode_fused(const FfnArgs &a, int E, int shared, const float
                                 const float *logits, uint8_t *ws, const WsLayout &L,
                                 size_t sync_off, size_t blkcnt_off, bool pdl, cudaStream_t st,
                                 bool *taken);
+
+// Zero Q8_1(h) (int8 layout) in the padded columns [F, hpad) of every slot.
+cudaError_t launch_hpad_zero(const FfnArgs &a, cudaStream_t st);
+
+// ---- tensor-core path for large batches (k_gemm_tc.cu)
+
+// One projection phase: 0 = gate/up over the gathered activations, 1 = down over Q8_1(h).
+struct TcPhaseArgs {
+    FfnArgs ffn;
+    const void *wmaps;          // device array of the experts' weight tensor maps
+    int phase, slots, keep_h;
+    __half *xg;
+    float *xgd, *xgsh, *xgsl;
+    __half *hg;
+    float *hgd, *hgsh, *hgsl;
+};
+
+// Host encoding of every expert's weight tensor maps into `out` (bytes to copy to the device);
+// false when the shape or a map is not supported.
+bool tc_build_weight_maps(const uint8_t *d_base, const moe_expert_desc *descs, int n, int H,
+                          int F, std::vector<uint8_t> &out);
+size_t tc_smem_bytes(int fmt_mask);
+cudaError_t launch_gemm_tc(const TcPhaseArgs &p, cudaStream_t st);
+cudaError_t launch_act_gather(const int8_t *xq, const uint16_t *xd, const float *xsum,
+                              const int32_t *perm, int T, int k, int H, int slots, __half *xg,
+                              float *xgd, float *xgsh, float *xgsl, cudaStream_t st);
+cudaError_t launch_hg_tail_zero(__half *hg, float *hgd, float *hgsh, float *hgsl, int slots,
+                                int F, int hpad, cudaStream_t st);
 
 cudaError_t launch_dequant(const uint8_t *m, int fmt, int rows, int nblocks, int stride,
                            float *out, cudaStream_t st);

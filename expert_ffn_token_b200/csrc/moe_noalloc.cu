@@ -11,10 +11,6 @@
 
 #include "moe_internal.cuh"
 
-namespace moe {
-WsLayout ws_layout(const moe_arena *A, int T, int k, uint32_t flags);
-}
-
 namespace {
 
 constexpr size_t kNoallocScratchBytes = size_t(4) << 20;   // 4 MiB per GPU
