@@ -22,9 +22,9 @@
 //   * Q8_0 rows (d_j per 32 weights, no min) rescale at every sub-block.
 // Results agree with the exact sums up to fp32 rounding.
 //
-// Roles (448 threads): warp 0 issues TMA loads (packed weights as stored, activations, scales);
-// warp 1 allocates tensor memory and issues the MMAs; warps 2-5 unpack the packed weights into
-// the fp16 operand (128-byte swizzled, K-major) and the per-row scales; warps 6-13 read the
+// Roles (576 threads): warp 0 issues TMA loads (packed weights as stored, activations, scales);
+// warp 1 allocates tensor memory and issues the MMAs; warps 2-9 unpack the packed weights into
+// the fp16 operand (128-byte swizzled, K-major) and the per-row scales; warps 10-17 read the
 // accumulators and finish the tile (SwiGLU + Q8_1(h), or the weighted scatter into out).  All
 // hand-offs are mbarriers; every wait is bounded and a timeout ends the kernel with
 // MOE_ERR_TIMEOUT.
@@ -51,9 +51,11 @@ constexpr int kWSt = 4;            // 64-wide contraction stages in flight
 constexpr int kRawSt = 2;          // packed super-block stages
 constexpr int kMnSt = 2;           // min-term operand stages
 constexpr int kEpSt = 2;           // epilogue scale stages
-constexpr int kJBuf = 6;           // accumulators (64 columns each), one per sub-block
+constexpr int kGrp = 3;            // accumulator groups: one per 64-wide stage (2 sub-blocks x 64 columns)
 constexpr int kMinBuf = 2;         // min-term accumulators, one per tile
-constexpr int kThreads = 448;
+constexpr int kUnpackWarps = 8;    // two threads per weight row, one sub-block each per stage
+constexpr int kEpiWarp0 = 2 + kUnpackWarps;
+constexpr int kThreads = (kEpiWarp0 + 8) * 32;
 constexpr uint64_t kWaitNs = 2000000000ull;
 
 constexpr uint32_t kA16 = kTM * 128;                   // 128 rows x 64 fp16
@@ -70,10 +72,10 @@ constexpr uint32_t kEpStage = 7168;
 static_assert(kEpXdT + kEpRatio + kEpUnit <= kEpStage, "epilogue stage");
 constexpr int kXbPitch = 36;                           // floats per token row (bank spread)
 constexpr uint32_t kXbuf = 4 * 32 * kXbPitch * 4;
-constexpr int kNumBars = 2 * kWSt + 2 * kRawSt + 2 * kMnSt + 2 * kEpSt + 2 * kJBuf +
+constexpr int kNumBars = 2 * kWSt + 2 * kRawSt + 2 * kMnSt + 2 * kEpSt + 2 * kGrp +
                          2 * kMinBuf + 2 * 4 + 1;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kMinCol0 = kJBuf * 64;              // 384
+constexpr uint32_t kMinCol0 = kGrp * 128;              // 384
 
 __host__ __device__ inline uint32_t sb_bytes(int fmt) {
     return fmt == MOE_FMT_Q4_K ? 144u : fmt == MOE_FMT_Q5_K ? 176u : 272u;
@@ -179,8 +181,8 @@ __device__ __forceinline__ Smem carve(uint8_t *base, uint32_t raw_stage) {
     s.mn_empty = b; b += kMnSt;
     s.ep_full = b; b += kEpSt;
     s.ep_empty = b; b += kEpSt;
-    s.tm_full = b; b += kJBuf;
-    s.tm_empty = b; b += kJBuf;
+    s.tm_full = b; b += kGrp;
+    s.tm_empty = b; b += kGrp;
     s.min_full = b; b += kMinBuf;
     s.min_empty = b; b += kMinBuf;
     s.xb_full = b; b += 4;
@@ -212,10 +214,17 @@ __device__ __noinline__ bool wait_bar(uint64_t *bar, uint32_t parity, int *abort
     return true;
 }
 
+// Fast path inline (the phase is usually complete already), bounded slow path out of line.
+__device__ __forceinline__ bool wait_fast(uint64_t *bar, uint32_t parity, int *abort,
+                                          uint32_t *status) {
+    if (mbar_try_wait(bar, parity)) return true;
+    return wait_bar(bar, parity, abort, status);
+}
+
 // The same for all 32 lanes of a warp, with one answer for the warp.
 __device__ __forceinline__ bool wait_bar_warp(uint64_t *bar, uint32_t parity, int *abort,
                                               uint32_t *status) {
-    const bool ok = wait_bar(bar, parity, abort, status);
+    const bool ok = wait_fast(bar, parity, abort, status);
     return __all_sync(0xFFFFFFFFu, ok);
 }
 
@@ -258,7 +267,7 @@ __device__ void role_producer(const GemmArgs &a, const Smem &S, int nj, const CU
             yb = ya + 64;
         }
         for (int sb = 0; sb < nsb; sb++) {
-            if (!wait_bar(S.raw_empty + rr.s, rr.ph ^ 1u, S.abort, a.status)) return;
+            if (!wait_fast(S.raw_empty + rr.s, rr.ph ^ 1u, S.abort, a.status)) return;
             uint8_t *rs = S.raw + rr.s * a.raw_stage;
             mbar_arrive_expect_tx(S.raw_full + rr.s, 128u * sbb + (uint32_t)t.nbox * 1024u);
             const int x = kq ? sb * (int)sbb : sb * 136;
@@ -269,7 +278,7 @@ __device__ void role_producer(const GemmArgs &a, const Smem &S, int nj, const CU
                             S.raw_full + rr.s);
             rr.adv(kRawSt);
             if (kq) {
-                if (!wait_bar(S.mn_empty + rm.s, rm.ph ^ 1u, S.abort, a.status)) return;
+                if (!wait_fast(S.mn_empty + rm.s, rm.ph ^ 1u, S.abort, a.status)) return;
                 uint8_t *ms = S.mn + rm.s * kMnStage;
                 mbar_arrive_expect_tx(S.mn_full + rm.s, (uint32_t)t.nbox * 2048u);
                 for (int b = 0; b < t.nbox; b++) {
@@ -281,7 +290,7 @@ __device__ void role_producer(const GemmArgs &a, const Smem &S, int nj, const CU
                 rm.adv(kMnSt);
             }
             for (int st = 0; st < 4; st++) {
-                if (!wait_bar(S.w_empty + rw.s, rw.ph ^ 1u, S.abort, a.status)) return;
+                if (!wait_fast(S.w_empty + rw.s, rw.ph ^ 1u, S.abort, a.status)) return;
                 uint8_t *ws = S.w + rw.s * kWStage;
                 mbar_arrive_expect_tx(S.w_full + rw.s, (uint32_t)t.nbox * 4096u);
                 for (int b = 0; b < t.nbox; b++)
@@ -293,7 +302,7 @@ __device__ void role_producer(const GemmArgs &a, const Smem &S, int nj, const CU
     }
 }
 
-// ---------------------------------------------------------------- warps 2-5: unpack
+// ---------------------------------------------------------------- warps 2-9: unpack
 
 // Operand order along K.  Inside every group of 4 consecutive weights the operands hold the
 // elements in the order (0, 2, 1, 3); both sides use the same order, so the products and sums
@@ -329,31 +338,28 @@ __device__ __forceinline__ void scale_pair(int s, uint32_t &s2, uint32_t &nb2) {
     nb2 = *reinterpret_cast<const uint32_t *>(&b);
 }
 
-// Row r's 64 weights of contraction stage st (sub-blocks 2st, 2st+1) as fp16 integers
-// sc_j * q (K-quants) or q (Q8_0), written into the 128-byte-swizzled K-major operand.
+// Row r's 32 weights of sub-block j = 2 st + hsel as fp16 integers sc_j * q (K-quants) or q
+// (Q8_0), written into their half of the 128-byte-swizzled K-major operand row.
 template <int FMT>
-__device__ __forceinline__ void unpack_stage(const uint8_t *rowp, int st, const int *sc,
-                                             bool zero, uint8_t *a16, int r) {
+__device__ __forceinline__ void unpack_half(const uint8_t *rowp, int st, int hsel, int scale,
+                                            bool zero, uint8_t *a16, int r) {
     constexpr uint32_t kM = 0x000F000Fu, kE = 0x64006400u;
-    uint32_t v[32];
+    uint32_t v[16];
     if (FMT == MOE_FMT_Q8_0) {
         // bytes b -> fp16 (1024 + (b ^ 0x80)) - 1152 = b
         const uint32_t k1152 = 0x64806480u;
+        const uint8_t *blk = rowp + 34 * (2 * st + hsel);
+        const uint16_t d16 = *reinterpret_cast<const uint16_t *>(blk);
+        const bool z = zero || d16 == 0 || d16 == 0x8000u;
+        const uint16_t *qp = reinterpret_cast<const uint16_t *>(blk + 2);
 #pragma unroll
-        for (int hb = 0; hb < 2; hb++) {
-            const uint8_t *blk = rowp + 34 * (2 * st + hb);
-            const bool z = zero || *reinterpret_cast<const uint16_t *>(blk) == 0 ||
-                           *reinterpret_cast<const uint16_t *>(blk) == 0x8000u;
-            const uint16_t *qp = reinterpret_cast<const uint16_t *>(blk + 2);
-#pragma unroll
-            for (int wi = 0; wi < 8; wi++) {
-                const uint32_t x = ((uint32_t)qp[2 * wi] | ((uint32_t)qp[2 * wi + 1] << 16)) ^
-                                   0x80808080u;
-                const uint32_t a = hsub2_u(prmt(x, 0x64646464u, 0x4240u), k1152);
-                const uint32_t b = hsub2_u(prmt(x, 0x64646464u, 0x4341u), k1152);
-                v[hb * 16 + 2 * wi] = z ? 0u : a;
-                v[hb * 16 + 2 * wi + 1] = z ? 0u : b;
-            }
+        for (int wi = 0; wi < 8; wi++) {
+            const uint32_t x =
+                ((uint32_t)qp[2 * wi] | ((uint32_t)qp[2 * wi + 1] << 16)) ^ 0x80808080u;
+            const uint32_t a = hsub2_u(prmt(x, 0x64646464u, 0x4240u), k1152);
+            const uint32_t b = hsub2_u(prmt(x, 0x64646464u, 0x4341u), k1152);
+            v[2 * wi] = z ? 0u : a;
+            v[2 * wi + 1] = z ? 0u : b;
         }
     } else {
         const int qs_off = FMT == MOE_FMT_Q5_K ? 48 : 16;
@@ -367,34 +373,27 @@ __device__ __forceinline__ void unpack_stage(const uint8_t *rowp, int st, const 
             hw[0] = ha.x; hw[1] = ha.y; hw[2] = ha.z; hw[3] = ha.w;
             hw[4] = hb2.x; hw[5] = hb2.y; hw[6] = hb2.z; hw[7] = hb2.w;
         }
-        const int j0 = 2 * st;
-        uint32_t s0, n0, s1, n1;
-        scale_pair(zero ? 0 : sc[j0], s0, n0);
-        scale_pair(zero ? 0 : sc[j0 + 1], s1, n1);
+        const int j = 2 * st + hsel, sh = 4 * hsel;   // low nibbles: sub-block 2st, high: 2st+1
+        uint32_t s2, n2;
+        scale_pair(zero ? 0 : scale, s2, n2);
 #pragma unroll
         for (int wi = 0; wi < 8; wi++) {
-            const uint32_t x = qw[wi];
-            uint32_t a = lop3_and_or(x, kM, kE);          // elements k, k+2 of sub-block j0
+            const uint32_t x = qw[wi] >> sh;
+            uint32_t a = lop3_and_or(x, kM, kE);          // elements k, k+2
             uint32_t b = lop3_and_or(x >> 8, kM, kE);     // k+1, k+3
-            uint32_t c = lop3_and_or(x >> 4, kM, kE);     // k, k+2 of sub-block j0+1
-            uint32_t d = lop3_and_or(x >> 12, kM, kE);    // k+1, k+3
             if (FMT == MOE_FMT_Q5_K) {                    // fifth bit -> value bit 4
-                const uint32_t t0 = hw[wi] >> j0, t1 = hw[wi] >> (j0 + 1);
-                a |= (t0 << 4) & 0x00100010u;
-                b |= (t0 >> 4) & 0x00100010u;
-                c |= (t1 << 4) & 0x00100010u;
-                d |= (t1 >> 4) & 0x00100010u;
+                const uint32_t t = hw[wi] >> j;
+                a |= (t << 4) & 0x00100010u;
+                b |= (t >> 4) & 0x00100010u;
             }
-            v[2 * wi] = hfma2_u(a, s0, n0);
-            v[2 * wi + 1] = hfma2_u(b, s0, n0);
-            v[16 + 2 * wi] = hfma2_u(c, s1, n1);
-            v[16 + 2 * wi + 1] = hfma2_u(d, s1, n1);
+            v[2 * wi] = hfma2_u(a, s2, n2);
+            v[2 * wi + 1] = hfma2_u(b, s2, n2);
         }
     }
     uint8_t *rowbase = a16 + (r >> 3) * 1024 + (r & 7) * 128;
 #pragma unroll
-    for (int c = 0; c < 8; c++) {
-        *reinterpret_cast<uint4 *>(rowbase + ((c ^ (r & 7)) << 4)) =
+    for (int c = 0; c < 4; c++) {
+        *reinterpret_cast<uint4 *>(rowbase + (((4 * hsel + c) ^ (r & 7)) << 4)) =
             make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
     }
 }
@@ -403,7 +402,7 @@ template <int FMT>
 __device__ __forceinline__ bool unpack_superblock(const GemmArgs &a, const Smem &S, Ring &rw,
                                                   Ring &rm, Ring &re, const uint8_t *rs,
                                                   float &U, int u) {
-    const int r = u;
+    const int r = u >> 1, hsel = u & 1;        // weight row, sub-block within each stage
     const int lane = threadIdx.x & 31;
     const uint32_t sbb = sb_bytes(FMT);
     const uint8_t *rowp = rs + (size_t)r * sbb;
@@ -428,7 +427,7 @@ __device__ __forceinline__ bool unpack_superblock(const GemmArgs &a, const Smem 
             rt = __fdiv_rn(U, d);
             U = d;
         }
-        ratio[r] = rt;
+        if (hsel == 0) ratio[r] = rt;
     } else {
 #pragma unroll
         for (int j = 0; j < 8; j++) {
@@ -440,10 +439,10 @@ __device__ __forceinline__ bool unpack_superblock(const GemmArgs &a, const Smem 
                 rt = __fdiv_rn(U, dj);
                 U = dj;
             }
-            ratio[j * kTM + r] = rt;
+            if (hsel == 0) ratio[j * kTM + r] = rt;
         }
     }
-    unit[r] = U;
+    if (hsel == 0) unit[r] = U;
     if (u < kTN) {
         const float4 *src = reinterpret_cast<const float4 *>(rs + a.raw_xd_off + u * 32);
         const float4 x0 = src[0], x1 = src[1];
@@ -471,12 +470,15 @@ __device__ __forceinline__ bool unpack_superblock(const GemmArgs &a, const Smem 
             wl[j] = wm - wh[j];
         }
         const int sw = (r >> 2) & 1;
-        float4 *dh = reinterpret_cast<float4 *>(ms + r * 32);
-        float4 *dl = reinterpret_cast<float4 *>(ms + kMnWm + r * 32);
-        dh[0 ^ sw] = make_float4(wh[0], wh[1], wh[2], wh[3]);
-        dh[1 ^ sw] = make_float4(wh[4], wh[5], wh[6], wh[7]);
-        dl[0 ^ sw] = make_float4(wl[0], wl[1], wl[2], wl[3]);
-        dl[1 ^ sw] = make_float4(wl[4], wl[5], wl[6], wl[7]);
+        if (hsel == 0) {
+            float4 *dh = reinterpret_cast<float4 *>(ms + r * 32);
+            dh[0 ^ sw] = make_float4(wh[0], wh[1], wh[2], wh[3]);
+            dh[1 ^ sw] = make_float4(wh[4], wh[5], wh[6], wh[7]);
+        } else {
+            float4 *dl = reinterpret_cast<float4 *>(ms + kMnWm + r * 32);
+            dl[0 ^ sw] = make_float4(wl[0], wl[1], wl[2], wl[3]);
+            dl[1 ^ sw] = make_float4(wl[4], wl[5], wl[6], wl[7]);
+        }
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(S.mn_full + rm.s);
@@ -486,7 +488,7 @@ __device__ __forceinline__ bool unpack_superblock(const GemmArgs &a, const Smem 
     const bool zero = FMT != MOE_FMT_Q8_0 && d == 0.0f;
     for (int st = 0; st < 4; st++) {
         if (!wait_bar_warp(S.w_empty + rw.s, rw.ph ^ 1u, S.abort, a.status)) return false;
-        unpack_stage<FMT>(rowp, st, sc, zero, S.w + rw.s * kWStage, r);
+        unpack_half<FMT>(rowp, st, hsel, sc[2 * st + hsel], zero, S.w + rw.s * kWStage, r);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(S.w_full + rw.s);
@@ -497,7 +499,7 @@ __device__ __forceinline__ bool unpack_superblock(const GemmArgs &a, const Smem 
 
 template <int PHASE>
 __device__ void role_unpack(const GemmArgs &a, const Smem &S, int nj) {
-    const int u = threadIdx.x - 64;              // weight row of the tile, 0..127
+    const int u = threadIdx.x - 64;              // 0..255: row u / 2, sub-block u % 2
     const int lane = threadIdx.x & 31;
     Cursor cur;
     Ring rw, rr, rm, re;
@@ -531,6 +533,11 @@ __device__ void role_mma(const GemmArgs &a, const Smem &S, int nj, uint32_t tbas
     Cursor cur;
     Ring rw, rm, rj, rmin;
     const int nsb = a.K / 256;
+    // Descriptors of stage 0; stage s and sub-block offsets are added to the start-address field
+    // (16-byte units; no carry out of the field since shared addresses stay below 256 KB).
+    const uint64_t dA0 = smem_desc(smem_u32(S.w), 1024, 2);
+    const uint64_t dB0 = smem_desc(smem_u32(S.w) + kA16, 1024, 2);
+    const uint64_t dM0 = smem_desc(smem_u32(S.mn), 256, 6);
     for (int i = blockIdx.x;; i += gridDim.x) {
         Tile t;
         if (!tile_at(a, nj, cur, i, t)) break;
@@ -539,39 +546,34 @@ __device__ void role_mma(const GemmArgs &a, const Smem &S, int nj, uint32_t tbas
         const uint32_t idt = instr_desc(2, kTM, t.n_mma);
         for (int sb = 0; sb < nsb; sb++) {
             for (int st = 0; st < 4; st++) {
-                if (!wait_bar(S.w_full + rw.s, rw.ph, S.abort, a.status)) return;
+                // one 64-wide stage = two sub-blocks, each into its own 64-column accumulator
+                if (!wait_fast(S.w_full + rw.s, rw.ph, S.abort, a.status)) return;
+                if (!wait_fast(S.tm_empty + rj.s, rj.ph ^ 1u, S.abort, a.status)) return;
                 tc_fence_after();
-                const uint32_t a_addr = smem_u32(S.w + rw.s * kWStage);
-                const uint32_t b_addr = a_addr + kA16;
-                for (int jj = 0; jj < 2; jj++) {
-                    if (!wait_bar(S.tm_empty + rj.s, rj.ph ^ 1u, S.abort, a.status)) return;
-                    tc_fence_after();
-                    const uint32_t dt = tbase + rj.s * 64;
-#pragma unroll
-                    for (int kk = 0; kk < 2; kk++) {
-                        const uint32_t off = jj * 64 + kk * 32;
-                        umma_f16(dt, smem_desc(a_addr + off, 1024, 2),
-                                 smem_desc(b_addr + off, 1024, 2), idf, (uint32_t)kk);
-                    }
-                    umma_commit(S.tm_full + rj.s);
-                    rj.adv(kJBuf);
-                }
+                const uint64_t so = (uint64_t)(rw.s * (kWStage >> 4));
+                const uint64_t da = dA0 + so, db = dB0 + so;
+                const uint32_t d0 = tbase + rj.s * 128;
+                umma_f16(d0, da, db, idf, 0u);
+                umma_f16(d0, da + 2, db + 2, idf, 1u);
+                umma_f16(d0 + 64, da + 4, db + 4, idf, 0u);
+                umma_f16(d0 + 64, da + 6, db + 6, idf, 1u);
+                umma_commit(S.tm_full + rj.s);
                 umma_commit(S.w_empty + rw.s);
+                rj.adv(kGrp);
                 rw.adv(kWSt);
             }
             if (kq) {
-                if (!wait_bar(S.mn_full + rm.s, rm.ph, S.abort, a.status)) return;
-                if (sb == 0 && !wait_bar(S.min_empty + rmin.s, rmin.ph ^ 1u, S.abort, a.status))
+                if (!wait_fast(S.mn_full + rm.s, rm.ph, S.abort, a.status)) return;
+                if (sb == 0 && !wait_fast(S.min_empty + rmin.s, rmin.ph ^ 1u, S.abort, a.status))
                     return;
                 tc_fence_after();
-                const uint32_t mb = smem_u32(S.mn + rm.s * kMnStage);
-                const uint32_t wh = mb, wl = mb + kMnWm, xh = mb + 2 * kMnWm,
-                               xl = mb + 2 * kMnWm + kMnXs;
+                const uint64_t mo = (uint64_t)(rm.s * (kMnStage >> 4));
+                const uint64_t wh = dM0 + mo, wl = wh + (kMnWm >> 4), xh = wh + (2 * kMnWm >> 4),
+                               xl = xh + (kMnXs >> 4);
                 const uint32_t dm = tbase + kMinCol0 + rmin.s * 64;
-                umma_tf32(dm, smem_desc(wh, 256, 6), smem_desc(xh, 256, 6), idt,
-                          sb > 0 ? 1u : 0u);
-                umma_tf32(dm, smem_desc(wh, 256, 6), smem_desc(xl, 256, 6), idt, 1u);
-                umma_tf32(dm, smem_desc(wl, 256, 6), smem_desc(xh, 256, 6), idt, 1u);
+                umma_tf32(dm, wh, xh, idt, sb > 0 ? 1u : 0u);
+                umma_tf32(dm, wh, xl, idt, 1u);
+                umma_tf32(dm, wl, xh, idt, 1u);
                 umma_commit(S.mn_empty + rm.s);
                 rm.adv(kMnSt);
             }
@@ -583,7 +585,7 @@ __device__ void role_mma(const GemmArgs &a, const Smem &S, int nj, uint32_t tbas
     }
 }
 
-// ---------------------------------------------------------------- warps 6-13: epilogue
+// ---------------------------------------------------------------- warps 10-17: epilogue
 
 // Q8_1 of 32 consecutive h values of one token (the reading of the quantizer the rest of the
 // library uses), stored as fp16 integers + scales for the down phase, and optionally in the
@@ -656,7 +658,7 @@ template <int PHASE>
 __device__ void role_epilogue(const GemmArgs &a, const Smem &S, int nj, uint32_t tbase) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int q = warp & 3;                  // tensor-memory lane quarter of this warp
-    const int hcol = (warp - 6) >> 2;        // column half: tokens [32 hcol, 32 hcol + 32)
+    const int hcol = (warp - kEpiWarp0) >> 2;  // column half: tokens [32 hcol, 32 hcol + 32)
     const int r = 32 * q + lane;             // weight row of the tile
     const uint32_t lane_addr = (uint32_t)(32 * q) << 16;
     Cursor cur;
@@ -672,12 +674,12 @@ __device__ void role_epilogue(const GemmArgs &a, const Smem &S, int nj, uint32_t
 #pragma unroll
         for (int c = 0; c < 32; c++) acc[c] = 0.f;
         float U = 1.0f;
-        uint32_t P[32];
-        const int nj_tile = nsb * 8;
+        uint32_t P[16];
+        const int nst_tile = nsb * 4;
         const float *xdT = nullptr, *ratio = nullptr, *unit = nullptr;
-        for (int jg = 0; jg < nj_tile; jg++) {
-            const int jj = jg & 7;
-            if (jj == 0) {
+        for (int sg = 0; sg < nst_tile; sg++) {
+            const int st = sg & 3;
+            if (st == 0) {
                 if (!wait_bar_warp(S.ep_full + re.s, re.ph, S.abort, a.status)) return;
                 const uint8_t *es = S.ep + re.s * kEpStage;
                 xdT = reinterpret_cast<const float *>(es);
@@ -692,51 +694,64 @@ __device__ void role_epilogue(const GemmArgs &a, const Smem &S, int nj, uint32_t
             if (!wait_bar_warp(S.tm_full + rj.s, rj.ph, S.abort, a.status)) return;
             tc_fence_after();
             if (active) {
-                tmem_ld32(tbase + lane_addr + rj.s * 64 + 32 * hcol, P);
-                tmem_ld_wait(P);
+                const uint32_t ta = tbase + lane_addr + rj.s * 128 + 32 * hcol;
+#pragma unroll 1
+                for (int h2 = 0; h2 < 2; h2++) {
+                    const int jj = 2 * st + h2;
+                    if (!kq) {
+                        const float rt = ratio[jj * kTM + r];
+#pragma unroll
+                        for (int c = 0; c < 32; c++) acc[c] *= rt;
+                    }
+#pragma unroll
+                    for (int q16 = 0; q16 < 2; q16++) {
+                        tmem_ld16(ta + 64 * h2 + 16 * q16, P);
+                        tmem_ld_wait(P);
+                        const float4 *xd4 =
+                            reinterpret_cast<const float4 *>(xdT + jj * kTN + 32 * hcol + 16 * q16);
+#pragma unroll
+                        for (int c4 = 0; c4 < 4; c4++) {
+                            const float4 x = xd4[c4];
+                            float *ac = acc + 16 * q16 + 4 * c4;
+                            ac[0] = fmaf(__uint_as_float(P[4 * c4 + 0]), x.x, ac[0]);
+                            ac[1] = fmaf(__uint_as_float(P[4 * c4 + 1]), x.y, ac[1]);
+                            ac[2] = fmaf(__uint_as_float(P[4 * c4 + 2]), x.z, ac[2]);
+                            ac[3] = fmaf(__uint_as_float(P[4 * c4 + 3]), x.w, ac[3]);
+                        }
+                    }
+                }
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(S.tm_empty + rj.s);
-            rj.adv(kJBuf);
-            if (active) {
-                if (!kq) {
-                    const float rt = ratio[jj * kTM + r];
-#pragma unroll
-                    for (int c = 0; c < 32; c++) acc[c] *= rt;
-                }
-                const float4 *xd4 = reinterpret_cast<const float4 *>(xdT + jj * kTN + 32 * hcol);
-#pragma unroll
-                for (int c4 = 0; c4 < 8; c4++) {
-                    const float4 x = xd4[c4];
-                    acc[4 * c4 + 0] = fmaf(__uint_as_float(P[4 * c4 + 0]), x.x, acc[4 * c4 + 0]);
-                    acc[4 * c4 + 1] = fmaf(__uint_as_float(P[4 * c4 + 1]), x.y, acc[4 * c4 + 1]);
-                    acc[4 * c4 + 2] = fmaf(__uint_as_float(P[4 * c4 + 2]), x.z, acc[4 * c4 + 2]);
-                    acc[4 * c4 + 3] = fmaf(__uint_as_float(P[4 * c4 + 3]), x.w, acc[4 * c4 + 3]);
-                }
-            }
-            if (jj == 7) {
+            rj.adv(kGrp);
+            if (st == 3) {
                 U = unit[r];
                 __syncwarp();
                 if (lane == 0) mbar_arrive(S.ep_empty + re.s);
                 re.adv(kEpSt);
             }
         }
-        // min term
+        // min term, then the row scale: y = acc * U - min
+#pragma unroll
+        for (int c = 0; c < 32; c++) acc[c] *= U;
         if (kq) {
             if (!wait_bar_warp(S.min_full + rmin.s, rmin.ph, S.abort, a.status)) return;
             tc_fence_after();
             if (active) {
-                tmem_ld32(tbase + lane_addr + kMinCol0 + rmin.s * 64 + 32 * hcol, P);
-                tmem_ld_wait(P);
+#pragma unroll
+                for (int q16 = 0; q16 < 2; q16++) {
+                    tmem_ld16(tbase + lane_addr + kMinCol0 + rmin.s * 64 + 32 * hcol + 16 * q16, P);
+                    tmem_ld_wait(P);
+#pragma unroll
+                    for (int c = 0; c < 16; c++) acc[16 * q16 + c] -= __uint_as_float(P[c]);
+                }
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(S.min_empty + rmin.s);
             rmin.adv(kMinBuf);
         }
-#pragma unroll
-        for (int c = 0; c < 32; c++) acc[c] = acc[c] * U - (kq ? __uint_as_float(P[c]) : 0.0f);
         if (!active) continue;
 
         if (PHASE == 0) {
@@ -798,7 +813,7 @@ __device__ void role_epilogue(const GemmArgs &a, const Smem &S, int nj, uint32_t
 // ---------------------------------------------------------------- the kernel
 
 template <int PHASE>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __maxnreg__(96)
     k_gemm_tc(const GemmArgs a, const __grid_constant__ CUtensorMap map_x,
               const __grid_constant__ CUtensorMap map_d,
               const __grid_constant__ CUtensorMap map_sh,
@@ -811,22 +826,22 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kWSt; i++) {
-            mbar_init(S.w_full + i, 5);
+            mbar_init(S.w_full + i, 1 + kUnpackWarps);
             mbar_init(S.w_empty + i, 1);
         }
         for (int i = 0; i < kRawSt; i++) {
             mbar_init(S.raw_full + i, 1);
-            mbar_init(S.raw_empty + i, 4);
+            mbar_init(S.raw_empty + i, kUnpackWarps);
         }
         for (int i = 0; i < kMnSt; i++) {
-            mbar_init(S.mn_full + i, 5);
+            mbar_init(S.mn_full + i, 1 + kUnpackWarps);
             mbar_init(S.mn_empty + i, 1);
         }
         for (int i = 0; i < kEpSt; i++) {
-            mbar_init(S.ep_full + i, 4);
+            mbar_init(S.ep_full + i, kUnpackWarps);
             mbar_init(S.ep_empty + i, 8);
         }
-        for (int i = 0; i < kJBuf; i++) {
+        for (int i = 0; i < kGrp; i++) {
             mbar_init(S.tm_full + i, 1);
             mbar_init(S.tm_empty + i, 8);
         }
@@ -862,7 +877,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             wait_bar(S.done, 0, S.abort, a.status);
         }
         __syncwarp();
-    } else if (warp < 6) {
+    } else if (warp < kEpiWarp0) {
         role_unpack<PHASE>(a, S, nj);
         __syncwarp();
     } else {
