@@ -12,7 +12,11 @@ A step is one pass of the whole layer (a1-a7) over one batch of synthetic input:
   mixed_prefill one 8192-token chunk, per-expert Q4_K / Q5_K / Q8_0, Zipf(1.3) routing
 The metric is MoE-layer tokens/s (tokens x layers / time); expert bytes read per step (the stored
 bytes of every distinct expert that received a token, plus the shared expert) give the HBM
-fraction; algorithmic int8 ops (2 * 3 * H * F per assignment) give TOPS.
+fraction; algorithmic int8 ops (2 * 3 * H * F per assignment) give TOPS.  The roofline object
+describes the dominant kernel: for decode the fused layer kernel against HBM bandwidth (expert
+bytes per launch / layer time); for prefill the gate/up grouped GEMM against the tensor-core
+peak (2 * assignments * 2F * H flops per launch / its own duration, timed with CUDA events that
+the library records around it in every timed step).
 
 --impl reference times the CPU oracle (the plain fp64 C implementation under oracle/) on the
 same workload, a bounded sample per step, on the host cores: the reference arm of this
@@ -50,6 +54,9 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layers", type=int, default=None,
+                    help="layers per step (default: 48 decode / 4 prefill / 2 mixed_prefill); "
+                         "fewer layers make a smaller case for profilers")
     return ap.parse_args()
 
 
@@ -117,11 +124,13 @@ def traffic_for(kernel: str, workload: str):
 # ------------------------------------------------------------------ workload set-up
 
 
-def workload(name):
+def workload(name, layers=None):
     from expert_ffn_token_b200 import synth
     w = synth.WORKLOADS[name]
     if name in ("prefill", "mixed_prefill"):
         w = synth.with_tokens(w, w.tokens, layers=4 if name == "prefill" else 2)
+    if layers is not None:
+        w = synth.with_tokens(w, w.tokens, layers=layers)
     return w
 
 
@@ -146,7 +155,7 @@ def run_ours(args, rank, world):
 
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
     torch.cuda.set_device(dev)
-    w = workload(args.workload)
+    w = workload(args.workload, args.layers)
     decode = args.workload in ("decode", "mtp_verify")
     K = args.steps if args.steps is not None else (200 if decode else 20)
     W = args.warmup if args.warmup is not None else (10 if decode else 3)
@@ -186,43 +195,74 @@ def run_ours(args, rank, world):
         distinct.append(u)
     del fmts0
 
-    def one_step():
+    def one_step(events=None):
         for l in range(w.layers):
+            if events is not None:
+                moe.set_timing_events(handles[l], *[e.cuda_event for e in events[l]])
             moe.forward(handles[l], x_d[l].data_ptr(), lg_d[l].data_ptr(), T, w.k,
                         out_d[l].data_ptr(), ws.data_ptr(), ws_bytes, 0,
                         torch.cuda.current_stream().cuda_stream)
 
-    # capture one step in a CUDA graph (decode) or run eagerly (prefill: a few launches/step)
-    side = torch.cuda.Stream()
-    side.wait_stream(torch.cuda.current_stream())
-    with torch.cuda.stream(side):
-        one_step()
-    torch.cuda.current_stream().wait_stream(side)
-    torch.cuda.synchronize()
-    n0 = moe.kernels_enqueued()
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph):
-        one_step()
-    kernels_per_step = moe.kernels_enqueued() - n0
-    torch.cuda.synchronize()
+    # decode: one step (48 layers x one launch) captured in a CUDA graph.  Prefill: eager steps
+    # (about ten launches per ~5 ms layer), with CUDA events around the grouped-GEMM kernels of
+    # every layer of every timed step.
+    graph = None
+    kernels_per_step = 0
+    if decode:
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            one_step()
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        n0 = moe.kernels_enqueued()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            one_step()
+        kernels_per_step = moe.kernels_enqueued() - n0
+        torch.cuda.synchronize()
+    step_events = []
+    if not decode:
+        for _ in range(K):
+            row = []
+            for _ in range(w.layers):
+                trio = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+                for e in trio:
+                    e.record()          # creates the handle
+                row.append(trio)
+            step_events.append(row)
+        torch.cuda.synchronize()
+
+    def run(step=None):
+        if graph is not None:
+            graph.replay()
+        else:
+            one_step(step_events[step] if step is not None else None)
 
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
     for _ in range(W):
-        graph.replay()
+        run()
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     clocks = Clocks(os.environ.get("CUDA_VISIBLE_DEVICES", str(dev.index)).split(",")[dev.index]
                     if "CUDA_VISIBLE_DEVICES" in os.environ else dev.index)
+    n0 = moe.kernels_enqueued()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
-    for _ in range(K):
-        graph.replay()
+    for i in range(K):
+        run(i)
     e1.record()
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1)
+    if not decode:
+        kernels_per_step = (moe.kernels_enqueued() - n0) // K
+        for h in handles:
+            moe.set_timing_events(h)
+        gateup_ms = statistics.mean(t[0].elapsed_time(t[1]) for row in step_events for t in row)
+        down_ms = statistics.mean(t[1].elapsed_time(t[2]) for row in step_events for t in row)
     if world > 1:
         t = torch.tensor([ms], device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -237,7 +277,7 @@ def run_ours(args, rank, world):
     for _ in range(2):
         x_d.copy_(x_h, non_blocking=True)
         lg_d.copy_(lg_h, non_blocking=True)
-        graph.replay()
+        run()
         out_h.copy_(out_d, non_blocking=True)
     torch.cuda.synchronize()
     K2 = max(3, K // 4)
@@ -246,7 +286,7 @@ def run_ours(args, rank, world):
     for _ in range(K2):
         x_d.copy_(x_h, non_blocking=True)
         lg_d.copy_(lg_h, non_blocking=True)
-        graph.replay()
+        run()
         out_h.copy_(out_d, non_blocking=True)
     f1.record()
     torch.cuda.synchronize()
@@ -260,17 +300,37 @@ def run_ours(args, rank, world):
     st = moe.read_status(ws.data_ptr(), stream)   # status word sits at workspace offset 0
     if st != 0:
         raise RuntimeError(f"device status {moe.status_string(st)}")
-    del graph
+    graph = None
     for h in handles:
         moe.arena_destroy(h)
 
     tok_per_step = T * w.layers
     ms_step = ms / K
-    value = world * tok_per_step * K / (ms / 1e3)
     hbm, bf16, src = peaks()
-    per_launch_s = ms_step / 1e3 / w.layers
-    bytes_per_launch = step_bytes / w.layers
-    achieved_gbs = bytes_per_launch / per_launch_s / 1e9
+    if decode:
+        per_launch_s = ms_step / 1e3 / w.layers
+        bytes_per_launch = step_bytes / w.layers
+        achieved_gbs = bytes_per_launch / per_launch_s / 1e9
+        roofline = {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm, "unit": "GB/s",
+                    "frac": achieved_gbs / hbm,
+                    "traffic": traffic_for("k_decode_fused", args.workload),
+                    "kernel": "k_decode_fused (one launch per layer)",
+                    "peak_source": src, "bytes_per_launch": bytes_per_launch}
+    else:
+        # dominant kernel: the gate/up grouped GEMM (k_gemm_tc<0>); 2 flops per multiply-add
+        assign = T * (w.k + (1 if w.shared else 0))
+        flops = 2.0 * assign * 2 * w.ffn * w.hidden
+        achieved = flops / (gateup_ms / 1e3) / 1e12
+        roofline = {"bound": "tensor", "achieved": achieved, "peak": bf16, "unit": "TFLOP/s",
+                    "frac": achieved / bf16,
+                    "traffic": traffic_for("k_gemm_tc<0>", args.workload),
+                    "kernel": "k_gemm_tc<0> (gate/up grouped GEMM, kind::f16 with exact integer "
+                              "operands), one launch per layer",
+                    "peak_source": f"{src} bf16 dense (same rate as f16)",
+                    "flops_per_launch": flops, "ms_per_launch": gateup_ms,
+                    "frac_of_int8_peak": achieved / (2 * bf16),
+                    "down_kernel_ms_per_launch": down_ms}
+    value = world * tok_per_step * K / (ms / 1e3)
     result = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
         "warmup": W, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
@@ -285,12 +345,7 @@ def run_ours(args, rank, world):
         "distinct_experts_per_layer": statistics.mean(distinct),
         "expert_gbs": step_bytes / (ms_step / 1e3) / 1e9,
         "int8_tops": step_ops / (ms_step / 1e3) / 1e12,
-        "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm, "unit": "GB/s",
-                     "frac": achieved_gbs / hbm,
-                     "traffic": traffic_for("k_decode_fused", args.workload) if decode else None,
-                     "kernel": "k_decode_fused (one launch per layer)" if decode else
-                               "moe_forward (one layer)",
-                     "peak_source": src, "bytes_per_launch": bytes_per_launch},
+        "roofline": roofline,
         "e2e": {"value": world * tok_per_step * K2 / (ms_e2e / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(xs.nbytes + lgs.nbytes),
                 "d2h_bytes_per_step": int(out_h.numel() * 4)},
@@ -343,7 +398,7 @@ def oracle_sample(w, seconds, max_layers=None):
 
 
 def run_reference(args):
-    w = workload(args.workload)
+    w = workload(args.workload, args.layers)
     K = args.steps if args.steps is not None else 5
     W = args.warmup if args.warmup is not None else 1
     per_step = max(1.0, args.cpu_seconds / max(1, K))
@@ -384,7 +439,7 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
     res = run_ours(args, rank, world)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        res["cpu_baseline"] = oracle_sample(workload(args.workload), args.cpu_seconds)
+        res["cpu_baseline"] = oracle_sample(workload(args.workload, args.layers), args.cpu_seconds)
     if rank == 0:
         print(json.dumps(res), flush=True)
     if world > 1:

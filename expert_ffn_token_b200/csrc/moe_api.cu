@@ -23,6 +23,7 @@ struct moe_arena {
     moe::ExpertDev *d_experts;
     void *d_wmaps;            // tensor maps of the packed matrices (tensor-core path) or null
     bool tc_ok;               // large batches may run on the tensor cores
+    cudaEvent_t ev[3];        // optional timing events around the tensor-core phases
     std::vector<moe_expert_desc> descs;
 };
 
@@ -181,6 +182,7 @@ moe_status moe_arena_create(const void *d_arena, size_t arena_bytes, int hidden,
     A->descs.assign(host_descs, host_descs + n);
     A->d_wmaps = nullptr;
     A->tc_ok = false;
+    A->ev[0] = A->ev[1] = A->ev[2] = nullptr;
     if (cudaMalloc(&A->d_experts, sizeof(ExpertDev) * n) != cudaSuccess ||
         cudaMemcpy(A->d_experts, dev.data(), sizeof(ExpertDev) * n, cudaMemcpyHostToDevice) !=
             cudaSuccess) {
@@ -436,16 +438,19 @@ moe_status moe_forward(const moe_arena *arena, const float *d_x, const float *d_
         if (err == cudaSuccess)
             err = launch_hg_tail_zero(p.hg, p.hgd, p.hgsh, p.hgsl, L.slots, arena->F, L.hpad, st);
         if (err == cudaSuccess && p.keep_h) err = launch_hpad_zero(a, st);
+        if (err == cudaSuccess && !(flags & MOE_F_DETERMINISTIC))
+            err = cudaMemsetAsync(d_out, 0, (size_t)T * H * sizeof(float), st);
+        if (err == cudaSuccess && arena->ev[0]) err = cudaEventRecord(arena->ev[0], st);
         if (err == cudaSuccess) {
             p.phase = 0;
             err = launch_gemm_tc(p, st);
         }
-        if (err == cudaSuccess && !(flags & MOE_F_DETERMINISTIC))
-            err = cudaMemsetAsync(d_out, 0, (size_t)T * H * sizeof(float), st);
+        if (err == cudaSuccess && arena->ev[1]) err = cudaEventRecord(arena->ev[1], st);
         if (err == cudaSuccess) {
             p.phase = 1;
             err = launch_gemm_tc(p, st);
         }
+        if (err == cudaSuccess && arena->ev[2]) err = cudaEventRecord(arena->ev[2], st);
         if (err == cudaSuccess && (flags & MOE_F_DETERMINISTIC))
             err = launch_combine(a, shared != 0, st);
         return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
@@ -464,6 +469,16 @@ moe_status moe_forward(const moe_arena *arena, const float *d_x, const float *d_
         if (err == cudaSuccess) err = launch_down_grouped(a, false, st);
     }
     return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status moe_set_timing_events(moe_arena *arena, void *ev_begin, void *ev_mid, void *ev_end) {
+    if (!arena) return MOE_ERR_INVALID_ARG;
+    if ((ev_begin == nullptr) != (ev_mid == nullptr) || (ev_mid == nullptr) != (ev_end == nullptr))
+        return MOE_ERR_INVALID_ARG;
+    arena->ev[0] = static_cast<cudaEvent_t>(ev_begin);
+    arena->ev[1] = static_cast<cudaEvent_t>(ev_mid);
+    arena->ev[2] = static_cast<cudaEvent_t>(ev_end);
+    return MOE_OK;
 }
 
 moe_status moe_debug_dequant(const moe_arena *arena, int expert, int which, float *d_out,

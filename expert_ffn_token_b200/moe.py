@@ -33,7 +33,7 @@ F_KEEP_H = 8
 EXPORTED = ["moe_arena_create", "moe_arena_destroy", "moe_workspace_size", "moe_quantize_act",
             "moe_route_workspace_size", "moe_route_topk", "moe_forward", "moe_ws_views",
             "moe_read_status", "moe_debug_dequant", "moe_status_string",
-            "moe_kernels_enqueued", "moe_forward_noalloc"]
+            "moe_kernels_enqueued", "moe_forward_noalloc", "moe_set_timing_events"]
 
 
 class ExpertDesc(ctypes.Structure):
@@ -69,6 +69,7 @@ _lib.moe_ws_views.argtypes = [_P, _P, _I, _I, _U, ctypes.POINTER(WsView)]
 _lib.moe_read_status.argtypes = [_P, _P, _I, ctypes.POINTER(_I)]
 _lib.moe_debug_dequant.argtypes = [_P, _I, _I, _P, _P]
 _lib.moe_forward_noalloc.argtypes = [_P, _P, _P, _I, _I, _P, _P, _P]
+_lib.moe_set_timing_events.argtypes = [_P, _P, _P, _P]
 _lib.moe_kernels_enqueued.argtypes = []
 _lib.moe_kernels_enqueued.restype = ctypes.c_uint64
 
@@ -167,6 +168,12 @@ def read_status(d_status: int, stream=None, clear: bool = True) -> int:
     _check(_lib.moe_read_status(d_status, stream, 1 if clear else 0, ctypes.byref(s)),
            "moe_read_status")
     return s.value
+
+
+def set_timing_events(arena: int, ev_begin=None, ev_mid=None, ev_end=None) -> None:
+    """moe_set_timing_events: cudaEvent_t handles (ints) recorded around the tensor-core phases
+    of later forwards on this arena, or None to stop."""
+    _check(_lib.moe_set_timing_events(arena, ev_begin, ev_mid, ev_end), "moe_set_timing_events")
 
 
 def kernels_enqueued() -> int:

@@ -179,6 +179,15 @@ moe_status moe_debug_dequant(const moe_arena *arena, int expert, int which, floa
 moe_status moe_forward_noalloc(const moe_arena *arena, const float *d_x, const float *d_logits,
                                int T, int k, float *d_out, uint32_t *d_status, void *stream);
 
+/* Kernel timing for profilers and benchmarks.  The three events (cudaEvent_t handles created
+ * by the caller, or NULL to stop) are recorded on the stream of every later moe_forward call on
+ * this arena that takes the tensor-core path (T > 16 or MOE_F_FORCE_PREFILL): ev_begin just
+ * before the gate/up projection kernel, ev_mid just after it, ev_end after the down projection
+ * kernel.  cudaEventElapsedTime(ev_begin, ev_mid) is then the gate/up kernel's duration.  The
+ * arena keeps the handles (not owned); calls that use them must not overlap.  The pages have
+ * no counterpart; it serves the measurement of the grouped GEMM alone.                       */
+moe_status moe_set_timing_events(moe_arena *arena, void *ev_begin, void *ev_mid, void *ev_end);
+
 /* Number of kernels this library has enqueued (or recorded into a CUDA graph under stream
  * capture) in this process since it was loaded.  Counting a captured forward gives the
  * kernels each replay of that graph launches. */
