@@ -47,7 +47,7 @@ using namespace ptx;
 
 constexpr int kTM = 128;           // weight rows per tile (MMA M)
 constexpr int kTN = 64;            // tokens per tile (largest MMA N)
-constexpr int kWSt = 4;            // 64-wide contraction stages in flight
+constexpr int kWSt = 2;            // 128-wide contraction stages in flight
 constexpr int kRawSt = 2;          // packed super-block stages
 constexpr int kMnSt = 2;           // min-term operand stages
 constexpr int kEpSt = 2;           // epilogue scale stages
@@ -58,9 +58,11 @@ constexpr int kEpiWarp0 = 2 + kUnpackWarps;
 constexpr int kThreads = (kEpiWarp0 + 8) * 32;
 constexpr uint64_t kWaitNs = 2000000000ull;
 
-constexpr uint32_t kA16 = kTM * 128;                   // 128 rows x 64 fp16
-constexpr uint32_t kB16 = kTN * 128;                   // 64 tokens x 64 fp16
-constexpr uint32_t kWStage = kA16 + kB16;
+// A 128-wide stage holds two 128-byte swizzle atoms of each operand along K:
+// [A atom 0 | A atom 1 | B atom 0 | B atom 1].
+constexpr uint32_t kA16 = kTM * 128;                   // one atom: 128 rows x 64 fp16
+constexpr uint32_t kB16 = kTN * 128;                   // one atom: 64 tokens x 64 fp16
+constexpr uint32_t kWStage = 2 * kA16 + 2 * kB16;
 constexpr uint32_t kRawXd = kTN * 32;                  // 64 tokens x 8 fp32 (xd per sub-block)
 constexpr uint32_t kMnWm = kTM * 32;                   // 128 rows x 8 tf32
 constexpr uint32_t kMnXs = kTN * 32;                   // 64 tokens x 8 tf32
@@ -289,13 +291,14 @@ __device__ void role_producer(const GemmArgs &a, const Smem &S, int nj, const CU
                 }
                 rm.adv(kMnSt);
             }
-            for (int st = 0; st < 4; st++) {
+            for (int st = 0; st < 2; st++) {
                 if (!wait_fast(S.w_empty + rw.s, rw.ph ^ 1u, S.abort, a.status)) return;
-                uint8_t *ws = S.w + rw.s * kWStage;
-                mbar_arrive_expect_tx(S.w_full + rw.s, (uint32_t)t.nbox * 4096u);
-                for (int b = 0; b < t.nbox; b++)
-                    tma_load_2d(ws + kA16 + b * 4096, mx, (sb * 4 + st) * 64,
-                                t.slot_base + 32 * b, S.w_full + rw.s);
+                uint8_t *ws = S.w + rw.s * kWStage + 2 * kA16;
+                mbar_arrive_expect_tx(S.w_full + rw.s, (uint32_t)t.nbox * 8192u);
+                for (int at = 0; at < 2; at++)
+                    for (int b = 0; b < t.nbox; b++)
+                        tma_load_2d(ws + at * kB16 + b * 4096, mx, (sb * 4 + 2 * st + at) * 64,
+                                    t.slot_base + 32 * b, S.w_full + rw.s);
                 rw.adv(kWSt);
             }
         }
@@ -484,11 +487,13 @@ __device__ __forceinline__ bool unpack_superblock(const GemmArgs &a, const Smem 
         if (lane == 0) mbar_arrive(S.mn_full + rm.s);
         rm.adv(kMnSt);
     }
-    // ---- the four 64-wide operand stages
+    // ---- the two 128-wide operand stages (two swizzle atoms, four sub-blocks each)
     const bool zero = FMT != MOE_FMT_Q8_0 && d == 0.0f;
-    for (int st = 0; st < 4; st++) {
+    for (int st = 0; st < 2; st++) {
         if (!wait_bar_warp(S.w_empty + rw.s, rw.ph ^ 1u, S.abort, a.status)) return false;
-        unpack_half<FMT>(rowp, st, hsel, sc[2 * st + hsel], zero, S.w + rw.s * kWStage, r);
+        uint8_t *a16 = S.w + rw.s * kWStage;
+        unpack_half<FMT>(rowp, 2 * st, hsel, sc[4 * st + hsel], zero, a16, r);
+        unpack_half<FMT>(rowp, 2 * st + 1, hsel, sc[4 * st + 2 + hsel], zero, a16 + kA16, r);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(S.w_full + rw.s);
@@ -536,7 +541,7 @@ __device__ void role_mma(const GemmArgs &a, const Smem &S, int nj, uint32_t tbas
     // Descriptors of stage 0; stage s and sub-block offsets are added to the start-address field
     // (16-byte units; no carry out of the field since shared addresses stay below 256 KB).
     const uint64_t dA0 = smem_desc(smem_u32(S.w), 1024, 2);
-    const uint64_t dB0 = smem_desc(smem_u32(S.w) + kA16, 1024, 2);
+    const uint64_t dB0 = smem_desc(smem_u32(S.w) + 2 * kA16, 1024, 2);
     const uint64_t dM0 = smem_desc(smem_u32(S.mn), 256, 6);
     for (int i = blockIdx.x;; i += gridDim.x) {
         Tile t;
@@ -545,21 +550,25 @@ __device__ void role_mma(const GemmArgs &a, const Smem &S, int nj, uint32_t tbas
         const uint32_t idf = instr_desc(0, kTM, t.n_mma);
         const uint32_t idt = instr_desc(2, kTM, t.n_mma);
         for (int sb = 0; sb < nsb; sb++) {
-            for (int st = 0; st < 4; st++) {
-                // one 64-wide stage = two sub-blocks, each into its own 64-column accumulator
+            for (int st = 0; st < 2; st++) {
+                // one 128-wide stage = two swizzle atoms; each atom holds two sub-blocks, each
+                // into its own 64-column accumulator of one group
                 if (!wait_fast(S.w_full + rw.s, rw.ph, S.abort, a.status)) return;
-                if (!wait_fast(S.tm_empty + rj.s, rj.ph ^ 1u, S.abort, a.status)) return;
-                tc_fence_after();
                 const uint64_t so = (uint64_t)(rw.s * (kWStage >> 4));
-                const uint64_t da = dA0 + so, db = dB0 + so;
-                const uint32_t d0 = tbase + rj.s * 128;
-                umma_f16(d0, da, db, idf, 0u);
-                umma_f16(d0, da + 2, db + 2, idf, 1u);
-                umma_f16(d0 + 64, da + 4, db + 4, idf, 0u);
-                umma_f16(d0 + 64, da + 6, db + 6, idf, 1u);
-                umma_commit(S.tm_full + rj.s);
+#pragma unroll
+                for (int at = 0; at < 2; at++) {
+                    if (!wait_fast(S.tm_empty + rj.s, rj.ph ^ 1u, S.abort, a.status)) return;
+                    tc_fence_after();
+                    const uint64_t da = dA0 + so + at * (kA16 >> 4), db = dB0 + so + at * (kB16 >> 4);
+                    const uint32_t d0 = tbase + rj.s * 128;
+                    umma_f16(d0, da, db, idf, 0u);
+                    umma_f16(d0, da + 2, db + 2, idf, 1u);
+                    umma_f16(d0 + 64, da + 4, db + 4, idf, 0u);
+                    umma_f16(d0 + 64, da + 6, db + 6, idf, 1u);
+                    umma_commit(S.tm_full + rj.s);
+                    rj.adv(kGrp);
+                }
                 umma_commit(S.w_empty + rw.s);
-                rj.adv(kGrp);
                 rw.adv(kWSt);
             }
             if (kq) {
