@@ -6,6 +6,7 @@
 //   word(k, n) = mix64(k + (n + 1) * 0x9E3779B97F4A7C15)
 //   raw byte p of a tensor  = byte p % 8 of word(k_raw, p / 8)
 //   block i's d (and dmin)  = fp16(fp32(1e-3 + 9e-3 * (word(k_d, i) >> 11) * 2^-53))
+//   Q5_1 block i's offset m = -16 * its dmin draw (exact in fp16)
 // K-quant blocks that end past the row's logical width get scale and min 0 for the sub-blocks
 // past it; pad bytes after a row's last block are 0.  The per-tensor keys are computed on the
 // host and passed in.
@@ -19,8 +20,9 @@ typedef struct {
     uint64_t key_raw, key_d, key_dmin;
     int32_t rows, stride;   // row count, row stride in bytes (multiple of 16)
     int32_t nblocks;        // blocks per row
-    int32_t block_bytes;    // 144, 176 or 34
-    int32_t kquant;         // 1: d and dmin at bytes 0-3 and packed scales at 4-15; 0: Q8_0
+    int32_t block_bytes;    // 144, 176, 34 or 24
+    int32_t kquant;         // 1: d and dmin at bytes 0-3 and packed scales at 4-15; 0: Q8_0;
+                            // 2: Q5_1 (d and m = -16 * dmin draw at bytes 0-3)
     int32_t valid_last;     // sub-blocks of the last block inside the logical width (8 = all)
 } synth_tensor;
 }
@@ -81,9 +83,12 @@ __global__ void k_synth_fill(uint8_t *dst, const synth_tensor *tensors) {
                 const uint64_t i = row * T.nblocks + blk;
                 if (o < 2) {
                     v = (scale_half(word(T.key_d, i)) >> (8 * o)) & 0xFFu;
-                } else if (T.kquant && o < 4) {
+                } else if (T.kquant == 2 && o < 4) {
+                    const uint32_t m = (scale_half(word(T.key_dmin, i)) + (4u << 10)) | 0x8000u;
+                    v = (m >> (8 * (o - 2))) & 0xFFu;
+                } else if (T.kquant == 1 && o < 4) {
                     v = (scale_half(word(T.key_dmin, i)) >> (8 * (o - 2))) & 0xFFu;
-                } else if (T.kquant && o < 16 && blk == T.nblocks - 1 && T.valid_last < 8) {
+                } else if (T.kquant == 1 && o < 16 && blk == T.nblocks - 1 && T.valid_last < 8) {
                     v = kill_scale_byte(v, o, T.valid_last);
                 }
             }

@@ -23,6 +23,7 @@ Weight tensors of expert e in layer l (tensor t: 0 gate, 1 up, 2 down), rows of 
     block i (= row * blocks + col // block_bytes):
         d    = fp16(fp32(1e-3 + 9e-3 * uniform(key(seed, l, e, t, 1), i)))   bytes 0-1
         dmin = fp16(fp32(1e-3 + 9e-3 * uniform(key(seed, l, e, t, 2), i)))   bytes 2-3 (K-quants)
+        m    = -16 * dmin (exact in fp16)                                  bytes 2-3 (Q5_1)
     K-quant blocks that run past the row's logical width (down rows of width 640 stored as
     768) get scale and min 0 for the sub-blocks past the width, so those weights are exactly 0.
     Pad bytes after the last block of a row are 0.
@@ -33,7 +34,7 @@ N(0, sigma) (key(seed, l, 102, attempt)) or Zipf(s) popularity plus Gumbel noise
 key(seed, l, 103), noise from key(seed, l, 104, attempt)); a token's row is drawn again with
 the next attempt until every adjacent gap among its k+1 largest fp32 logits is >= 1e-3.
 Per-expert formats (mixed workload): uniform(key(seed, l, 105), e) < 0.60 Q4_K, < 0.85 Q5_K,
-else Q8_0.
+else Q8_0; a workload's `mix` can give other thresholds and Q5_1.
 """
 from __future__ import annotations
 
@@ -42,10 +43,10 @@ from dataclasses import dataclass, field
 
 import numpy as np
 
-Q4_K, Q5_K, Q8_0 = 0, 1, 2
-FMT_NAMES = {Q4_K: "Q4_K", Q5_K: "Q5_K", Q8_0: "Q8_0"}
-BLOCK_WEIGHTS = {Q4_K: 256, Q5_K: 256, Q8_0: 32}
-BLOCK_BYTES = {Q4_K: 144, Q5_K: 176, Q8_0: 34}
+Q4_K, Q5_K, Q8_0, Q5_1 = 0, 1, 2, 3
+FMT_NAMES = {Q4_K: "Q4_K", Q5_K: "Q5_K", Q8_0: "Q8_0", Q5_1: "Q5_1"}
+BLOCK_WEIGHTS = {Q4_K: 256, Q5_K: 256, Q8_0: 32, Q5_1: 32}
+BLOCK_BYTES = {Q4_K: 144, Q5_K: 176, Q8_0: 34, Q5_1: 24}
 TENSOR_ALIGN = 256
 
 G = np.uint64(0x9E3779B97F4A7C15)
@@ -245,7 +246,12 @@ def tensor_bytes(w: Workload, layer: int, e: int, t: int, fmt: int) -> np.ndarra
     d = scale_to_half(uniform(key(w.seed, layer, e, t, 1), 0, nblk)).reshape(rows, nb)
     blocks[:, :, 0] = (d & 0xFF).astype(np.uint8)
     blocks[:, :, 1] = (d >> 8).astype(np.uint8)
-    if fmt != Q8_0:
+    if fmt == Q5_1:
+        dm = scale_to_half(uniform(key(w.seed, layer, e, t, 2), 0, nblk)).reshape(rows, nb)
+        mm = (dm + np.uint16(4 << 10)) | np.uint16(0x8000)      # -16 * dmin: exponent + 4, sign
+        blocks[:, :, 2] = (mm & 0xFF).astype(np.uint8)
+        blocks[:, :, 3] = (mm >> 8).astype(np.uint8)
+    elif fmt != Q8_0:
         dm = scale_to_half(uniform(key(w.seed, layer, e, t, 2), 0, nblk)).reshape(rows, nb)
         blocks[:, :, 2] = (dm & 0xFF).astype(np.uint8)
         blocks[:, :, 3] = (dm >> 8).astype(np.uint8)
@@ -414,8 +420,8 @@ def device_fill_layer(w: Workload, layer: int, d_base: int, stream=None) -> Aren
             r.stride = int(lay.strides[e, t])
             r.nblocks = nb
             r.block_bytes = BLOCK_BYTES[f]
-            r.kquant = 0 if f == Q8_0 else 1
-            r.valid_last = 8 if f == Q8_0 else (width - (nb - 1) * 256) // 32
+            r.kquant = {Q8_0: 0, Q5_1: 2}.get(f, 1)
+            r.valid_last = 8 if f in (Q8_0, Q5_1) else (width - (nb - 1) * 256) // 32
     rc = _synth().synth_fill_tensors(d_base, ctypes.cast(tab, ctypes.c_void_p), lay.n * 3, stream)
     if rc != 0:
         raise RuntimeError(f"synth_fill_tensors failed ({rc})")

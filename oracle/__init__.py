@@ -21,7 +21,7 @@ _HERE = Path(__file__).resolve().parent
 _SRC = _HERE / "moe_oracle.c"
 _LIB = _HERE / "liboracle.so"
 
-FMT_Q4_K, FMT_Q5_K, FMT_Q8_0 = 0, 1, 2
+FMT_Q4_K, FMT_Q5_K, FMT_Q8_0, FMT_Q5_1 = 0, 1, 2, 3
 
 _lib = None
 

@@ -9,11 +9,11 @@
  * What it computes (the layer of "Strata: a 125B MoE at 94 tok/s on a 12 GB Card", section
  * "Three architecture facts": experts per layer, routed + shared; the per-expert formats of the
  * "Strata v0.1.31" release notes, section "Experimental: Unsloth UD-Q4_K_XL on a normal PC":
- * Q4_K, Q5_K and Q8_0 experts whose dequantizers follow llama.cpp's bit for bit; the q8_1
+ * Q4_K, Q5_K, Q5_1 and Q8_0 experts whose dequantizers follow llama.cpp's bit for bit; the q8_1
  * activations of the "Strata v0.1.39" release notes, fixes list, #606):
  *
- *   O1  block decode (Q4_K, Q5_K, Q8_0) to exact fp64 and to the fp32 value
- *       RN32( RN32(d*sc)*q - RN32(dmin*m) )             (Q8_0: RN32(d*q))
+ *   O1  block decode (Q4_K, Q5_K, Q5_1, Q8_0) to exact fp64 and to the fp32 value
+ *       RN32( RN32(d*sc)*q - RN32(dmin*m) )             (Q8_0: RN32(d*q); Q5_1: RN32(d*q + m))
  *   O2  Q8_1 quantization of 32-value blocks: amax, d = amax/127 (fp32 division),
  *       q = round-half-away(x/d) clamped to [-127,127], stored d16 = fp16(d),
  *       s16 = fp16(d * sum(q)); a block holding a non-finite value becomes all zero
@@ -41,14 +41,16 @@
 #include <omp.h>
 #endif
 
-enum { ORC_Q4_K = 0, ORC_Q5_K = 1, ORC_Q8_0 = 2 };
+enum { ORC_Q4_K = 0, ORC_Q5_K = 1, ORC_Q8_0 = 2, ORC_Q5_1 = 3 };
 
 /* weights and bytes per block of each format */
-static int orc_block_weights(int fmt) { return fmt == ORC_Q8_0 ? 32 : 256; }
-static int orc_block_bytes(int fmt) { return fmt == ORC_Q4_K ? 144 : fmt == ORC_Q5_K ? 176 : 34; }
+static int orc_block_weights(int fmt) { return fmt == ORC_Q8_0 || fmt == ORC_Q5_1 ? 32 : 256; }
+static int orc_block_bytes(int fmt) {
+    return fmt == ORC_Q4_K ? 144 : fmt == ORC_Q5_K ? 176 : fmt == ORC_Q8_0 ? 34 : 24;
+}
 
-int oracle_block_weights(int fmt) { return fmt >= 0 && fmt <= 2 ? orc_block_weights(fmt) : -1; }
-int oracle_block_bytes(int fmt) { return fmt >= 0 && fmt <= 2 ? orc_block_bytes(fmt) : -1; }
+int oracle_block_weights(int fmt) { return fmt >= 0 && fmt <= 3 ? orc_block_weights(fmt) : -1; }
+int oracle_block_bytes(int fmt) { return fmt >= 0 && fmt <= 3 ? orc_block_bytes(fmt) : -1; }
 
 /* ---------------------------------------------------------------- IEEE binary16 <-> binary64 */
 
@@ -109,8 +111,25 @@ static void orc_kquant_scale_min(const uint8_t *S, int j, int *sc, int *m) {
  *   r >= 32 -> sub-block 2c+1, q = high nibble of qs[32c + r - 32].
  * Q5_K (176 B): d, dmin, S as Q4_K; qh[32] (16-47); qs[128] (48-175); the fifth bit of
  *   element n is bit (2c) of qh[r] for r < 32 and bit (2c+1) of qh[r-32] for r >= 32.
- * Q8_0 (34 B): d (fp16), q[32] int8.                                                          */
+ * Q8_0 (34 B): d (fp16), q[32] int8.
+ * Q5_1 (24 B): d, m (fp16, bytes 0-3), qh (32 bits, little endian, bytes 4-7), qs[16] (8-23);
+ *   element n < 16: q = low nibble of qs[n], n >= 16: high nibble of qs[n-16]; bit n of qh is
+ *   the fifth bit of element n; w = d*q + m (d*q has <= 16 significant bits, so the fp32 value
+ *   is RN32(d*q + m) whether or not the multiply-add is fused).                               */
 static void orc_decode_block(int fmt, const uint8_t *b, double *w64, float *w32) {
+    if (fmt == ORC_Q5_1) {
+        double d = orc_half_to_double((uint16_t)(b[0] | (b[1] << 8)));
+        double m = orc_half_to_double((uint16_t)(b[2] | (b[3] << 8)));
+        uint32_t qh = (uint32_t)b[4] | ((uint32_t)b[5] << 8) | ((uint32_t)b[6] << 16) |
+                      ((uint32_t)b[7] << 24);
+        for (int n = 0; n < 32; n++) {
+            int q = n < 16 ? (b[8 + n] & 15) : (b[8 + n - 16] >> 4);
+            q |= (int)((qh >> n) & 1u) << 4;
+            w64[n] = d * q + m;
+            if (w32) w32[n] = fmaf((float)d, (float)q, (float)m);
+        }
+        return;
+    }
     if (fmt == ORC_Q8_0) {
         double d = orc_half_to_double((uint16_t)(b[0] | (b[1] << 8)));
         for (int n = 0; n < 32; n++) {
@@ -147,7 +166,7 @@ static void orc_decode_block(int fmt, const uint8_t *b, double *w64, float *w32)
 
 /* O1 over a packed row of nblocks blocks.  Returns 0, or -1 for an unknown format. */
 int oracle_dequant_row(int fmt, const uint8_t *row, int64_t nblocks, double *w64, float *w32) {
-    if (fmt < 0 || fmt > 2) return -1;
+    if (fmt < 0 || fmt > 3) return -1;
     int bw = orc_block_weights(fmt), bb = orc_block_bytes(fmt);
     for (int64_t i = 0; i < nblocks; i++)
         orc_decode_block(fmt, row + i * bb, w64 + i * bw, w32 ? w32 + i * bw : NULL);
@@ -245,6 +264,7 @@ int oracle_topk(const float *logits, int T, int E, int k, int32_t *ids, float *w
 int oracle_group(const int32_t *ids, int T, int k, int E, int32_t *counts, int32_t *offsets,
                  int32_t *perm, int32_t *inv_perm) {
     int64_t A = (int64_t)T * k;
+    if (E <= 0 || T < 0 || k < 0) return -1;
     for (int e = 0; e < E; e++) counts[e] = 0;
     for (int64_t a = 0; a < A; a++) {
         if (ids[a] < 0 || ids[a] >= E) return -1;
@@ -253,6 +273,7 @@ int oracle_group(const int32_t *ids, int T, int k, int E, int32_t *counts, int32
     offsets[0] = 0;
     for (int e = 0; e < E; e++) offsets[e + 1] = offsets[e] + counts[e];
     int32_t *fill = (int32_t *)calloc((size_t)E, sizeof(int32_t));
+    if (!fill) return -1;
     for (int64_t a = 0; a < A; a++) {               /* ascending a = ascending t, then j */
         int e = ids[a];
         int64_t i = offsets[e] + fill[e]++;
@@ -265,7 +286,7 @@ int oracle_group(const int32_t *ids, int T, int k, int E, int32_t *counts, int32
 
 /* ------------------------------------------------------------------------ O5-O9: the FFN */
 
-/* One expert's three matrices inside a host arena.  fmt: 0 Q4_K, 1 Q5_K, 2 Q8_0.
+/* One expert's three matrices inside a host arena.  fmt: 0 Q4_K, 1 Q5_K, 2 Q8_0, 3 Q5_1.
  * gate, up: ffn rows of hidden weights; down: hidden rows of ffn weights (padded to whole
  * blocks).  Offsets and row strides are in bytes.                                             */
 typedef struct {
@@ -303,7 +324,7 @@ int oracle_expert_ffn(const uint8_t *arena, const oracle_expert *ex, int hidden,
                       const double *xhat, double *g, double *u, double *h, int8_t *hq,
                       uint16_t *hd, uint16_t *hs, double *y) {
     int fmt = ex->fmt;
-    if (fmt < 0 || fmt > 2) return -1;
+    if (fmt < 0 || fmt > 3) return -1;
     int bw = orc_block_weights(fmt);
     if (hidden % bw) return -1;
     int64_t fp = orc_padded(fmt, ffn);

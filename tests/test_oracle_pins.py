@@ -78,6 +78,54 @@ def test_q8_0_hand_decoded_block():
         assert w64[int(n)] == v, n
 
 
+def _q5_1_block(d16, m16, qh=0, qs=None):
+    b = bytearray(24)
+    b[0:2] = d16.to_bytes(2, "little")
+    b[2:4] = m16.to_bytes(2, "little")
+    b[4:8] = qh.to_bytes(4, "little")
+    for i, v in (qs or {}).items():
+        b[8 + i] = v
+    return np.frombuffer(bytes(b), np.uint8)
+
+
+def test_q5_1_hand_decoded_block():
+    g = _load("q5_1_e5.json")
+    blk = _q5_1_block(int(g["block"]["d"], 16), int(g["block"]["m"], 16), int(g["block"]["qh"], 16),
+                      {int(i): int(v, 16) for i, v in g["block"]["qs_nonzero"].items()})
+    w64, w32 = oracle.dequant_row(oracle.FMT_Q5_1, blk)
+    for n, v in g["expected"].items():
+        assert w64[int(n)] == v and w32[int(n)] == np.float32(v), n
+    # every other element has q = 0 and equals the offset m
+    for n in range(32):
+        if str(n) not in g["expected"] and n not in (0, 1, 15, 16, 17, 31):
+            assert w64[n] == -2.0, n
+
+
+def test_q5_1_nibble_and_fifth_bit_every_element():
+    # d = 1, m = 0: one nibble or one qh bit at a time lights exactly one element
+    for byte in range(16):
+        for hi in (0, 1):
+            w, _ = oracle.dequant_row(oracle.FMT_Q5_1,
+                                      _q5_1_block(0x3C00, 0, 0, {byte: 0x70 if hi else 0x07}))
+            (nz,) = np.nonzero(w)
+            assert list(nz) == [byte + 16 * hi] and w[byte + 16 * hi] == 7
+    for bit in range(32):
+        w, _ = oracle.dequant_row(oracle.FMT_Q5_1, _q5_1_block(0x3C00, 0, 1 << bit))
+        (nz,) = np.nonzero(w)
+        assert list(nz) == [bit] and w[bit] == 16
+
+
+def test_q5_1_offset_rounds_once_in_fp32():
+    # d = 1024, q = 31 (all bits set), m = 2^-14: the exact value 31744 + 2^-14 needs 29 bits,
+    # so the fp32 weight is 31744 (one rounding) while the fp64 value keeps the offset
+    w64, w32 = oracle.dequant_row(oracle.FMT_Q5_1,
+                                  _q5_1_block(0x6400, 0x0400, 0xFFFFFFFF, {i: 0xFF for i in range(16)}))
+    assert (w64 == 31744 + 2.0 ** -14).all() and (w32 == 31744.0).all()
+    # negative offset with d = 0: the block is the constant m
+    w64, _ = oracle.dequant_row(oracle.FMT_Q5_1, _q5_1_block(0, 0xBC00, 0x12345678, {3: 0x9A}))
+    assert (w64 == -1.0).all()
+
+
 def _pack_scales(sc, m):
     """Inverse of the 6-bit scale/min unpacking: 8 (sc, m) pairs -> 12 bytes."""
     S = [0] * 12
@@ -149,13 +197,17 @@ def _f16(bits):
 
 def test_dequant_exact_rational_and_single_rounding():
     rng = np.random.default_rng(11)
-    for fmt, bb in ((oracle.FMT_Q4_K, 144), (oracle.FMT_Q5_K, 176), (oracle.FMT_Q8_0, 34)):
+    for fmt, bb in ((oracle.FMT_Q4_K, 144), (oracle.FMT_Q5_K, 176), (oracle.FMT_Q8_0, 34),
+                    (oracle.FMT_Q5_1, 24)):
         raw = rng.integers(0, 256, size=bb * 64, dtype=np.uint8)
         # scales in the generator's range and a few extremes
         for i in range(64):
             d = np.float16(rng.uniform(1e-3, 1e-2)) if i % 8 else np.float16(rng.uniform(1, 100))
             raw[i * bb:i * bb + 2] = np.array([d]).view(np.uint8)
-            if fmt != oracle.FMT_Q8_0:
+            if fmt == oracle.FMT_Q5_1:
+                mm = np.float16(-rng.uniform(1e-3, 0.5))
+                raw[i * bb + 2:i * bb + 4] = np.array([mm]).view(np.uint8)
+            elif fmt != oracle.FMT_Q8_0:
                 dm = np.float16(rng.uniform(1e-3, 1e-2))
                 raw[i * bb + 2:i * bb + 4] = np.array([dm]).view(np.uint8)
         w64, w32 = oracle.dequant_row(fmt, raw)
@@ -165,8 +217,13 @@ def test_dequant_exact_rational_and_single_rounding():
         for i in range(64):
             blk = raw[i * bb:(i + 1) * bb]
             d = _f16(int(blk[0]) | int(blk[1]) << 8)
-            vals = [Fraction(float(v)) for v in w64[i * (32 if fmt == 2 else 256):][:8]]
-            if fmt == oracle.FMT_Q8_0:
+            vals = [Fraction(float(v)) for v in w64[i * (32 if fmt >= 2 else 256):][:8]]
+            if fmt == oracle.FMT_Q5_1:
+                mm = _f16(int(blk[2]) | int(blk[3]) << 8)
+                qh = int.from_bytes(bytes(blk[4:8]), "little")
+                for n, v in enumerate(vals):
+                    assert v == d * ((int(blk[8 + n]) & 15) | ((qh >> n) & 1) << 4) + mm
+            elif fmt == oracle.FMT_Q8_0:
                 for n, v in enumerate(vals):
                     assert v == d * int(np.int8(blk[2 + n]))
             else:
@@ -343,6 +400,9 @@ def _q8_1_values(v):
     (1, None, 512, 384, 6, 3, 4, True),                       # down rows padded 384 -> 512
     (2, ((synth.Q8_0, 1.0),), 256, 160, 5, 2, 3, True),      # Q8_0, width 160
     (3, ((synth.Q4_K, 0.3), (synth.Q5_K, 0.7), (synth.Q8_0, 1.0)), 512, 640, 12, 4, 5, True),
+    (4, ((synth.Q5_1, 1.0),), 256, 160, 5, 2, 3, True),      # Q5_1, width 160
+    (5, ((synth.Q4_K, 0.25), (synth.Q5_K, 0.5), (synth.Q8_0, 0.75), (synth.Q5_1, 1.0)),
+     512, 640, 12, 4, 5, True),
 ])
 def test_forward_matches_dense_fp64(case):
     idx, mix, H, F, E, k, T, shared = case
@@ -439,3 +499,26 @@ def test_q8_1_uses_ieee_fp32_division():
         assert np.array_equal(q, q_ieee.astype(np.int8))
         cases += 1
     assert cases >= 20
+
+
+def test_generator_q5_1_blocks():
+    # Q5_1 tensors: d from the scale draw, m = -16 * the dmin draw (both fp16), so every weight
+    # lies in [m, m + 31 d] and the block's offset is negative
+    w = _tiny(((synth.Q5_1, 1.0),), 256, 96, 3, 1, 2, False, 6)
+    arena, lay = synth.host_arena(w, 0)
+    assert (lay.fmts == synth.Q5_1).all() and lay.strides[0, 0] == 8 * 24 and lay.strides[0, 2] == 80
+    for e in range(lay.n):
+        for t in range(3):
+            rows, width = synth.tensor_shape(w, t)
+            nb = synth.row_blocks(synth.Q5_1, width)
+            st = int(lay.strides[e, t])
+            mat = arena[lay.offs[e, t]:lay.offs[e, t] + rows * st].reshape(rows, st)
+            assert not mat[:, nb * 24:].any()
+            blk = mat[:, :nb * 24].reshape(rows, nb, 24)
+            d = blk[:, :, 0:2].copy().view(np.float16)[..., 0].astype(np.float64)
+            m = blk[:, :, 2:4].copy().view(np.float16)[..., 0].astype(np.float64)
+            assert (d >= 1e-3 * 0.999).all() and (d <= 1e-2 * 1.001).all()
+            assert (m <= -16e-3 * 0.999).all() and (m >= -0.16 * 1.001).all()
+            W, _ = oracle.dequant_matrix(synth.Q5_1, mat.ravel(), rows, st, nb)
+            lo = np.repeat(m, 32, axis=1)
+            assert (W >= lo).all() and (W <= lo + 31 * np.repeat(d, 32, axis=1)).all()
