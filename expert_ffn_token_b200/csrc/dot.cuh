@@ -1,9 +1,10 @@
-// dot.cuh -- per-lane partial dot products of packed K-quant / Q8_0 rows with Q8_1 activations,
-// and the small warp-level helpers the FFN kernels share.
+// dot.cuh -- per-lane partial dot products of packed K-quant / Q8_0 / Q5_1 rows with Q8_1
+// activations, and the small warp-level helpers the FFN kernels share.
 //
 // For a sub-block of 32 weights w = d*sc*q - dmin*m and Q8_1 activations xd*qx, the dot is
 //   d*sc*xd*sum(q*qx) - dmin*m*(xd*sum qx)
-// where xd*sum(qx) is kept exactly in fp32 per activation block ("xsum").
+// where xd*sum(qx) is kept exactly in fp32 per activation block ("xsum").  A Q5_1 block
+// (w = d*q + m) is the same with sc = 1 and the offset added: d*xd*sum(q*qx) + m*(xd*sum qx).
 #pragma once
 
 #include "moe_internal.cuh"
@@ -16,6 +17,14 @@ __device__ __forceinline__ uint4 ld_stream16(const uint8_t *p) {
     uint4 v;
     asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
                  : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ uint2 ld_stream8(const uint8_t *p) {
+    uint2 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];"
+                 : "=r"(v.x), "=r"(v.y)
                  : "l"(p));
     return v;
 }
@@ -138,6 +147,52 @@ __device__ __forceinline__ float q80_dot(const Q80Block &w, const int8_t *xq, fl
     return w.d * xd * (float)acc;
 }
 
+// Q5_1 block b of a row (24-byte blocks; rows start 16-byte aligned, so every block is 8-byte
+// aligned): its 32 five-bit quants as bytes (elements 4i..4i+3 in word i) and d, m.
+struct Q51Block {
+    uint32_t w[8];
+    float d, m;
+};
+
+// Four consecutive bits of qh to bit 4 of four consecutive bytes.
+__device__ __forceinline__ uint32_t q51_fifth(uint32_t qh, int n0) {
+    return (((qh >> n0) & 0xFu) * 0x00204081u & 0x01010101u) << 4;
+}
+
+__device__ __forceinline__ Q51Block q51_unpack(uint2 h, uint2 a, uint2 c) {
+    Q51Block r;
+    r.d = half_bits_to_float(h.x & 0xFFFFu);
+    r.m = half_bits_to_float(h.x >> 16);
+    const uint32_t qh = h.y;
+    const uint32_t qs[4] = {a.x, a.y, c.x, c.y};
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+        r.w[i] = (qs[i] & 0x0F0F0F0Fu) | q51_fifth(qh, 4 * i);
+        r.w[4 + i] = ((qs[i] >> 4) & 0x0F0F0F0Fu) | q51_fifth(qh, 16 + 4 * i);
+    }
+    return r;
+}
+
+__device__ __forceinline__ Q51Block q51_load(const uint8_t *row, int b) {
+    const uint8_t *p = row + (size_t)b * kQ51Bytes;
+    return q51_unpack(ld_stream8(p), ld_stream8(p + 8), ld_stream8(p + 16));
+}
+
+// sum over the block of (d*q + m) * (xd*qx) = d*xd*sum(q*qx) + m*xs, xs = xd*sum(qx) exact.
+__device__ __forceinline__ float q51_dot(const Q51Block &w, const int8_t *xq, float xd, float xs) {
+    const int4 a = *reinterpret_cast<const int4 *>(xq);
+    const int4 b = *reinterpret_cast<const int4 *>(xq + 16);
+    int acc = __dp4a((int)w.w[0], a.x, 0);
+    acc = __dp4a((int)w.w[1], a.y, acc);
+    acc = __dp4a((int)w.w[2], a.z, acc);
+    acc = __dp4a((int)w.w[3], a.w, acc);
+    acc = __dp4a((int)w.w[4], b.x, acc);
+    acc = __dp4a((int)w.w[5], b.y, acc);
+    acc = __dp4a((int)w.w[6], b.z, acc);
+    acc = __dp4a((int)w.w[7], b.w, acc);
+    return fmaf(w.d * xd, (float)acc, w.m * xs);
+}
+
 // Whole-row partial dots for NT activation rows (lane's share; reduce across the warp after).
 // x[t] for t < nt are valid; the rest are ignored.
 template <int FMT, int NT>
@@ -150,6 +205,15 @@ __device__ __forceinline__ void row_parts(const uint8_t *row, int K, const ActRo
 #pragma unroll
             for (int t = 0; t < NT; t++)
                 if (t < nt) acc[t] += q80_dot(w, x[t].q + 32 * b, x[t].d[b]);
+        }
+        return;
+    }
+    if (FMT == MOE_FMT_Q5_1) {
+        for (int b = lane; b < K / 32; b += 32) {
+            const Q51Block w = q51_load(row, b);
+#pragma unroll
+            for (int t = 0; t < NT; t++)
+                if (t < nt) acc[t] += q51_dot(w, x[t].q + 32 * b, x[t].d[b], x[t].s[b]);
         }
         return;
     }
@@ -188,7 +252,8 @@ __device__ __forceinline__ void row_parts_fmt(int fmt, const uint8_t *row, int K
                                               int nt, float *acc) {
     if (fmt == MOE_FMT_Q4_K) row_parts<MOE_FMT_Q4_K, NT>(row, K, x, nt, acc);
     else if (fmt == MOE_FMT_Q5_K) row_parts<MOE_FMT_Q5_K, NT>(row, K, x, nt, acc);
-    else row_parts<MOE_FMT_Q8_0, NT>(row, K, x, nt, acc);
+    else if (fmt == MOE_FMT_Q8_0) row_parts<MOE_FMT_Q8_0, NT>(row, K, x, nt, acc);
+    else row_parts<MOE_FMT_Q5_1, NT>(row, K, x, nt, acc);
 }
 
 // Q8_1 of 32 values, one per lane (the h of one 32-row block of one slot).

@@ -74,22 +74,25 @@ struct DecParams {
 //
 // A K-quant row is cut into 16-byte quant chunks p = 8*sb + j (sb super-block, j = 0..7,
 // c = j/2, hh = j%2): chunk p holds elements 64c+16hh+[0,16) (low nibbles, sub-block 2c) and
-// 64c+32+16hh+[0,16) (high nibbles, sub-block 2c+1) of super-block sb.  A Q8_0 row is cut
-// into its 32-weight blocks (chunk p = block p).
+// 64c+32+16hh+[0,16) (high nibbles, sub-block 2c+1) of super-block sb.  A Q8_0 or Q5_1 row is
+// cut into its 32-weight blocks (chunk p = block p).
 
 struct ActChunk {            // one token's activations matching one chunk
-    int4 xa, xb;             // 16 bytes for the low nibbles, 16 for the high (Q8_0: 32 bytes)
-    float dl, dh, sl, sh;    // Q8_1 d and exact d*sum(q) of the two 32-blocks (Q8_0: dl only)
+    int4 xa, xb;             // 16 bytes for the low nibbles, 16 for the high (32-weight blocks:
+                             // the block's 32 bytes)
+    float dl, dh, sl, sh;    // Q8_1 d and exact d*sum(q) of the two 32-blocks (32-weight
+                             // blocks: dl, sl)
 };
 
 __device__ __forceinline__ ActChunk load_act(const int8_t *q, const float *d, const float *s,
-                                             int p, bool q80) {
+                                             int p, bool small) {
     ActChunk a;
-    if (q80) {
+    if (small) {
         a.xa = *reinterpret_cast<const int4 *>(q + 32 * p);
         a.xb = *reinterpret_cast<const int4 *>(q + 32 * p + 16);
         a.dl = d[p];
-        a.dh = a.sl = a.sh = 0.f;
+        a.sl = s[p];
+        a.dh = a.sh = 0.f;
     } else {
         const int sb = p >> 3, j = p & 7, c = j >> 1, hh = j & 1;
         const int kl = sb * 256 + c * 64 + hh * 16;
@@ -191,6 +194,21 @@ __device__ __forceinline__ float q80_chunk_dot(const uint8_t *blk, const ActChun
     return d * (a.dl * (float)acc);
 }
 
+// Q5_1 block (24 bytes, 8-byte aligned): d*xd*sum(q*qx) + m*xs.
+__device__ __forceinline__ float q51_chunk_dot(const uint8_t *blk, const ActChunk &a) {
+    const uint2 *p = reinterpret_cast<const uint2 *>(blk);
+    const Q51Block w = q51_unpack(p[0], p[1], p[2]);
+    int acc = __dp4a((int)w.w[0], a.xa.x, 0);
+    acc = __dp4a((int)w.w[1], a.xa.y, acc);
+    acc = __dp4a((int)w.w[2], a.xa.z, acc);
+    acc = __dp4a((int)w.w[3], a.xa.w, acc);
+    acc = __dp4a((int)w.w[4], a.xb.x, acc);
+    acc = __dp4a((int)w.w[5], a.xb.y, acc);
+    acc = __dp4a((int)w.w[6], a.xb.z, acc);
+    acc = __dp4a((int)w.w[7], a.xb.w, acc);
+    return fmaf(w.d * a.dl, (float)acc, w.m * a.sl);
+}
+
 // Format classes the kernel is specialised for: every expert Q4_K, every expert Q5_K, or any.
 enum { FK_Q4K = 0, FK_Q5K = 1, FK_ANY = 2 };
 
@@ -206,7 +224,8 @@ __device__ __forceinline__ void rows_dot(int fmt_rt, const uint8_t *const (&rows
     const int lane = threadIdx.x & 31;
     const int nchunk = K / 32;
     const int fmt = FK == FK_Q4K ? MOE_FMT_Q4_K : FK == FK_Q5K ? MOE_FMT_Q5_K : fmt_rt;
-    const bool q80 = fmt == MOE_FMT_Q8_0, q5 = fmt == MOE_FMT_Q5_K;
+    const bool q80 = fmt == MOE_FMT_Q8_0, q51 = fmt == MOE_FMT_Q5_1, q5 = fmt == MOE_FMT_Q5_K;
+    const bool small = q80 || q51;
     const int SBB = q5 ? kQ5KBytes : kQ4KBytes;
     for (int p = lane % lpr; p < nchunk; p += lpr) {
         const int sb = p >> 3, j = p & 7;
@@ -215,19 +234,20 @@ __device__ __forceinline__ void rows_dot(int fmt_rt, const uint8_t *const (&rows
         // each token's chunk per row from shared memory (saves registers, costs a few loads)
         ActChunk a0;
         if (NT == 1) a0 = load_act(q + (size_t)act[0] * astride, d + act[0] * (astride / 32),
-                                   s + act[0] * (astride / 32), p, q80);
+                                   s + act[0] * (astride / 32), p, small);
 #pragma unroll
         for (int r = 0; r < R; r++) {
             const uint8_t *row = rows[r];
             if (!row) continue;
-            if (FK == FK_ANY && q80) {
+            if (FK == FK_ANY && small) {
 #pragma unroll
                 for (int t = 0; t < NT; t++) {
                     if (t < n) {
                         const ActChunk a = NT == 1 ? a0
                             : load_act(q + (size_t)act[t] * astride, d + act[t] * (astride / 32),
                                        s + act[t] * (astride / 32), p, true);
-                        acc[r][t] += q80_chunk_dot(row + (size_t)p * kQ80Bytes, a);
+                        acc[r][t] += q80 ? q80_chunk_dot(row + (size_t)p * kQ80Bytes, a)
+                                         : q51_chunk_dot(row + (size_t)p * kQ51Bytes, a);
                     }
                 }
             } else {
@@ -820,7 +840,7 @@ __device__ __forceinline__ void consumer(const DecParams &P, const Ctx &C) {
 #pragma unroll 1
                     for (int jj = m.c; jj < m.c + jl; jj++) joff += (uint32_t)rows * C.s_jobs[jj].stride[2];
                 }
-                const int Kd = (FK == FK_ANY && J.fmt == MOE_FMT_Q8_0) ? ((F + 31) / 32) * 32 : P.hpad;
+                const int Kd = (FK == FK_ANY && small_block(J.fmt)) ? ((F + 31) / 32) * 32 : P.hpad;
                 const uint8_t *const rp[1] = {valid ? stage + joff + (size_t)r * J.stride[2] : nullptr};
                 const int jn = valid ? J.n : 0;
                 int nmax = jn;
@@ -933,7 +953,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_fused(const DecParams P)
     int kmax_down = 0;
 #pragma unroll 1
     for (int u = 0; u < C.U; u++)
-        kmax_down = max(kmax_down, C.s_jobs[u].fmt == MOE_FMT_Q8_0 ? (P.F + 31) / 32 : P.hpad / 32);
+        kmax_down = max(kmax_down, small_block(C.s_jobs[u].fmt) ? (P.F + 31) / 32 : P.hpad / 32);
     C.down_lpr = kmax_down <= 16 ? 16 : 32;
 
     if (warp == kCW) {

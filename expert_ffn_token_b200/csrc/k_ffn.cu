@@ -1,4 +1,5 @@
-// k_ffn.cu -- a4-a7 on CUDA cores: grouped dequant-GEMV over packed Q4_K / Q5_K / Q8_0 rows.
+// k_ffn.cu -- a4-a7 on CUDA cores: grouped dequant-GEMV over packed Q4_K / Q5_K / Q8_0 / Q5_1
+// rows.
 //
 // Decode on the pages streams each selected expert's rows once with register reductions
 // ("decode chain: register reductions, a side stream for the gate projections",
@@ -12,7 +13,8 @@
 //            each product by the routing weight and writes out[t][i] once -- deterministic, no
 //            atomics.  Large batches: one CTA per (job, 32-row tile) with a weighted
 //            scatter-add (or per-slot y plus a gather combine).
-// The dequantized weight is d*sc*q - dmin*m (Q4_K/Q5_K) or d*q (Q8_0): for a sub-block of 32
+// The dequantized weight is d*sc*q - dmin*m (Q4_K/Q5_K), d*q (Q8_0) or d*q + m (Q5_1): for a
+// sub-block of 32
 // the dot with Q8_1 values xd*qx is  d*sc*xd*sum(q*qx) - dmin*m*(xd*sum qx), where the second
 // factor xd*sum(qx) is kept exactly in fp32 per activation block (xsum).
 #include "dot.cuh"
@@ -190,6 +192,23 @@ __global__ void __launch_bounds__(256) k_down_decode(FfnArgs a) {
             }
             continue;
         }
+        if (ex.fmt == MOE_FMT_Q5_1) {
+            for (int b = lane; b < (a.F + 31) / 32; b += 32) {
+                const Q51Block w = q51_load(row, b);
+                for (int s = 0; s < job.n; s++) {
+                    const int slot = job.slot0 + s;
+                    const size_t hbase = (size_t)slot * hb + b;
+                    const float v = q51_dot(w, a.hq + (size_t)slot * a.hpad + 32 * b,
+                                            half_bits_to_float(a.hd[hbase]), a.hsum[hbase]);
+                    const int t = s_tok[slot];
+                    const float wv = s_w[slot] * v;
+#pragma unroll
+                    for (int tt = 0; tt < NT; tt++)
+                        if (tt == t) acc[tt] += wv;
+                }
+            }
+            continue;
+        }
         const bool q5 = ex.fmt == MOE_FMT_Q5_K;
         const int nsb = (a.F + 255) / 256;
         const int j = lane & 7, c = j >> 1, hh = j & 1;
@@ -265,7 +284,7 @@ __global__ void __launch_bounds__(256) k_down_grouped(FfnArgs a, int determinist
     float *s_s = s_d + NT * nb;
     __shared__ int s_tok[NT];
     __shared__ float s_w[NT];
-    const int Kfmt = ex.fmt == MOE_FMT_Q8_0 ? ((a.F + 31) / 32) * 32 : ((a.F + 255) / 256) * 256;
+    const int Kfmt = small_block(ex.fmt) ? ((a.F + 31) / 32) * 32 : ((a.F + 255) / 256) * 256;
     for (int c0 = 0; c0 < job.n; c0 += NT) {
         const int nt = min(NT, job.n - c0);
         if (threadIdx.x < NT) {
@@ -364,7 +383,8 @@ cudaError_t launch_combine(const FfnArgs &a, bool shared, cudaStream_t st) {
 
 // ------------------------------------------------------------------ debug dequant export
 
-// One thread per weight: RN32(RN32(d*sc)*q - RN32(dmin*m)) (K-quants), d*q (Q8_0).
+// One thread per weight: RN32(RN32(d*sc)*q - RN32(dmin*m)) (K-quants), d*q (Q8_0),
+// RN32(d*q + m) (Q5_1; d*q is exact in fp32, so the fused multiply-add rounds once).
 __global__ void k_dequant(const uint8_t *__restrict__ m, int fmt, int rows, int nblocks,
                           int stride, float *out) {
     const int bw = block_weights(fmt), bb = block_bytes(fmt);
@@ -380,6 +400,12 @@ __global__ void k_dequant(const uint8_t *__restrict__ m, int fmt, int rows, int 
         float w;
         if (fmt == MOE_FMT_Q8_0) {
             w = __fmul_rn(half_bits_to_float(d16), (float)(int8_t)p[2 + n]);
+        } else if (fmt == MOE_FMT_Q5_1) {
+            const uint32_t m16 = p[2] | (p[3] << 8);
+            const uint32_t qh = p[4] | (p[5] << 8) | (p[6] << 16) | ((uint32_t)p[7] << 24);
+            int q = n < 16 ? (p[8 + n] & 15) : (p[8 + n - 16] >> 4);
+            q |= (int)((qh >> n) & 1u) << 4;
+            w = __fmaf_rn(half_bits_to_float(d16), (float)q, half_bits_to_float(m16));
         } else {
             const uint32_t m16 = p[2] | (p[3] << 8);
             const int c = n / 64, rr = n % 64;

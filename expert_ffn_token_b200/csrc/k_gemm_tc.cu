@@ -20,6 +20,8 @@
 //   * the min term is a contraction over the sub-blocks, done on the tensor cores in tf32 with
 //     a hi/lo split of both factors (hi*hi + hi*lo + lo*hi): relative error ~2^-22.
 //   * Q8_0 rows (d_j per 32 weights, no min) rescale at every sub-block.
+//   * Q5_1 rows (w = d_j*q + m_j per 32 weights) rescale at every sub-block like Q8_0 and take
+//     the offsets through the min term with wm_j = -m_j (an fp16 value, exact in tf32).
 // Results agree with the exact sums up to fp32 rounding.
 //
 // Roles (576 threads): warp 0 issues TMA loads (packed weights as stored, activations, scales);
@@ -79,9 +81,16 @@ constexpr int kNumBars = 2 * kWSt + 2 * kRawSt + 2 * kMnSt + 2 * kEpSt + 2 * kGr
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kMinCol0 = kGrp * 128;              // 384
 
+// Packed bytes of 256 weights, and how the per-row scale and the min term run for a format:
+// per 32-weight block (Q8_0, Q5_1) or per super-block (K-quants); with a min/offset term
+// (everything but Q8_0).
 __host__ __device__ inline uint32_t sb_bytes(int fmt) {
-    return fmt == MOE_FMT_Q4_K ? 144u : fmt == MOE_FMT_Q5_K ? 176u : 272u;
+    return fmt == MOE_FMT_Q4_K ? 144u : fmt == MOE_FMT_Q5_K ? 176u : fmt == MOE_FMT_Q8_0 ? 272u : 192u;
 }
+__host__ __device__ inline bool per_block_scale(int fmt) {
+    return fmt == MOE_FMT_Q8_0 || fmt == MOE_FMT_Q5_1;
+}
+__host__ __device__ inline bool has_min(int fmt) { return fmt != MOE_FMT_Q8_0; }
 
 struct GemmArgs {
     const CUtensorMap *wmaps;     // [n_experts (+ shared)][3] packed gate, up, down
@@ -255,7 +264,7 @@ __device__ void role_producer(const GemmArgs &a, const Smem &S, int nj, const CU
     for (int i = blockIdx.x;; i += gridDim.x) {
         Tile t;
         if (!tile_at(a, nj, cur, i, t)) break;
-        const bool kq = t.fmt != MOE_FMT_Q8_0;
+        const bool mnt = has_min(t.fmt);
         const uint32_t sbb = sb_bytes(t.fmt);
         const CUtensorMap *ma, *mb;
         int ya, yb;
@@ -272,14 +281,15 @@ __device__ void role_producer(const GemmArgs &a, const Smem &S, int nj, const CU
             if (!wait_fast(S.raw_empty + rr.s, rr.ph ^ 1u, S.abort, a.status)) return;
             uint8_t *rs = S.raw + rr.s * a.raw_stage;
             mbar_arrive_expect_tx(S.raw_full + rr.s, 128u * sbb + (uint32_t)t.nbox * 1024u);
-            const int x = kq ? sb * (int)sbb : sb * 136;
+            // Q8_0 maps count 16-bit elements (34-byte blocks), the others bytes
+            const int x = t.fmt == MOE_FMT_Q8_0 ? sb * 136 : sb * (int)sbb;
             tma_load_2d(rs, ma, x, ya, S.raw_full + rr.s);
             tma_load_2d(rs + 64 * sbb, mb, x, yb, S.raw_full + rr.s);
             for (int b = 0; b < t.nbox; b++)
                 tma_load_2d(rs + a.raw_xd_off + b * 1024, md, sb * 8, t.slot_base + 32 * b,
                             S.raw_full + rr.s);
             rr.adv(kRawSt);
-            if (kq) {
+            if (mnt) {
                 if (!wait_fast(S.mn_empty + rm.s, rm.ph ^ 1u, S.abort, a.status)) return;
                 uint8_t *ms = S.mn + rm.s * kMnStage;
                 mbar_arrive_expect_tx(S.mn_full + rm.s, (uint32_t)t.nbox * 2048u);
@@ -342,7 +352,7 @@ __device__ __forceinline__ void scale_pair(int s, uint32_t &s2, uint32_t &nb2) {
 }
 
 // Row r's 32 weights of sub-block j = 2 st + hsel as fp16 integers sc_j * q (K-quants) or q
-// (Q8_0), written into their half of the 128-byte-swizzled K-major operand row.
+// (Q8_0, Q5_1), written into their half of the 128-byte-swizzled K-major operand row.
 template <int FMT>
 __device__ __forceinline__ void unpack_half(const uint8_t *rowp, int st, int hsel, int scale,
                                             bool zero, uint8_t *a16, int r) {
@@ -363,6 +373,23 @@ __device__ __forceinline__ void unpack_half(const uint8_t *rowp, int st, int hse
             const uint32_t b = hsub2_u(prmt(x, 0x64646464u, 0x4341u), k1152);
             v[2 * wi] = z ? 0u : a;
             v[2 * wi + 1] = z ? 0u : b;
+        }
+    } else if (FMT == MOE_FMT_Q5_1) {
+        // element n < 16: low nibble of qs[n], n >= 16: high nibble of qs[n - 16]; bit n of qh
+        // is its fifth bit.  Word wi of the operand covers elements 4 wi .. 4 wi + 3.
+        const uint2 *bp = reinterpret_cast<const uint2 *>(rowp + 24 * (2 * st + hsel));
+        const uint2 h = bp[0], qa = bp[1], qb = bp[2];
+        const bool z = zero || (h.x & 0x7FFFu) == 0;
+        const uint32_t qw[4] = {qa.x, qa.y, qb.x, qb.y};
+#pragma unroll
+        for (int wi = 0; wi < 8; wi++) {
+            const uint32_t x = wi < 4 ? qw[wi] : qw[wi - 4] >> 4;
+            const uint32_t t = h.y >> (4 * wi);
+            // bits 0, 2 of t -> bits 4, 20 (elements k, k+2); bits 1, 3 -> (k+1, k+3)
+            const uint32_t a = lop3_and_or(x, kM, kE) | (((t & 5u) * 0x40010u) & 0x00100010u);
+            const uint32_t b = lop3_and_or(x >> 8, kM, kE) | (((t & 10u) * 0x20008u) & 0x00100010u);
+            v[2 * wi] = z ? 0u : hsub2_u(a, kE);
+            v[2 * wi + 1] = z ? 0u : hsub2_u(b, kE);
         }
     } else {
         const int qs_off = FMT == MOE_FMT_Q5_K ? 48 : 16;
@@ -411,13 +438,14 @@ __device__ __forceinline__ bool unpack_superblock(const GemmArgs &a, const Smem 
     const uint8_t *rowp = rs + (size_t)r * sbb;
     int sc[8], mn[8];
     float d = 0.f, dmin = 0.f;
+    float off[8];                              // Q5_1: the blocks' offsets m_j
     // ---- epilogue scales: unit ratios, unit, transposed xd
     if (!wait_bar_warp(S.ep_empty + re.s, re.ph ^ 1u, S.abort, a.status)) return false;
     uint8_t *es = S.ep + re.s * kEpStage;
     float *xdT = reinterpret_cast<float *>(es);
     float *ratio = reinterpret_cast<float *>(es + kEpXdT);
     float *unit = reinterpret_cast<float *>(es + kEpXdT + kEpRatio);
-    if (FMT != MOE_FMT_Q8_0) {
+    if (!per_block_scale(FMT)) {
         d = ld_half(rowp);
         dmin = ld_half(rowp + 2);
         const uint32_t s0 = *reinterpret_cast<const uint32_t *>(rowp + 4);
@@ -432,11 +460,13 @@ __device__ __forceinline__ bool unpack_superblock(const GemmArgs &a, const Smem 
         }
         if (hsel == 0) ratio[r] = rt;
     } else {
+        constexpr int kBB = FMT == MOE_FMT_Q8_0 ? 34 : 24;
 #pragma unroll
         for (int j = 0; j < 8; j++) {
             sc[j] = 1;
             mn[j] = 0;
-            const float dj = ld_half(rowp + 34 * j);
+            off[j] = FMT == MOE_FMT_Q5_1 ? ld_half(rowp + kBB * j + 2) : 0.0f;
+            const float dj = ld_half(rowp + kBB * j);
             float rt = 1.0f;
             if (dj != 0.0f) {
                 rt = __fdiv_rn(U, dj);
@@ -461,14 +491,15 @@ __device__ __forceinline__ bool unpack_superblock(const GemmArgs &a, const Smem 
     __syncwarp();
     if (lane == 0) mbar_arrive(S.ep_full + re.s);
     re.adv(kEpSt);
-    // ---- min-term operand rows (K-quants): RN32(dmin * m_j) split into tf32 hi + lo
-    if (FMT != MOE_FMT_Q8_0) {
+    // ---- min-term operand rows: RN32(dmin * m_j) (K-quants) or -m_j (Q5_1), split into
+    // tf32 hi + lo (for Q5_1 lo is 0: an fp16 value is exact in tf32)
+    if (has_min(FMT)) {
         if (!wait_bar_warp(S.mn_empty + rm.s, rm.ph ^ 1u, S.abort, a.status)) return false;
         uint8_t *ms = S.mn + rm.s * kMnStage;
         float wh[8], wl[8];
 #pragma unroll
         for (int j = 0; j < 8; j++) {
-            const float wm = __fmul_rn(dmin, (float)mn[j]);
+            const float wm = FMT == MOE_FMT_Q5_1 ? -off[j] : __fmul_rn(dmin, (float)mn[j]);
             wh[j] = tf32_round(wm);
             wl[j] = wm - wh[j];
         }
@@ -488,7 +519,7 @@ __device__ __forceinline__ bool unpack_superblock(const GemmArgs &a, const Smem 
         rm.adv(kMnSt);
     }
     // ---- the two 128-wide operand stages (two swizzle atoms, four sub-blocks each)
-    const bool zero = FMT != MOE_FMT_Q8_0 && d == 0.0f;
+    const bool zero = !per_block_scale(FMT) && d == 0.0f;
     for (int st = 0; st < 2; st++) {
         if (!wait_bar_warp(S.w_empty + rw.s, rw.ph ^ 1u, S.abort, a.status)) return false;
         uint8_t *a16 = S.w + rw.s * kWStage;
@@ -521,8 +552,10 @@ __device__ void role_unpack(const GemmArgs &a, const Smem &S, int nj) {
                 ok = unpack_superblock<MOE_FMT_Q4_K>(a, S, rw, rm, re, rs, U, u);
             else if (t.fmt == MOE_FMT_Q5_K)
                 ok = unpack_superblock<MOE_FMT_Q5_K>(a, S, rw, rm, re, rs, U, u);
-            else
+            else if (t.fmt == MOE_FMT_Q8_0)
                 ok = unpack_superblock<MOE_FMT_Q8_0>(a, S, rw, rm, re, rs, U, u);
+            else
+                ok = unpack_superblock<MOE_FMT_Q5_1>(a, S, rw, rm, re, rs, U, u);
             if (!ok) return;
             __syncwarp();
             if (lane == 0) mbar_arrive(S.raw_empty + rr.s);
@@ -546,7 +579,7 @@ __device__ void role_mma(const GemmArgs &a, const Smem &S, int nj, uint32_t tbas
     for (int i = blockIdx.x;; i += gridDim.x) {
         Tile t;
         if (!tile_at(a, nj, cur, i, t)) break;
-        const bool kq = t.fmt != MOE_FMT_Q8_0;
+        const bool mnt = has_min(t.fmt);
         const uint32_t idf = instr_desc(0, kTM, t.n_mma);
         const uint32_t idt = instr_desc(2, kTM, t.n_mma);
         for (int sb = 0; sb < nsb; sb++) {
@@ -571,7 +604,7 @@ __device__ void role_mma(const GemmArgs &a, const Smem &S, int nj, uint32_t tbas
                 umma_commit(S.w_empty + rw.s);
                 rw.adv(kWSt);
             }
-            if (kq) {
+            if (mnt) {
                 if (!wait_fast(S.mn_full + rm.s, rm.ph, S.abort, a.status)) return;
                 if (sb == 0 && !wait_fast(S.min_empty + rmin.s, rmin.ph ^ 1u, S.abort, a.status))
                     return;
@@ -587,7 +620,7 @@ __device__ void role_mma(const GemmArgs &a, const Smem &S, int nj, uint32_t tbas
                 rm.adv(kMnSt);
             }
         }
-        if (kq) {
+        if (mnt) {
             umma_commit(S.min_full + rmin.s);
             rmin.adv(kMinBuf);
         }
@@ -676,7 +709,7 @@ __device__ void role_epilogue(const GemmArgs &a, const Smem &S, int nj, uint32_t
     for (int i = blockIdx.x;; i += gridDim.x) {
         Tile t;
         if (!tile_at(a, nj, cur, i, t)) break;
-        const bool kq = t.fmt != MOE_FMT_Q8_0;
+        const bool pbs = per_block_scale(t.fmt), mnt = has_min(t.fmt);
         const int ncol = min(32, t.n_valid - 32 * hcol);
         const bool active = ncol > 0;
         float acc[32];
@@ -694,7 +727,7 @@ __device__ void role_epilogue(const GemmArgs &a, const Smem &S, int nj, uint32_t
                 xdT = reinterpret_cast<const float *>(es);
                 ratio = reinterpret_cast<const float *>(es + kEpXdT);
                 unit = reinterpret_cast<const float *>(es + kEpXdT + kEpRatio);
-                if (kq && active) {
+                if (!pbs && active) {
                     const float rt = ratio[r];
 #pragma unroll
                     for (int c = 0; c < 32; c++) acc[c] *= rt;
@@ -707,7 +740,7 @@ __device__ void role_epilogue(const GemmArgs &a, const Smem &S, int nj, uint32_t
 #pragma unroll 1
                 for (int h2 = 0; h2 < 2; h2++) {
                     const int jj = 2 * st + h2;
-                    if (!kq) {
+                    if (pbs) {
                         const float rt = ratio[jj * kTM + r];
 #pragma unroll
                         for (int c = 0; c < 32; c++) acc[c] *= rt;
@@ -744,7 +777,7 @@ __device__ void role_epilogue(const GemmArgs &a, const Smem &S, int nj, uint32_t
         // min term, then the row scale: y = acc * U - min
 #pragma unroll
         for (int c = 0; c < 32; c++) acc[c] *= U;
-        if (kq) {
+        if (mnt) {
             if (!wait_bar_warp(S.min_full + rmin.s, rmin.ph, S.abort, a.status)) return;
             tc_fence_after();
             if (active) {
@@ -1031,6 +1064,10 @@ bool tc_build_weight_maps(const uint8_t *d_base, const moe_expert_desc *descs, i
                 const uint64_t nb = (uint64_t)((width + 31) / 32);
                 ok = encode_2d(&maps[e * 3 + t], CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, base, nb * 17,
                                (uint64_t)rows, d.stride[t], 136, 64, CU_TENSOR_MAP_SWIZZLE_NONE);
+            } else if (d.fmt == MOE_FMT_Q5_1) {
+                const uint64_t nb = (uint64_t)((width + 31) / 32);
+                ok = encode_2d(&maps[e * 3 + t], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, base, nb * 24,
+                               (uint64_t)rows, d.stride[t], 192, 64, CU_TENSOR_MAP_SWIZZLE_NONE);
             } else {
                 const uint32_t sbb = sb_bytes(d.fmt);
                 const uint64_t nsb = (uint64_t)((width + 255) / 256);
@@ -1064,7 +1101,7 @@ cudaError_t launch_gemm_tc(const TcPhaseArgs &p, cudaStream_t st) {
     a.K = p.phase == 0 ? f.H : f.hpad;
     a.mt_count = p.phase == 0 ? (f.F + 63) / 64 : (f.H + kTM - 1) / kTM;
     uint32_t sbb_max = 0;
-    for (int fm = 0; fm < 3; fm++)
+    for (int fm = 0; fm <= MOE_FMT_Q5_1; fm++)
         if (f.fmt_mask & (1 << fm)) sbb_max = sbb_max > sb_bytes(fm) ? sbb_max : sb_bytes(fm);
     a.raw_xd_off = 128u * sbb_max;
     a.raw_stage = ((a.raw_xd_off + kRawXd) + 1023u) & ~1023u;
@@ -1145,7 +1182,7 @@ cudaError_t launch_hg_tail_zero(__half *hg, float *hgd, float *hgsh, float *hgsl
 
 size_t tc_smem_bytes(int fmt_mask) {
     uint32_t sbb_max = 0;
-    for (int fm = 0; fm < 3; fm++)
+    for (int fm = 0; fm <= MOE_FMT_Q5_1; fm++)
         if (fmt_mask & (1 << fm)) sbb_max = sbb_max > sb_bytes(fm) ? sbb_max : sb_bytes(fm);
     const uint32_t raw_stage = ((128u * sbb_max + kRawXd) + 1023u) & ~1023u;
     return smem_bytes(raw_stage);

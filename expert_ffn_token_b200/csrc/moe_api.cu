@@ -147,7 +147,7 @@ moe_status moe_arena_create(const void *d_arena, size_t arena_bytes, int hidden,
     uint64_t ms01 = 0, ms2 = 0;
     for (int e = 0; e < n; e++) {
         const moe_expert_desc &d = host_descs[e];
-        if (d.fmt < 0 || d.fmt > 2 || d.reserved != 0) return MOE_ERR_INVALID_ARG;
+        if (d.fmt < 0 || d.fmt > MOE_FMT_Q5_1 || d.reserved != 0) return MOE_ERR_INVALID_ARG;
         const int bw = block_weights(d.fmt), bb = block_bytes(d.fmt);
         if (hidden % bw) return MOE_ERR_UNSUPPORTED;
         const int rows[3] = {ffn, ffn, hidden};

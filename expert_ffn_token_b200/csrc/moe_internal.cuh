@@ -7,6 +7,8 @@
 //   Q5_K 176 B: as Q4_K with qh[32] at [16,48) and qs at [48,176); bit 2c of qh[r] is the fifth
 //        bit of element 64c+r, bit 2c+1 that of element 64c+32+r.
 //   Q8_0 34 B / 32 weights: fp16 d, int8 q[32].
+//   Q5_1 24 B / 32 weights: fp16 d, fp16 m, uint32 qh (bit n: fifth bit of element n),
+//        qs[16]: byte i holds element i (low nibble) and element 16+i (high nibble); w = d*q + m.
 //   Q8_1 (activations, stored SoA): per 32 values int8 q[32], fp16 d, fp16 s = d * sum(q).
 #pragma once
 
@@ -29,14 +31,22 @@ constexpr int kSB = 256;          // K-quant super-block length
 constexpr int kQ4KBytes = 144;
 constexpr int kQ5KBytes = 176;
 constexpr int kQ80Bytes = 34;
+constexpr int kQ51Bytes = 24;
 constexpr int kMaxK = 32;         // routed experts per token
 constexpr int kMaxE = 4096;       // experts per layer
 constexpr int kDecodeMaxT = 16;   // largest batch the dequant-GEMV path takes by default
 constexpr int kChunk = 64;        // tokens per histogram chunk in the grouping kernels
 
-__host__ __device__ inline int block_weights(int fmt) { return fmt == MOE_FMT_Q8_0 ? 32 : 256; }
+// Q8_0 and Q5_1 carry their scale per 32 weights; the K-quants per 256-weight super-block.
+__host__ __device__ inline bool small_block(int fmt) {
+    return fmt == MOE_FMT_Q8_0 || fmt == MOE_FMT_Q5_1;
+}
+__host__ __device__ inline int block_weights(int fmt) { return small_block(fmt) ? 32 : 256; }
 __host__ __device__ inline int block_bytes(int fmt) {
-    return fmt == MOE_FMT_Q4_K ? kQ4KBytes : fmt == MOE_FMT_Q5_K ? kQ5KBytes : kQ80Bytes;
+    return fmt == MOE_FMT_Q4_K   ? kQ4KBytes
+           : fmt == MOE_FMT_Q5_K ? kQ5KBytes
+           : fmt == MOE_FMT_Q8_0 ? kQ80Bytes
+                                 : kQ51Bytes;
 }
 
 // Device copy of one expert (the descriptor with the arena base folded in).

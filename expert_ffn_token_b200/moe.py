@@ -23,7 +23,7 @@ OK = 0
 ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_ALIGNMENT, ERR_CUDA = 1, 2, 3, 4
 ERR_NONFINITE, ERR_BOUNDS, ERR_TIMEOUT, ERR_WORKSPACE = 5, 6, 7, 8
 
-FMT_Q4_K, FMT_Q5_K, FMT_Q8_0 = 0, 1, 2
+FMT_Q4_K, FMT_Q5_K, FMT_Q8_0, FMT_Q5_1 = 0, 1, 2, 3
 
 F_DETERMINISTIC = 1
 F_FORCE_DECODE = 2

@@ -6,7 +6,7 @@
  *     512 experts per layer, 10 routed + 1 always-on shared expert, hidden size 2,560;
  *     "Strata-Sage-A1.5-GGUF": 256 experts, top-8.
  *   - "Strata v0.1.31" release notes, section "Experimental: Unsloth UD-Q4_K_XL on a normal
- *     PC": experts stored as Q4_K, Q5_K and Q8_0 blocks (GGUF), decoded bit for bit as
+ *     PC": experts stored as Q4_K, Q5_K, Q5_1 and Q8_0 blocks (GGUF), decoded bit for bit as
  *     llama.cpp decodes them, dot products equal to ggml's within float rounding.
  *   - "Strata v0.1.39" release notes, fixes list, #606: q8_1 activations;
  *     "Strata-Sage-A1.5-GGUF", round-2 table: one activation quantization per token.
@@ -60,8 +60,11 @@ typedef enum {
  *   Q4_K  256 weights in 144 B: fp16 d, fp16 dmin, 12 B of packed 6-bit sub-block scales and
  *         mins (8 sub-blocks of 32), 128 B of 4-bit quants; w = d*sc*q - dmin*m
  *   Q5_K  256 weights in 176 B: as Q4_K plus a 32 B plane of fifth bits before the quants
- *   Q8_0  32 weights in 34 B: fp16 d, 32 int8 q; w = d*q                                      */
-typedef enum { MOE_FMT_Q4_K = 0, MOE_FMT_Q5_K = 1, MOE_FMT_Q8_0 = 2 } moe_fmt;
+ *   Q8_0  32 weights in 34 B: fp16 d, 32 int8 q; w = d*q
+ *   Q5_1  32 weights in 24 B: fp16 d, fp16 m, 32 fifth bits (uint32), 16 B of 4-bit quants
+ *         (element n < 16: low nibble of byte n, n >= 16: high nibble of byte n-16);
+ *         w = d*q + m                                                                        */
+typedef enum { MOE_FMT_Q4_K = 0, MOE_FMT_Q5_K = 1, MOE_FMT_Q8_0 = 2, MOE_FMT_Q5_1 = 3 } moe_fmt;
 
 /* One expert inside the arena.  Matrices follow the GGUF convention: a row is one output
  * neuron, blocks run along the input dimension.  gate and up: ffn rows of `hidden` weights;
@@ -80,7 +83,7 @@ typedef struct moe_arena moe_arena;
 /* Register a device-resident expert arena: `n_experts` routed experts plus, when
  * shared_expert >= 0, one more descriptor at index n_experts for the always-on shared expert
  * (shared_expert must then equal n_experts).  host_descs has n_experts (+1) entries.
- * hidden: multiple of 256 (K-quants) or 32 (Q8_0 only); ffn: multiple of 32.
+ * hidden: multiple of 256 (K-quants) or 32 (Q8_0 and Q5_1 only); ffn: multiple of 32.
  * Checks every descriptor against arena_bytes (MOE_ERR_BOUNDS) and alignment; copies the table
  * to the device (the one allocation the library makes, freed by moe_arena_destroy).  d_arena
  * (256-byte aligned) must stay valid until moe_arena_destroy.                                */
@@ -160,7 +163,8 @@ moe_status moe_read_status(uint32_t *d_status_word, void *stream, int clear,
 
 /* Debug export of one matrix (which: 0 gate, 1 up, 2 down; expert n_experts = shared) as
  * fp32 [rows][row weights] where row weights = whole blocks.  Each value is
- * RN32(RN32(d*sc)*q - RN32(dmin*m)) (K-quants) or d*q (Q8_0), bit for bit.               */
+ * RN32(RN32(d*sc)*q - RN32(dmin*m)) (K-quants), d*q (Q8_0) or RN32(d*q + m) (Q5_1), bit
+ * for bit.                                                                                 */
 moe_status moe_debug_dequant(const moe_arena *arena, int expert, int which, float *d_out,
                              void *stream);
 

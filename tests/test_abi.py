@@ -65,6 +65,8 @@ def test_arena_create_rejects_bad_arguments(moe):
     assert create(shared=3) == moe.ERR_INVALID_ARG                # shared must be E
     assert create(H=8192) == moe.ERR_UNSUPPORTED
     assert create(descs=_desc(fmt=7)) == moe.ERR_INVALID_ARG
+    assert create(descs=_desc(fmt=4)) == moe.ERR_INVALID_ARG       # formats are 0..3
+    assert create(descs=_desc(fmt=3, stride=(176, 176, 176))) == moe.ERR_INVALID_ARG  # Q5_1 row: 192 B
     assert create(descs=_desc(off=(8, 36864, 73728))) == moe.ERR_ALIGNMENT
     assert create(descs=_desc(stride=(128, 144, 144))) == moe.ERR_INVALID_ARG  # < packed row
     assert create(nbytes=100000) == moe.ERR_BOUNDS                # down matrix ends past it

@@ -307,3 +307,61 @@ def test_decode_large_expert_count_uses_grouped_kernels(torch):
     w = synth.Workload("wideE", 70, 256, 256, 2048, 4, 3, True, 1, "normal", sigma=2.0)
     x, logits = inputs(w, 0)
     _check_layer(torch, w, 0, x, logits, keep_h=True)
+
+
+# ------------------------------------------------------------------ Q5_1 experts
+
+# hidden 512, width 320 (down rows padded to 512 on the tensor-core path), 32 experts, top-4
+# + shared: every expert Q5_1, or the four formats mixed a quarter each
+Q51 = synth.Workload("q5_1_layer", 23, 512, 320, 32, 4, 40, True, 1, "normal", sigma=1.5,
+                     mix=((synth.Q5_1, 1.0),), note="Q5_1 experts")
+FOUR = synth.Workload("four_formats", 24, 512, 320, 32, 4, 150, True, 1, "normal", sigma=1.5,
+                      mix=((synth.Q4_K, 0.25), (synth.Q5_K, 0.5), (synth.Q8_0, 0.75),
+                           (synth.Q5_1, 1.0)),
+                      note="Q4_K, Q5_K, Q8_0 and Q5_1 experts in one layer")
+
+
+def test_q5_1_device_fill_and_dequant_bit_exact(torch):
+    from expert_ffn_token_b200 import moe
+    w = FOUR
+    fmts = synth.layer_formats(w, 0)
+    assert set(int(f) for f in fmts) == {0, 1, 2, 3}
+    L, arena, lay = device_layer(w, 0, max_tokens=1)
+    host = arena.cpu().numpy()
+    for e in range(lay.n):
+        for t in range(3):
+            ref = synth.tensor_bytes(w, 0, e, t, int(fmts[e]))
+            assert np.array_equal(host[lay.offs[e, t]:lay.offs[e, t] + ref.size], ref), (e, t)
+    for e in [int(np.nonzero(fmts == 3)[0][i]) for i in (0, 1)]:
+        for t in range(3):
+            rows, width = synth.tensor_shape(w, t)
+            nb = -(-width // 32)
+            out = torch.empty((rows, nb * 32), dtype=torch.float32, device="cuda")
+            moe.debug_dequant(L.handle, e, t, out.data_ptr(), _stream(torch))
+            _, ref32 = oracle.dequant_matrix(3, host[lay.offs[e, t]:], rows,
+                                             int(lay.strides[e, t]), nb)
+            assert np.array_equal(out.cpu().numpy().view(np.uint32), ref32.view(np.uint32)), (e, t)
+    L.close()
+
+
+@pytest.mark.parametrize("T,flags", [(1, 0), (3, 0), (16, 0), (40, 2), (40, 4), (40, 5)])
+def test_q5_1_layer_every_path(torch, T, flags):
+    # T <= 16: the fused decode kernel; 40 tokens forced to the CUDA-core grouped kernels (2),
+    # or to the tensor cores (4), deterministic (5)
+    w = synth.with_tokens(Q51, T)
+    x, logits = inputs(w, 0)
+    _check_layer(torch, w, 0, x, logits, flags=flags, keep_h=True)
+
+
+@pytest.mark.parametrize("T,flags", [(2, 0), (12, 0), (150, 2), (150, 4), (150, 5)])
+def test_four_formats_layer_every_path(torch, T, flags):
+    w = synth.with_tokens(FOUR, T)
+    x, logits = inputs(w, 0)
+    _check_layer(torch, w, 0, x, logits, flags=flags, keep_h=T <= 12)
+
+
+def test_q5_1_large_expert_count_grouped_decode(torch):
+    w = synth.Workload("wideE_q51", 71, 256, 256, 2048, 4, 3, True, 1, "normal", sigma=2.0,
+                       mix=((synth.Q5_1, 1.0),))
+    x, logits = inputs(w, 0)
+    _check_layer(torch, w, 0, x, logits, keep_h=True)
