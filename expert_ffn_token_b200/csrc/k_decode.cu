@@ -21,9 +21,10 @@
 //     set of 16-byte quant chunks (activations loaded once per chunk, reused over the rows);
 //     h = silu(g) * u goes to shared memory and, once the 32-row block is complete, to Q8_1.
 //   down: after every CTA has published its blocks (bounded wait on one counter), all Q8_1(h)
-//     rows are staged in shared memory; each warp keeps one or two output rows (16 lanes per
-//     row when a row has <= 16 chunks), runs over every job, weights each slot's product in the
-//     lanes and reduces once per row -- deterministic, each output element written once.
+//     rows are staged in shared memory; each warp owns one or two output rows of its CTA's
+//     range, its lanes split the (expert, chunk) pairs of those rows, weight each slot's
+//     product and keep per-token sums, reduced across the lanes once per row --
+//     deterministic, each output element written once.
 // Every wait is bounded by %globaltimer and reports MOE_ERR_TIMEOUT instead of hanging.  The
 // down phase waits on the gate/up work of every CTA: the grid is one CTA per SM (all resident
 // together; a programmatically launched successor starts only once every CTA here has
@@ -65,6 +66,7 @@ struct DecParams {
     WsLayout L;
     int T, H, F, E, k, shared, hpad;
     int stage_bytes, nstages, max_jobs, slots;
+    int keep_h;            // also store fp32 h
     int o_bar, o_meta, o_xq, o_xd, o_xs, o_jobs, o_stok, o_sw, o_hq, o_hd, o_hs, o_gu, o_h,
         o_acc, o_misc;
     int smem_bytes;
@@ -227,6 +229,7 @@ __device__ __forceinline__ void rows_dot(int fmt_rt, const uint8_t *const (&rows
     const bool q80 = fmt == MOE_FMT_Q8_0, q51 = fmt == MOE_FMT_Q5_1, q5 = fmt == MOE_FMT_Q5_K;
     const bool small = q80 || q51;
     const int SBB = q5 ? kQ5KBytes : kQ4KBytes;
+#pragma unroll 2
     for (int p = lane % lpr; p < nchunk; p += lpr) {
         const int sb = p >> 3, j = p & 7;
         const float mf = (j & 1) ? 0.f : 1.f;
@@ -387,16 +390,22 @@ struct Ctx {
     int *s_stok;
     float *s_sw;
     int8_t *s_hq;
-    float *s_hd, *s_hs, *s_part, *s_h;
+    float *s_hd, *s_hs, *s_h;
     int *s_misc;             // [0] jobs [2] timeout
-    uint64_t *full, *empty;
+    uint64_t *full, *empty, *desc_bar;
     StageMeta *meta;
     uint8_t *ring;
     uint8_t *ws;
     uint32_t *status, *ctr;  // ctr: [1] blocks published [2] CTAs finished
-    int T, H, F, E, k, U, nb32, n_blk, my_blocks, i_lo, i_hi, hb, down_lpr;
+    int T, H, F, E, k, U, nb32, n_blk, my_blocks, i_lo, i_hi, hb;
     bool cta0;
 };
+
+// Where the prologue keeps the expert descriptor table: in the stage ring, after the routing
+// scratch (counts, offsets, bitmap, ids, weights), 16-byte aligned.
+__device__ __forceinline__ ExpertDev *desc_table(uint8_t *sm, int E, int T, int k) {
+    return reinterpret_cast<ExpertDev *>(sm + (((2 * E + 64 + 2 * T * k) * 4 + 15) / 16) * 16);
+}
 
 // a1-a3 for the whole batch (every CTA; CTA 0 also stores the intermediates).
 template <int VPL>
@@ -414,18 +423,10 @@ __device__ __forceinline__ void prologue(const DecParams &P, Ctx &C, uint8_t *sm
     int *s_wbase = reinterpret_cast<int *>(s_bits + 32);     // [32]
     int *s_ids = s_wbase + 32;                               // [T*k]
     float *s_wt = reinterpret_cast<float *>(s_ids + T * k);  // [T*k]
-    ExpertDev *s_ex = reinterpret_cast<ExpertDev *>(
-        sm + (((2 * E + 64 + 2 * T * k) * 4 + 15) / 16) * 16);   // [E + shared] descriptors
+    const ExpertDev *s_ex = desc_table(sm, E, T, k);   // filled by the entry's bulk copy
 #pragma unroll 1
     for (int e = tid; e < E; e += kThreads) s_cnt[e] = 0;
     if (tid < 32) s_bits[tid] = 0;
-    {   // the descriptor table, fetched while the experts are being chosen
-        const int nd = (E + P.shared) * (int)(sizeof(ExpertDev) / 8);
-        const unsigned long long *src = reinterpret_cast<const unsigned long long *>(P.experts);
-        unsigned long long *dst = reinterpret_cast<unsigned long long *>(s_ex);
-#pragma unroll 1
-        for (int i = tid; i < nd; i += kThreads) dst[i] = __ldg(src + i);
-    }
     // ---- a2 on warps 0..T-1 (T <= 4), a1 on the rest, at the same time
     const int topk_warps = T <= 4 ? T : 0;
     uint16_t *g_xd = cta0 ? reinterpret_cast<uint16_t *>(ws + L.xd) : nullptr;
@@ -451,6 +452,7 @@ __device__ __forceinline__ void prologue(const DecParams &P, Ctx &C, uint8_t *sm
             for (int u = 0; u < 4; u++) {
                 const int blk = b0 + g0 + u * groups;
                 const bool act = blk < nxb;
+                if (!__any_sync(kFullMask, act)) break;   // blocks ascend with u: none left
                 quant_x_block(v[u], act, sub, act ? blk : 0, C.s_xq, C.s_xd, C.s_xs, g_xd, g_xs,
                               g_xsum, st);
             }
@@ -545,6 +547,7 @@ __device__ __forceinline__ void prologue(const DecParams &P, Ctx &C, uint8_t *sm
         C.s_stok[A + t] = t;
         C.s_sw[A + t] = 1.0f;
     }
+    if (tid < U && !ptx::mbar_wait_bounded(C.desc_bar, 0, kWaitNs)) set_status(status, MOE_ERR_TIMEOUT);
 #pragma unroll 1
     for (int u = tid; u < U; u += kThreads) {
         JobX &J = s_jobs[u];
@@ -676,7 +679,7 @@ __device__ __forceinline__ void quantize_h_block(const DecParams &P, const Ctx &
     for (int t = warp; t < J.n; t += kCW) {
         const int slot = J.slot0 + t;
         const float v = C.s_h[lane * 16 + t];
-        g_h[(size_t)slot * F + 32 * b + lane] = v;
+        if (P.keep_h) g_h[(size_t)slot * F + 32 * b + lane] = v;
         bool fin;
         uint16_t d16, s16;
         float dsum;
@@ -736,19 +739,103 @@ __device__ __forceinline__ bool wait_and_stage_h(const DecParams &P, const Ctx &
     return C.s_misc[2] == 0;
 }
 
-// Sum a down unit's per-warp partials in a fixed order and write the outputs.
-template <int TT>
-__device__ __forceinline__ void finish_down_unit(const DecParams &P, const Ctx &C, int i0, int rows) {
-    const int ctid = threadIdx.x;
+// One down stage: rows [0, rows) of the unit (warp w owns rows w and w + 16) times the jobs
+// [j0, j1) staged here, job after job, each `rows` rows of its down matrix.  The lanes of a warp
+// split the (job, chunk) pairs of a row; each pair is dotted with Q8_1(h) of every slot of its
+// job and added, weighted, into the lane's per-token sums.  The order of the sums is fixed, so
+// the result is deterministic; the lanes are reduced once, at the end of the unit.
+template <int TT, int FK>
+__device__ __forceinline__ void down_stage(const DecParams &P, const Ctx &C, const uint8_t *stage,
+                                           int rows, int j0, int j1, float (&dacc)[2][TT]) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int kq_chunks = P.hpad / 32;          // K-quant rows: 16-byte chunks of 32 weights
+    const int sm_chunks = (C.F + 31) / 32;      // Q8_0 / Q5_1 rows: one chunk per block
+    const int hb = C.hb;
+    uint32_t base = 0;                          // offset of job g0 inside the stage
 #pragma unroll 1
-    for (int i = ctid; i < rows * C.T; i += kCW * 32) {
-        const int r = i / C.T, t = i % C.T;
-        float v = 0.f;
+    for (int g0 = j0; g0 < j1; g0 += 32) {
+        const int ng = min(32, j1 - g0);
+        // lane l < ng: job g0 + l -- its bytes in the stage and its chunk count, scanned
+        uint32_t sz = 0;
+        int nch = 0;
+        if (lane < ng) {
+            const JobX &J = C.s_jobs[g0 + lane];
+            sz = (uint32_t)rows * J.stride[2];
+            nch = (FK == FK_ANY && small_block(J.fmt)) ? sm_chunks : kq_chunks;
+        }
+        uint32_t off = sz;
+        int cend = nch;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t a = __shfl_up_sync(kFullMask, off, o);
+            const int b = __shfl_up_sync(kFullMask, cend, o);
+            if (lane >= o) {
+                off += a;
+                cend += b;
+            }
+        }
+        off = base + off - sz;                   // exclusive: this lane's job offset
+        const int total = __shfl_sync(kFullMask, cend, 31);
+#pragma unroll 2
+        for (int f0 = 0; f0 < total; f0 += 32) {
+            const int f = f0 + lane;
+            // the pair (jl, p) of item f
+            int jl = 0;
+            if (FK != FK_ANY) {
+                jl = f / kq_chunks;
+            } else {
 #pragma unroll 1
-        for (int w = 0; w < kCW; w++)
-            v += C.s_part[((size_t)w * 2 * 32 + r) * TT + t] +
-                 C.s_part[((size_t)w * 2 * 32 + 32 + r) * TT + t];
-        P.out[(size_t)t * C.H + i0 + r] = v;
+                for (int l = 0; l < ng - 1; l++)
+                    if (f >= __shfl_sync(kFullMask, cend, l)) jl = l + 1;
+            }
+            const int cbeg = __shfl_sync(kFullMask, cend - nch, jl & 31);
+            const uint32_t joff = __shfl_sync(kFullMask, off, jl & 31);
+            if (f >= total) continue;
+            const int p = f - cbeg;
+            const JobX &J = C.s_jobs[g0 + jl];
+            const int fmt = FK == FK_Q4K ? MOE_FMT_Q4_K : FK == FK_Q5K ? MOE_FMT_Q5_K : J.fmt;
+#pragma unroll
+            for (int rr = 0; rr < 2; rr++) {
+                const int r = warp + kCW * rr;
+                if (r >= rows) break;
+                const uint8_t *row = stage + joff + (size_t)r * J.stride[2];
+                if (FK == FK_ANY && small_block(fmt)) {
+                    const bool q80 = fmt == MOE_FMT_Q8_0;
+#pragma unroll 1
+                    for (int t = 0; t < J.n; t++) {
+                        const int slot = J.slot0 + t;
+                        const ActChunk a = load_act(C.s_hq + (size_t)slot * P.hpad, C.s_hd + slot * hb,
+                                                    C.s_hs + slot * hb, p, true);
+                        const float v = q80 ? q80_chunk_dot(row + (size_t)p * kQ80Bytes, a)
+                                            : q51_chunk_dot(row + (size_t)p * kQ51Bytes, a);
+                        const int tok = C.s_stok[slot];
+                        const float wv = C.s_sw[slot] * v;
+#pragma unroll
+                        for (int tt = 0; tt < TT; tt++)
+                            if (tt == tok) dacc[rr][tt] += wv;
+                    }
+                } else {
+                    const int SBB = fmt == MOE_FMT_Q5_K ? kQ5KBytes : kQ4KBytes;
+                    const int sb = p >> 3, j = p & 7;
+                    const WChunk w = fmt == MOE_FMT_Q5_K ? kq_chunk<true>(row + (size_t)sb * SBB, j)
+                                                         : kq_chunk<false>(row + (size_t)sb * SBB, j);
+                    const float mf = (j & 1) ? 0.f : 1.f;
+#pragma unroll 1
+                    for (int t = 0; t < J.n; t++) {
+                        const int slot = J.slot0 + t;
+                        const ActChunk a = load_act(C.s_hq + (size_t)slot * P.hpad, C.s_hd + slot * hb,
+                                                    C.s_hs + slot * hb, p, false);
+                        const float v = kq_chunk_dot(w, a, mf);
+                        const int tok = C.s_stok[slot];
+                        const float wv = C.s_sw[slot] * v;
+#pragma unroll
+                        for (int tt = 0; tt < TT; tt++)
+                            if (tt == tok) dacc[rr][tt] += wv;
+                    }
+                }
+            }
+        }
+        base = __shfl_sync(kFullMask, off + sz, ng - 1);
     }
 }
 
@@ -756,11 +843,11 @@ __device__ __forceinline__ void finish_down_unit(const DecParams &P, const Ctx &
 template <int NT, int TT, int FK>
 __device__ __forceinline__ void consumer(const DecParams &P, const Ctx &C) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int H = C.H, F = C.F;
+    const int H = C.H;
     int s = 0;
     uint32_t ph = 0;
-    bool gu_done = false, have_h = false, skip_down = false;
-    int done_blocks = 0;
+    bool have_h = false, skip_down = false;
+    float dacc[2][TT];   // down sums of this warp's rows (warp, warp + 16) per token
 #pragma unroll 1
     while (true) {
         if (!ptx::mbar_wait_bounded(&C.full[s], ph, kWaitNs)) {
@@ -768,15 +855,6 @@ __device__ __forceinline__ void consumer(const DecParams &P, const Ctx &C) {
             break;
         }
         const StageMeta m = C.meta[s];
-        if (m.kind != ST_GU && !gu_done) {
-            // publish this CTA's Q8_1(h) blocks
-            gu_done = true;
-            ptx::named_barrier(1, kCW * 32);
-            if (threadIdx.x == 0 && done_blocks > 0) {
-                __threadfence();
-                atomicAdd(&C.ctr[1], (uint32_t)done_blocks);
-            }
-        }
         if (m.kind == ST_END) break;
         const uint8_t *stage = C.ring + (size_t)s * P.stage_bytes;
         if (m.kind == ST_GU) {
@@ -807,8 +885,13 @@ __device__ __forceinline__ void consumer(const DecParams &P, const Ctx &C) {
             if (hrow0 == 16) {   // the block is complete: Q8_1 of its 32 rows, per slot
                 ptx::named_barrier(1, kCW * 32);
                 quantize_h_block(P, C, J, r0 / 32);
-                done_blocks++;
-                ptx::named_barrier(1, kCW * 32);   // s_h is rewritten by the next block
+                // every slot's Q8_1(h) of this block is written (and s_h is free for the next
+                // block): publish the block
+                ptx::named_barrier(1, kCW * 32);
+                if (threadIdx.x == 0) {
+                    __threadfence();
+                    atomicAdd(&C.ctr[1], 1u);
+                }
             }
         } else {   // ST_DOWN
             if (!have_h) {
@@ -816,75 +899,27 @@ __device__ __forceinline__ void consumer(const DecParams &P, const Ctx &C) {
                 have_h = true;
             }
             const int i0 = m.a, rows = m.b;
-            const int lpr = C.down_lpr, sr = lane / lpr;
-            float *part = C.s_part + (size_t)warp * 2 * 32 * TT;   // this warp's [2][32][TT]
-            if (m.c == 0) {   // first stage of a down unit: clear this warp's partials
-#pragma unroll 1
-                for (int i = lane; i < 2 * 32 * TT; i += 32) part[i] = 0.f;
-                __syncwarp();
+            if (m.c == 0) {   // first stage of a down unit
+#pragma unroll
+                for (int rr = 0; rr < 2; rr++)
+#pragma unroll
+                    for (int t = 0; t < TT; t++) dacc[rr][t] = 0.f;
             }
-            // items (job, row) of this stage, job-major; a lane group takes one item
-            const int nj = m.d - m.c, nitems = nj * rows;
-            const int per_pass = kCW * (32 / lpr);
-#pragma unroll 1
-            for (int base_i = warp * (32 / lpr); base_i < nitems && !skip_down; base_i += per_pass) {
-                const int it = base_i + sr;
-                const bool valid = it < nitems;
-                const int jl = valid ? it / rows : 0, r = valid ? it % rows : 0;
-                const JobX &J = C.s_jobs[m.c + jl];
-                uint32_t joff;
-                if (FK != FK_ANY) {
-                    joff = (uint32_t)jl * rows * J.stride[2];
-                } else {
-                    joff = 0;
-#pragma unroll 1
-                    for (int jj = m.c; jj < m.c + jl; jj++) joff += (uint32_t)rows * C.s_jobs[jj].stride[2];
-                }
-                const int Kd = (FK == FK_ANY && small_block(J.fmt)) ? ((F + 31) / 32) * 32 : P.hpad;
-                const uint8_t *const rp[1] = {valid ? stage + joff + (size_t)r * J.stride[2] : nullptr};
-                const int jn = valid ? J.n : 0;
-                int nmax = jn;
-                if (lpr == 16) nmax = max(nmax, __shfl_xor_sync(kFullMask, nmax, 16));
-#pragma unroll 1
-                for (int t0 = 0; t0 < nmax; t0 += NT) {
-                    const int n = max(0, min(NT, jn - t0));
-                    int act[NT];
-#pragma unroll
-                    for (int t = 0; t < NT; t++) act[t] = t < n ? J.slot0 + t0 + t : 0;
-                    float acc[1][NT];
-#pragma unroll
-                    for (int t = 0; t < NT; t++) acc[0][t] = 0.f;
-                    rows_dot<NT, 1, FK>(J.fmt, rp, Kd, C.s_hq, C.s_hd, C.s_hs, P.hpad, act, n, lpr, acc);
-#pragma unroll
-                    for (int t = 0; t < NT; t++) {
-                        float v = acc[0][t];
-                        if (lpr == 32) v += __shfl_xor_sync(kFullMask, v, 16);
-                        v += __shfl_xor_sync(kFullMask, v, 8);
-                        v += __shfl_xor_sync(kFullMask, v, 4);
-                        v += __shfl_xor_sync(kFullMask, v, 2);
-                        v += __shfl_xor_sync(kFullMask, v, 1);
-                        acc[0][t] = v;
-                    }
-                    // the lane groups write their own halves of the partials in turn
-                    if (lane % lpr == 0) {
-                        float *pr = part + (sr * 32 + r) * TT;
-#pragma unroll
-                        for (int t = 0; t < NT; t++) {
-                            if (t < n) {
-                                const int slot = J.slot0 + t0 + t;
-                                pr[C.s_stok[slot]] += C.s_sw[slot] * acc[0][t];
-                            }
-                        }
-                    }
-                    __syncwarp();
-                }
-            }
+            if (!skip_down) down_stage<TT, FK>(P, C, stage, rows, m.c, m.d, dacc);
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(&C.empty[s]);
-            if (m.e) {   // last stage of the unit: sum the partials in warp order, write
-                ptx::named_barrier(1, kCW * 32);
-                if (!skip_down) finish_down_unit<TT>(P, C, i0, rows);
-                ptx::named_barrier(1, kCW * 32);
+            if (m.e && !skip_down) {   // last stage of the unit: reduce across the lanes, write
+#pragma unroll
+                for (int rr = 0; rr < 2; rr++) {
+                    const int r = warp + kCW * rr;
+                    if (r >= rows) break;
+#pragma unroll
+                    for (int t = 0; t < TT; t++) {
+                        if (t >= C.T) break;
+                        const float v = warp_sum(dacc[rr][t]);
+                        if (lane == 0) P.out[(size_t)t * H + i0 + r] = v;
+                    }
+                }
             }
         }
         if (++s == P.nstages) {
@@ -910,11 +945,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_fused(const DecParams P)
     C.s_hq = reinterpret_cast<int8_t *>(sm + P.o_hq);
     C.s_hd = reinterpret_cast<float *>(sm + P.o_hd);
     C.s_hs = reinterpret_cast<float *>(sm + P.o_hs);
-    C.s_part = reinterpret_cast<float *>(sm + P.o_gu);
     C.s_h = reinterpret_cast<float *>(sm + P.o_h);
     C.s_misc = reinterpret_cast<int *>(sm + P.o_misc);
     C.full = reinterpret_cast<uint64_t *>(sm + P.o_bar);
     C.empty = C.full + P.nstages;
+    C.desc_bar = C.full + 32;
     C.meta = reinterpret_cast<StageMeta *>(sm + P.o_meta);
     C.ring = sm;
     C.ws = P.ws;
@@ -929,17 +964,24 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_fused(const DecParams P)
     C.hb = P.hpad / 32;
     C.nb32 = P.F / 32;
 
-    ptx::grid_dependency_wait();
-    ptx::launch_dependents();
     if (tid == 0) {
 #pragma unroll 1
         for (int s = 0; s < P.nstages; s++) {
             ptx::mbar_init(&C.full[s], 1);
             ptx::mbar_init(&C.empty[s], kCW);
         }
+        ptx::mbar_init(C.desc_bar, 1);
         ptx::fence_barrier_init();
         C.s_misc[2] = 0;
+        // the descriptor table is the arena's (not written by the previous kernel): fetch it
+        // now, in the background, before waiting for the previous grid
+        const uint32_t nb = (uint32_t)((P.E + P.shared) * sizeof(ExpertDev));
+        ptx::mbar_arrive_expect_tx(C.desc_bar, nb);
+        ptx::bulk_g2s(desc_table(sm, P.E, P.T, P.k), P.experts, nb, C.desc_bar,
+                      ptx::policy_evict_last());
     }
+    ptx::grid_dependency_wait();
+    ptx::launch_dependents();
     prologue<VPL>(P, C, sm);
     // the prologue scratch in the stage ring is dead from here on
     const int G = gridDim.x, cta = blockIdx.x;
@@ -949,12 +991,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_fused(const DecParams P)
     // down rows: computed after the barrier by every CTA, so split evenly
     C.i_lo = (int)((long long)P.H * cta / G);
     C.i_hi = (int)((long long)P.H * (cta + 1) / G);
-    // down: rows with <= 16 chunks are handled by 16-lane groups (two items per warp)
-    int kmax_down = 0;
-#pragma unroll 1
-    for (int u = 0; u < C.U; u++)
-        kmax_down = max(kmax_down, small_block(C.s_jobs[u].fmt) ? (P.F + 31) / 32 : P.hpad / 32);
-    C.down_lpr = kmax_down <= 16 ? 16 : 32;
 
     if (warp == kCW) {
         if ((tid & 31) == 0) producer(P, C);
@@ -1037,14 +1073,14 @@ cudaError_t launch_decode_fused(const FfnArgs &a, int E, int shared, const float
     P.hpad = a.hpad;
     P.max_jobs = a.max_jobs;
     P.slots = a.T * a.k + a.T;
+    P.keep_h = a.h != nullptr;
     auto al = [](int v, int q) { return (v + q - 1) / q * q; };
-    const int tt = a.T <= 1 ? 1 : a.T <= 4 ? 4 : 16;
     const int fk = a.fmt_mask == (1 << MOE_FMT_Q4_K) ? FK_Q4K
                    : a.fmt_mask == (1 << MOE_FMT_Q5_K) ? FK_Q5K : FK_ANY;
     P.stage_bytes = al(std::max(2 * kUnitPairs * max_s01, kDownRowsMax * max_s2), 1024);
     const int slots = P.slots;
     const int sizes[] = {
-        2 * 16 * 8,                                  // barriers (<= 16 stages)
+        2 * 16 * 8 + 16,                             // barriers (<= 16 stages) + descriptors
         16 * (int)sizeof(StageMeta),                 // stage meta
         al(a.T * a.H, 128),                          // xq
         al(a.T * (a.H / 32) * 4, 16),                // xd
@@ -1055,7 +1091,7 @@ cudaError_t launch_decode_fused(const FfnArgs &a, int E, int shared, const float
         al(slots * a.hpad, 128),                     // Q8_1(h) q
         al(slots * (a.hpad / 32) * 4, 16),           // Q8_1(h) d
         al(slots * (a.hpad / 32) * 4, 16),           // Q8_1(h) xd*sum(q)
-        kCW * 2 * 32 * tt * 4,                       // down partials [kCW][2][32][TT]
+        16,                                          // (unused)
         32 * 16 * 4,                                 // one block of h [32][16]
         16,                                          // (unused)
         64};                                         // misc

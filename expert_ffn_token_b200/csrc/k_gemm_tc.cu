@@ -24,10 +24,13 @@
 //     the offsets through the min term with wm_j = -m_j (an fp16 value, exact in tf32).
 // Results agree with the exact sums up to fp32 rounding.
 //
-// Roles (576 threads): warp 0 issues TMA loads (packed weights as stored, activations, scales);
-// warp 1 allocates tensor memory and issues the MMAs; warps 2-9 unpack the packed weights into
-// the fp16 operand (128-byte swizzled, K-major) and the per-row scales; warps 10-17 read the
-// accumulators and finish the tile (SwiGLU + Q8_1(h), or the weighted scatter into out).  All
+// Roles (608 threads): warp 0 issues the TMA loads of the packed weights, the activation
+// scales and the min-term operands, as far ahead as their rings allow; warp 18 issues the
+// activation tiles into the operand stages (two producers, so that neither ring waits on the
+// other); warp 1 allocates tensor memory and issues the MMAs; warps 2-9 unpack the packed
+// weights into the fp16 operand (128-byte swizzled, K-major) and the per-row scales; warps
+// 10-17 read the accumulators and finish the tile (SwiGLU + Q8_1(h), or the weighted scatter
+// into out).  All
 // hand-offs are mbarriers; every wait is bounded and a timeout ends the kernel with
 // MOE_ERR_TIMEOUT.
 #include <cuda.h>
@@ -57,7 +60,8 @@ constexpr int kGrp = 3;            // accumulator groups: one per 64-wide stage 
 constexpr int kMinBuf = 2;         // min-term accumulators, one per tile
 constexpr int kUnpackWarps = 8;    // two threads per weight row, one sub-block each per stage
 constexpr int kEpiWarp0 = 2 + kUnpackWarps;
-constexpr int kThreads = (kEpiWarp0 + 8) * 32;
+constexpr int kActWarp = kEpiWarp0 + 8;        // issues the activation-tile loads
+constexpr int kThreads = (kActWarp + 1) * 32;
 constexpr uint64_t kWaitNs = 2000000000ull;
 
 // A 128-wide stage holds two 128-byte swizzle atoms of each operand along K:
@@ -252,9 +256,11 @@ __device__ __forceinline__ float ld_half(const uint8_t *p) {
     return __half2float(*reinterpret_cast<const __half *>(p));
 }
 
-// ---------------------------------------------------------------- warp 0: TMA producer
+// ---------------------------------------------------------------- warps 0 and 18: TMA producers
 
-template <int PHASE>
+// WHICH 0: packed weight rows + xd per super-block, and the min-term activation operands;
+// WHICH 1: the fp16 activation tiles of every 128-wide operand stage.
+template <int PHASE, int WHICH>
 __device__ void role_producer(const GemmArgs &a, const Smem &S, int nj, const CUtensorMap *mx,
                               const CUtensorMap *md, const CUtensorMap *msh,
                               const CUtensorMap *msl) {
@@ -278,6 +284,19 @@ __device__ void role_producer(const GemmArgs &a, const Smem &S, int nj, const CU
             yb = ya + 64;
         }
         for (int sb = 0; sb < nsb; sb++) {
+            if (WHICH == 1) {
+                for (int st = 0; st < 2; st++) {
+                    if (!wait_fast(S.w_empty + rw.s, rw.ph ^ 1u, S.abort, a.status)) return;
+                    uint8_t *ws = S.w + rw.s * kWStage + 2 * kA16;
+                    mbar_arrive_expect_tx(S.w_full + rw.s, (uint32_t)t.nbox * 8192u);
+                    for (int at = 0; at < 2; at++)
+                        for (int b = 0; b < t.nbox; b++)
+                            tma_load_2d(ws + at * kB16 + b * 4096, mx, (sb * 4 + 2 * st + at) * 64,
+                                        t.slot_base + 32 * b, S.w_full + rw.s);
+                    rw.adv(kWSt);
+                }
+                continue;
+            }
             if (!wait_fast(S.raw_empty + rr.s, rr.ph ^ 1u, S.abort, a.status)) return;
             uint8_t *rs = S.raw + rr.s * a.raw_stage;
             mbar_arrive_expect_tx(S.raw_full + rr.s, 128u * sbb + (uint32_t)t.nbox * 1024u);
@@ -300,16 +319,6 @@ __device__ void role_producer(const GemmArgs &a, const Smem &S, int nj, const CU
                                 t.slot_base + 32 * b, S.mn_full + rm.s);
                 }
                 rm.adv(kMnSt);
-            }
-            for (int st = 0; st < 2; st++) {
-                if (!wait_fast(S.w_empty + rw.s, rw.ph ^ 1u, S.abort, a.status)) return;
-                uint8_t *ws = S.w + rw.s * kWStage + 2 * kA16;
-                mbar_arrive_expect_tx(S.w_full + rw.s, (uint32_t)t.nbox * 8192u);
-                for (int at = 0; at < 2; at++)
-                    for (int b = 0; b < t.nbox; b++)
-                        tma_load_2d(ws + at * kB16 + b * 4096, mx, (sb * 4 + 2 * st + at) * 64,
-                                    t.slot_base + 32 * b, S.w_full + rw.s);
-                rw.adv(kWSt);
             }
         }
     }
@@ -910,7 +919,10 @@ __global__ void __maxnreg__(96)
     const int nj = *a.njobs;
 
     if (warp == 0) {
-        if (lane == 0) role_producer<PHASE>(a, S, nj, &map_x, &map_d, &map_sh, &map_sl);
+        if (lane == 0) role_producer<PHASE, 0>(a, S, nj, &map_x, &map_d, &map_sh, &map_sl);
+        __syncwarp();
+    } else if (warp == kActWarp) {
+        if (lane == 0) role_producer<PHASE, 1>(a, S, nj, &map_x, &map_d, &map_sh, &map_sl);
         __syncwarp();
     } else if (warp == 1) {
         if (lane == 0) {

@@ -367,6 +367,7 @@ moe_status moe_forward(const moe_arena *arena, const float *d_x, const float *d_
         a.fmt_mask = arena->fmt_mask;
         a.max_stride01 = arena->max_stride01;
         a.max_stride2 = arena->max_stride2;
+        a.h = (flags & MOE_F_KEEP_H) ? reinterpret_cast<float *>(ws + L.h) : nullptr;
         bool taken = false;
         cudaError_t e = launch_decode_fused(a, E, shared, d_x, d_logits, ws, L, L.sync, L.blkcnt,
                                             true, st, &taken);
