@@ -243,6 +243,12 @@ __device__ __forceinline__ bool wait_bar_warp(uint64_t *bar, uint32_t parity, in
     return __all_sync(0xFFFFFFFFu, ok);
 }
 
+// silu(g) * u with the fast exponential and divide: relative error ~1e-6, far inside the
+// layer's tolerance (the Q8_1 rounding of h applies to whatever h is computed).
+__device__ __forceinline__ float silu_mul_fast(float g, float u) {
+    return __fdividef(g, 1.0f + __expf(-g)) * u;
+}
+
 __device__ __forceinline__ float tf32_round(float x) {
     return __uint_as_float((__float_as_uint(x) + 0x1000u) & 0xFFFFE000u);
 }
@@ -662,12 +668,26 @@ __device__ __noinline__ void quantize_h_block(const GemmArgs &a, const float *v3
     const float d = __fdiv_rn(am, 127.0f);
     int q[32];
     int sum = 0;
+    if (fin && d != 0.0f) {
+        // q = round-half-away(RN(v / d)).  For normal d, v * RN(1/d) is within 2 ulp of
+        // RN(v / d), and |v / d| <= 127 makes 2 ulp < 2^-15: unless the product lies that close
+        // to a half-integer, both round to the same integer.  The rare close cases, and a
+        // subnormal d, take the IEEE division.
+        const bool fast = d >= 0x1p-125f;
+        const float inv = __frcp_rn(d);
 #pragma unroll
-    for (int i = 0; i < 32; i++) {
-        int qi = 0;
-        if (fin && d != 0.0f) qi = max(-127, min(127, (int)roundf(__fdiv_rn(v[i], d))));
-        q[i] = qi;
-        sum += qi;
+        for (int i = 0; i < 32; i++) {
+            const float r = v[i] * inv;
+            const float a = fabsf(r);
+            const bool near_tie = !fast || fabsf(a - floorf(a) - 0.5f) < 0x1p-15f;
+            const float rq = near_tie ? __fdiv_rn(v[i], d) : r;
+            const int qi = max(-127, min(127, (int)roundf(rq)));
+            q[i] = qi;
+            sum += qi;
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 32; i++) q[i] = 0;
     }
     const int hb = a.hpad / 32;
     const size_t bi = (size_t)slot * hb + f0 / 32;
@@ -822,7 +842,7 @@ __device__ void role_epilogue(const GemmArgs &a, const Smem &S, int nj, uint32_t
                 if (!wait_bar_warp(S.xb_full + pi, rx.ph, S.abort, a.status)) return;
 #pragma unroll
                 for (int c = 0; c < 32; c++)
-                    xb[c * kXbPitch + lane] = silu_mul(acc[c], xb[c * kXbPitch + lane]);
+                    xb[c * kXbPitch + lane] = silu_mul_fast(acc[c], xb[c * kXbPitch + lane]);
                 __syncwarp();
                 const int f0 = t.mt * 64 + 32 * p;
                 if (lane < ncol && f0 < a.F)
