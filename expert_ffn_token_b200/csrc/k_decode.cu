@@ -858,26 +858,37 @@ __device__ __forceinline__ void consumer(const DecParams &P, const Ctx &C) {
         if (m.kind == ST_END) break;
         const uint8_t *stage = C.ring + (size_t)s * P.stage_bytes;
         if (m.kind == ST_GU) {
-            // warp w computes gate row r0+w and up row r0+w for every token of the job
+            // the two halves of a 32-row block go to the two groups of 8 warps, so that the
+            // second half is computed while the first still is; warp w8 of the group computes
+            // gate and up rows w8 and w8 + 8 of its half, for every token of the job
             const int ju = m.a, r0 = m.b;
             const JobX &J = C.s_jobs[ju];
             const int hrow0 = r0 & 31;   // 0 or 16 inside the block
-            const uint8_t *const rp[2] = {stage + (size_t)warp * J.stride[0],
-                                          stage + 16u * J.stride[0] + (size_t)warp * J.stride[1]};
+            const int w8 = warp & 7;
+            if ((hrow0 >> 4) == (warp >> 3)) {
+                const uint32_t s0 = J.stride[0], s1 = J.stride[1];
+                const uint8_t *const rp[4] = {stage + (size_t)w8 * s0, stage + 16u * s0 + (size_t)w8 * s1,
+                                              stage + (size_t)(w8 + 8) * s0,
+                                              stage + 16u * s0 + (size_t)(w8 + 8) * s1};
 #pragma unroll 1
-            for (int t0 = 0; t0 < J.n; t0 += NT) {
-                const int n = min(NT, J.n - t0);
-                int act[NT];
+                for (int t0 = 0; t0 < J.n; t0 += NT) {
+                    const int n = min(NT, J.n - t0);
+                    int act[NT];
 #pragma unroll
-                for (int t = 0; t < NT; t++) act[t] = t < n ? C.s_stok[J.slot0 + t0 + t] : 0;
-                float acc[2][NT];
+                    for (int t = 0; t < NT; t++) act[t] = t < n ? C.s_stok[J.slot0 + t0 + t] : 0;
+                    float acc[4][NT];
 #pragma unroll
-                for (int t = 0; t < NT; t++) acc[0][t] = acc[1][t] = 0.f;
-                rows_dot<NT, 2, FK>(J.fmt, rp, H, C.s_xq, C.s_xd, C.s_xs, H, act, n, 32, acc);
+                    for (int t = 0; t < NT; t++) acc[0][t] = acc[1][t] = acc[2][t] = acc[3][t] = 0.f;
+                    rows_dot<NT, 4, FK>(J.fmt, rp, H, C.s_xq, C.s_xd, C.s_xs, H, act, n, 32, acc);
 #pragma unroll
-                for (int t = 0; t < NT; t++) {
-                    const float g = warp_sum(acc[0][t]), u = warp_sum(acc[1][t]);
-                    if (lane == 0 && t < n) C.s_h[(hrow0 + warp) * 16 + t0 + t] = silu_mul(g, u);
+                    for (int t = 0; t < NT; t++) {
+                        const float g0 = warp_sum(acc[0][t]), u0 = warp_sum(acc[1][t]);
+                        const float g1 = warp_sum(acc[2][t]), u1 = warp_sum(acc[3][t]);
+                        if (lane == 0 && t < n) {
+                            C.s_h[(hrow0 + w8) * 16 + t0 + t] = silu_mul(g0, u0);
+                            C.s_h[(hrow0 + w8 + 8) * 16 + t0 + t] = silu_mul(g1, u1);
+                        }
+                    }
                 }
             }
             __syncwarp();
