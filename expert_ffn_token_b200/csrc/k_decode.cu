@@ -101,10 +101,13 @@ __device__ __forceinline__ ActChunk load_act(const int8_t *q, const float *d, co
         const int bl = sb * 8 + 2 * c;
         a.xa = *reinterpret_cast<const int4 *>(q + kl);
         a.xb = *reinterpret_cast<const int4 *>(q + kl + 32);
-        a.dl = d[bl];
-        a.dh = d[bl + 1];
-        a.sl = s[bl];
-        a.sh = s[bl + 1];
+        // bl is even and K-quant rows hold a multiple of 8 blocks: 8-byte aligned pairs
+        const float2 dd = *reinterpret_cast<const float2 *>(d + bl);
+        const float2 ss = *reinterpret_cast<const float2 *>(s + bl);
+        a.dl = dd.x;
+        a.dh = dd.y;
+        a.sl = ss.x;
+        a.sh = ss.y;
     }
     return a;
 }
