@@ -121,6 +121,27 @@ def traffic_for(kernel: str, workload: str):
     return d["bytes_per_launch"] if d.get("source_sha256") == h.hexdigest() else None
 
 
+# ------------------------------------------------------------------ ranks
+
+
+def max_over_ranks(v: float, world: int, device=None) -> float:
+    """The largest value over all ranks (the job's time), the same on every rank.  Every rank
+    must call it at the same point (it is a collective)."""
+    if world <= 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank_step: float, steps: int, world: int, ms: float) -> float:
+    """Units per second of the whole job: every rank processes units_per_rank_step per step
+    (weak scaling), the job takes ms (the max over ranks) for `steps` steps."""
+    return world * units_per_rank_step * steps / (ms / 1e3)
+
+
 # ------------------------------------------------------------------ workload set-up
 
 
@@ -264,9 +285,7 @@ def run_ours(args, rank, world):
         gateup_ms = statistics.mean(t[0].elapsed_time(t[1]) for row in step_events for t in row)
         down_ms = statistics.mean(t[1].elapsed_time(t[2]) for row in step_events for t in row)
     if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+        ms = max_over_ranks(ms, world, dev)
         dist.barrier()
     clk = clocks.stop()
 
@@ -291,10 +310,7 @@ def run_ours(args, rank, world):
     f1.record()
     torch.cuda.synchronize()
     ms_e2e = f0.elapsed_time(f1)
-    if world > 1:
-        t = torch.tensor([ms_e2e], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_e2e = float(t.item())
+    ms_e2e = max_over_ranks(ms_e2e, world, dev)
     assert np.isfinite(out_h.numpy()).all()
 
     st = moe.read_status(ws.data_ptr(), stream)   # status word sits at workspace offset 0
@@ -330,7 +346,7 @@ def run_ours(args, rank, world):
                     "flops_per_launch": flops, "ms_per_launch": gateup_ms,
                     "frac_of_int8_peak": achieved / (2 * bf16),
                     "down_kernel_ms_per_launch": down_ms}
-    value = world * tok_per_step * K / (ms / 1e3)
+    value = job_throughput(tok_per_step, K, world, ms)
     result = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
         "warmup": W, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
@@ -346,7 +362,7 @@ def run_ours(args, rank, world):
         "expert_gbs": step_bytes / (ms_step / 1e3) / 1e9,
         "int8_tops": step_ops / (ms_step / 1e3) / 1e12,
         "roofline": roofline,
-        "e2e": {"value": world * tok_per_step * K2 / (ms_e2e / 1e3), "unit": "tokens/s",
+        "e2e": {"value": job_throughput(tok_per_step, K2, world, ms_e2e), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(xs.nbytes + lgs.nbytes),
                 "d2h_bytes_per_step": int(out_h.numel() * 4)},
         "gpu_launches": int(kernels_per_step * K),
@@ -372,7 +388,7 @@ def oracle_sample(w, seconds, max_layers=None):
     layers = 0
     sample_tokens = w.tokens if w.tokens <= 64 else 16
     l = 0
-    while t_total < seconds and (max_layers is None or layers < max_layers):
+    while (layers == 0 or t_total < seconds) and (max_layers is None or layers < max_layers):
         layer = l % w.layers
         x = synth.activations(w, layer)
         logits = synth.router_logits(w, layer)

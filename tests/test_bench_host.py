@@ -1,0 +1,87 @@
+"""Host-side checks of bench.py that need no GPU: the reference arm (the CPU oracle), its
+rank handling under torchrun, and the multi-rank reduction and job throughput on two gloo
+ranks on the CPU."""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+
+
+def _run_bench(args, env_extra=None, timeout=300):
+    env = dict(os.environ)
+    env.update(env_extra or {})
+    return subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), *args], cwd=ROOT,
+                          env=env, capture_output=True, text=True, timeout=timeout)
+
+
+def test_reference_arm_prints_one_line():
+    r = _run_bench(["--impl", "reference", "--steps", "1", "--warmup", "1", "--cpu-seconds", "1"])
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["value"] > 0 and d["unit"] == "tokens/s"
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["e2e"] == {"value": d["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
+    assert d["steps"] == 1 and d["warmup"] == 1 and d["higher_is_better"] is True
+
+
+def test_reference_arm_other_ranks_exit_quietly():
+    r = _run_bench(["--impl", "reference", "--steps", "1", "--warmup", "1"],
+                   {"RANK": "1", "WORLD_SIZE": "2"})
+    assert r.returncode == 0 and r.stdout.strip() == ""
+
+
+def test_oracle_sample_runs_at_least_one_layer():
+    w = bench.workload("decode")
+    s = bench.oracle_sample(w, 0.0, max_layers=1)
+    assert s["value"] > 0 and s["sample"].startswith("1 layer(s)")
+
+
+def test_job_throughput_counts_every_rank():
+    # 48 layer-tokens per step on each of 4 ranks, 10 steps in 20 ms -> 96,000 tokens/s
+    assert bench.job_throughput(48, 10, 4, 20.0) == pytest.approx(96000.0)
+    assert bench.max_over_ranks(3.5, 1) == 3.5
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank(rank, world, port, q):
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        ms = bench.max_over_ranks(10.0 + 5.0 * rank, world)
+        q.put((rank, ms, bench.job_throughput(48, 10, world, ms)))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_two_gloo_ranks():
+    import multiprocessing as mp
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    got = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    # both ranks see the slower rank's 15 ms; the job processed 2 x 48 x 10 tokens in it
+    assert [g[1] for g in got] == [15.0, 15.0]
+    assert got[0][2] == pytest.approx(2 * 48 * 10 / 0.015)
