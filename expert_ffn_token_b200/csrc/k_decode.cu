@@ -28,7 +28,7 @@
 // Every wait is bounded by %globaltimer and reports MOE_ERR_TIMEOUT instead of hanging.  The
 // down phase waits on the gate/up work of every CTA: the grid is one CTA per SM (all resident
 // together; a programmatically launched successor starts only once every CTA here has
-// started).  The last CTA to finish resets the counters.
+// started).  The last CTA to pass the grid-wide wait resets the counters.
 #include "dot.cuh"
 #include "ptx.cuh"
 #include "route_dev.cuh"
@@ -467,6 +467,89 @@ __device__ __forceinline__ void prologue(const DecParams &P, Ctx &C, uint8_t *sm
         for (int t = warp; t < T; t += kCW + 1)
             warp_topk_reg<VPL>(P.logits + (size_t)t * E, E, k, s_ids + t * k, s_wt + t * k, st);
     }
+    if (T == 1 && k <= 32) {
+        // One token: its k experts are distinct, so warp 0 (which chose them) builds the job
+        // list in registers -- one job per expert in ascending id, one slot each -- while the
+        // other warps finish quantizing x.
+        if (warp == 0) {
+            const bool v = lane < k;
+            const int id = v ? s_ids[lane] : 0x7FFFFFFF;
+            int rank = 0;
+#pragma unroll 1
+            for (int i = 0; i < k; i++) rank += __shfl_sync(kFullMask, id, i) < id ? 1 : 0;
+            JobX *jobs = C.s_jobs;
+            if (v) {
+                JobX &J = jobs[rank];
+                J.expert = id;
+                J.slot0 = rank;
+                J.n = 1;
+                J.shared = 0;
+                C.s_stok[rank] = 0;
+                C.s_sw[rank] = s_wt[lane];
+                if (cta0) {
+                    reinterpret_cast<int32_t *>(ws + L.ids)[lane] = id;
+                    reinterpret_cast<float *>(ws + L.w)[lane] = s_wt[lane];
+                    reinterpret_cast<int32_t *>(ws + L.perm)[rank] = lane;
+                    reinterpret_cast<int32_t *>(ws + L.inv_perm)[lane] = rank;
+                }
+            }
+            const int U = k + (P.shared ? 1 : 0);
+            if (lane == 0) {
+                if (P.shared) {
+                    JobX &J = jobs[k];
+                    J.expert = E;
+                    J.slot0 = k;
+                    J.n = 1;
+                    J.shared = 1;
+                }
+                C.s_stok[k] = 0;
+                C.s_sw[k] = 1.0f;
+                C.s_misc[0] = U;
+            }
+            __syncwarp();
+            if (!ptx::mbar_wait_bounded(C.desc_bar, 0, kWaitNs) && lane == 0)
+                set_status(status, MOE_ERR_TIMEOUT);
+#pragma unroll 1
+            for (int u = lane; u < U; u += 32) {
+                JobX &J = jobs[u];
+                const ExpertDev &ex = s_ex[J.expert];
+                J.m[0] = ex.m[0];
+                J.m[1] = ex.m[1];
+                J.m[2] = ex.m[2];
+                J.stride[0] = ex.stride[0];
+                J.stride[1] = ex.stride[1];
+                J.stride[2] = ex.stride[2];
+                J.fmt = ex.fmt;
+            }
+        }
+        __syncthreads();
+        if (cta0) {   // the intermediates of a1-a3 in the workspace
+            const int U = C.s_misc[0];
+#pragma unroll 1
+            for (int i = tid; i < H / 16; i += kThreads)
+                reinterpret_cast<int4 *>(ws + L.xq)[i] = reinterpret_cast<const int4 *>(C.s_xq)[i];
+#pragma unroll 1
+            for (int e = tid; e < E; e += kThreads) {
+                int c = 0, o = 0;
+#pragma unroll 1
+                for (int i = 0; i < k; i++) {
+                    const int x = s_ids[i];
+                    c += x == e ? 1 : 0;
+                    o += x < e ? 1 : 0;
+                }
+                reinterpret_cast<int32_t *>(ws + L.counts)[e] = c;
+                reinterpret_cast<int32_t *>(ws + L.offsets)[e] = o;
+            }
+            if (tid == 0) reinterpret_cast<int32_t *>(ws + L.offsets)[E] = k;
+#pragma unroll 1
+            for (int u = tid; u < U; u += kThreads) {
+                const JobX &J = C.s_jobs[u];
+                reinterpret_cast<Job *>(ws + L.jobs)[u] = Job{J.expert, J.slot0, J.n, J.shared};
+            }
+            if (tid == 0) *reinterpret_cast<int32_t *>(ws + L.njobs) = U;
+        }
+        return;
+    }
     __syncthreads();
     // ---- a3: counts and an expert bitmap, then one warp builds offsets and jobs
     const int A = T * k;
@@ -709,7 +792,8 @@ __device__ __forceinline__ void quantize_h_block(const DecParams &P, const Ctx &
 
 // After this CTA's gate/up work: wait (bounded) until every block of h is published, then stage
 // every slot's Q8_1(h) in shared memory.  Returns false on timeout.
-__device__ __forceinline__ bool wait_and_stage_h(const DecParams &P, const Ctx &C) {
+__device__ __forceinline__ bool wait_and_stage_h(const DecParams &P, const Ctx &C,
+                                                 uint32_t &arrived) {
     const int ctid = threadIdx.x;
     const WsLayout &L = P.L;
     if (ctid == 0) {
@@ -725,6 +809,11 @@ __device__ __forceinline__ bool wait_and_stage_h(const DecParams &P, const Ctx &
         }
         C.s_misc[2] = to;
         if (to) set_status(C.status, MOE_ERR_TIMEOUT);
+        // this CTA is past the grid-wide wait: count it.  The CTA that counts last resets both
+        // counters for the next launch; its result is read only at the end of the consumer, so
+        // the atomic's latency hides behind the down pass.
+        arrived = atomicAdd(&C.ctr[2], 1u);
+        C.s_misc[5] = 1;
     }
     ptx::named_barrier(1, kCW * 32);
     const int8_t *g_hq = reinterpret_cast<const int8_t *>(P.ws + L.hq);
@@ -850,6 +939,7 @@ __device__ __forceinline__ void consumer(const DecParams &P, const Ctx &C) {
     int s = 0;
     uint32_t ph = 0;
     bool have_h = false, skip_down = false;
+    uint32_t arrived = 0;
     float dacc[2][TT];   // down sums of this warp's rows (warp, warp + 16) per token
 #pragma unroll 1
     while (true) {
@@ -909,7 +999,7 @@ __device__ __forceinline__ void consumer(const DecParams &P, const Ctx &C) {
             }
         } else {   // ST_DOWN
             if (!have_h) {
-                skip_down = !wait_and_stage_h(P, C);
+                skip_down = !wait_and_stage_h(P, C, arrived);
                 have_h = true;
             }
             const int i0 = m.a, rows = m.b;
@@ -940,6 +1030,10 @@ __device__ __forceinline__ void consumer(const DecParams &P, const Ctx &C) {
             s = 0;
             ph ^= 1u;
         }
+    }
+    if (threadIdx.x == 0 && have_h && arrived == gridDim.x - 1) {
+        C.ctr[1] = 0;
+        C.ctr[2] = 0;
     }
 }
 
@@ -987,6 +1081,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_fused(const DecParams P)
         ptx::mbar_init(C.desc_bar, 1);
         ptx::fence_barrier_init();
         C.s_misc[2] = 0;
+        C.s_misc[5] = 0;
         // the descriptor table is the arena's (not written by the previous kernel): fetch it
         // now, in the background, before waiting for the previous grid
         const uint32_t nb = (uint32_t)((P.E + P.shared) * sizeof(ExpertDev));
@@ -1011,13 +1106,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_fused(const DecParams P)
     } else {
         consumer<NT, TT, FK>(P, C);
     }
-    __syncthreads();
-    if (tid == 0) {
-        __threadfence();
+    // A CTA that never reached the grid-wide wait (no down rows, or an early timeout) is
+    // counted here.  Its blocks were published before: either some other CTA saw all of them
+    // at the wait before counting, or this is the last CTA and all the others did.
+    if (tid == 0 && C.s_misc[5] == 0) {
         if (atomicAdd(&C.ctr[2], 1u) == gridDim.x - 1) {
             C.ctr[1] = 0;
             C.ctr[2] = 0;
-            __threadfence();
         }
     }
 }
