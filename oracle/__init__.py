@@ -52,6 +52,11 @@ def lib():
         L.oracle_forward.argtypes = [P, P, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                      ctypes.c_int, P, P, P, ctypes.c_int, ctypes.c_int, P,
                                      ctypes.c_int, P, P]
+        L.oracle_forward_gated.argtypes = [P, P, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                           ctypes.c_int, P, P, P, ctypes.c_int, ctypes.c_int, P,
+                                           ctypes.c_int, P, P, P]
+        L.oracle_router.argtypes = [P, P, ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P]
+        L.oracle_shared_gate.argtypes = [P, P, ctypes.c_int, ctypes.c_int, P]
         L.oracle_set_threads.argtypes = [ctypes.c_int]
         L.oracle_half_to_double.argtypes = [ctypes.c_uint16]
         L.oracle_half_to_double.restype = ctypes.c_double
@@ -174,9 +179,36 @@ def expert_ffn(arena: np.ndarray, expert: np.ndarray, hidden: int, ffn: int, xha
     return out
 
 
+def router(x: np.ndarray, Wr: np.ndarray):
+    """O10: router logits of x [T][H] and rows Wr [E][H]: (fp32 [T][E], fp64 sums [T][E])."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    Wr = np.ascontiguousarray(Wr, dtype=np.float32)
+    T, H = x.shape
+    E = Wr.shape[0]
+    assert Wr.shape[1] == H
+    l32 = np.empty((T, E), np.float32)
+    l64 = np.empty((T, E), np.float64)
+    if lib().oracle_router(_p(x), _p(Wr), T, H, E, _p(l32), _p(l64)) != 0:
+        raise ValueError("oracle_router: bad arguments")
+    return l32, l64
+
+
+def shared_gate(x: np.ndarray, wg: np.ndarray) -> np.ndarray:
+    """O11: the shared-expert gate sigmoid(x . wg) per token, fp64 [T]."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    wg = np.ascontiguousarray(wg, dtype=np.float32)
+    T, H = x.shape
+    assert wg.shape == (H,)
+    g = np.empty(T, np.float64)
+    if lib().oracle_shared_gate(_p(x), _p(wg), T, H, _p(g)) != 0:
+        raise ValueError("oracle_shared_gate: bad arguments")
+    return g
+
+
 def forward(arena: np.ndarray, experts: np.ndarray, shared: int, hidden: int, ffn: int,
-            x: np.ndarray, ids: np.ndarray, w: np.ndarray, tokens=None):
-    """O1-O9: (out fp32, out fp64), one row per listed token (all tokens if `tokens` is None)."""
+            x: np.ndarray, ids: np.ndarray, w: np.ndarray, tokens=None, gate=None):
+    """O1-O9: (out fp32, out fp64), one row per listed token (all tokens if `tokens` is None).
+    With `gate` (fp64 [T], from shared_gate) the shared expert's output is scaled by it (O11)."""
     arena = np.ascontiguousarray(arena, dtype=np.uint8)
     experts = np.ascontiguousarray(experts, dtype=EXPERT_DTYPE)
     x = np.ascontiguousarray(x, dtype=np.float32)
@@ -192,8 +224,15 @@ def forward(arena: np.ndarray, experts: np.ndarray, shared: int, hidden: int, ff
         tp = _p(tokens)
     out = np.empty((n, hidden), np.float32)
     out64 = np.empty((n, hidden), np.float64)
-    rc = lib().oracle_forward(_p(arena), _p(experts), len(experts), shared, hidden, ffn, _p(x),
-                              _p(ids), _p(w), T, k, tp, n, _p(out), _p(out64))
+    if gate is None:
+        rc = lib().oracle_forward(_p(arena), _p(experts), len(experts), shared, hidden, ffn,
+                                  _p(x), _p(ids), _p(w), T, k, tp, n, _p(out), _p(out64))
+    else:
+        gate = np.ascontiguousarray(gate, dtype=np.float64)
+        assert gate.shape == (T,)
+        rc = lib().oracle_forward_gated(_p(arena), _p(experts), len(experts), shared, hidden,
+                                        ffn, _p(x), _p(ids), _p(w), T, k, tp, n, _p(gate),
+                                        _p(out), _p(out64))
     if rc != 0:
         raise ValueError("oracle_forward: bad arguments")
     return out, out64

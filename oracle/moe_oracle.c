@@ -25,6 +25,11 @@
  *   O7  Q8_1 of fp32(h), zero-padded to the down rows' stored width
  *   O8  down rows times the dequantized Q8_1(h), in fp64
  *   O9  out[t] = sum_j w[t][j] * y[t][e_j] + y[t][shared], in fp64, stored as fp32
+ *   O10 router logits[t][e] = sum_h x[t][h] * Wr[e][h] of the fp32 hidden state and fp32
+ *       router rows, summed in fp64 in h order, stored as fp32 (the per-token router the
+ *       engine keeps on the GPU, "Strata: a 125B MoE at 94 tok/s on a 12 GB Card")
+ *   O11 optional shared-expert gate: g[t] = 1 / (1 + exp(-sum_h x[t][h] * wg[h])) in fp64;
+ *       with it, O9's shared term is g[t] * y[t][shared]
  *
  * Nothing here is blocked, fused or reordered beyond these definitions.  Per-token work may run
  * on several OpenMP threads; every token's arithmetic is the same whatever the thread count.
@@ -359,6 +364,39 @@ int oracle_expert_ffn(const uint8_t *arena, const oracle_expert *ex, int hidden,
     return 0;
 }
 
+/* O10: logits [T][E] (fp32, and the fp64 sums when l64 is not NULL) of x [T][H] and the
+ * router rows Wr [E][H].  Returns 0, or -1 for bad arguments.                                */
+int oracle_router(const float *x, const float *Wr, int T, int H, int E, float *l32,
+                  double *l64) {
+    if (T < 0 || H <= 0 || E <= 0 || !x || !Wr || !l32) return -1;
+    for (int t = 0; t < T; t++) {
+        for (int e = 0; e < E; e++) {
+            double s = 0.0;
+            for (int h = 0; h < H; h++)
+                s += (double)x[(int64_t)t * H + h] * (double)Wr[(int64_t)e * H + h];
+            l32[(int64_t)t * E + e] = (float)s;
+            if (l64) l64[(int64_t)t * E + e] = s;
+        }
+    }
+    return 0;
+}
+
+/* O11: the shared-expert gate g [T] of x [T][H] and the gate row wg [H], in fp64.           */
+int oracle_shared_gate(const float *x, const float *wg, int T, int H, double *g) {
+    if (T < 0 || H <= 0 || !x || !wg || !g) return -1;
+    for (int t = 0; t < T; t++) {
+        double s = 0.0;
+        for (int h = 0; h < H; h++) s += (double)x[(int64_t)t * H + h] * (double)wg[h];
+        g[t] = 1.0 / (1.0 + exp(-s));
+    }
+    return 0;
+}
+
+static int orc_forward(const uint8_t *arena, const oracle_expert *experts, int n_experts,
+                       int shared, int hidden, int ffn, const float *x, const int32_t *ids,
+                       const float *w, int T, int k, const int32_t *tokens, int n_tokens,
+                       const double *gate, float *out, double *out64);
+
 /* O1-O9 for a list of tokens.  x [T][hidden], ids/w [T][k] (from O3); experts[0..E) routed,
  * experts[shared] the always-on shared expert (shared < 0: none).  tokens[0..n_tokens) names
  * the tokens to compute (NULL: all T in order); out/out64 get one row [hidden] per listed
@@ -366,6 +404,24 @@ int oracle_expert_ffn(const uint8_t *arena, const oracle_expert *ex, int hidden,
 int oracle_forward(const uint8_t *arena, const oracle_expert *experts, int n_experts, int shared,
                    int hidden, int ffn, const float *x, const int32_t *ids, const float *w, int T,
                    int k, const int32_t *tokens, int n_tokens, float *out, double *out64) {
+    return orc_forward(arena, experts, n_experts, shared, hidden, ffn, x, ids, w, T, k, tokens,
+                       n_tokens, NULL, out, out64);
+}
+
+/* The same with the O11 gate on the shared expert: gate [T] (from oracle_shared_gate).       */
+int oracle_forward_gated(const uint8_t *arena, const oracle_expert *experts, int n_experts,
+                         int shared, int hidden, int ffn, const float *x, const int32_t *ids,
+                         const float *w, int T, int k, const int32_t *tokens, int n_tokens,
+                         const double *gate, float *out, double *out64) {
+    if (!gate) return -1;
+    return orc_forward(arena, experts, n_experts, shared, hidden, ffn, x, ids, w, T, k, tokens,
+                       n_tokens, gate, out, out64);
+}
+
+static int orc_forward(const uint8_t *arena, const oracle_expert *experts, int n_experts,
+                       int shared, int hidden, int ffn, const float *x, const int32_t *ids,
+                       const float *w, int T, int k, const int32_t *tokens, int n_tokens,
+                       const double *gate, float *out, double *out64) {
     if (hidden % 32 || n_tokens < 0) return -1;
     if (!tokens) n_tokens = T;
     int err = 0;
@@ -390,7 +446,7 @@ int oracle_forward(const uint8_t *arena, const oracle_expert *experts, int n_exp
             } else {
                 if (shared < 0) break;
                 e = shared;
-                wt = 1.0;                                                /* no gate */
+                wt = gate ? gate[t] : 1.0;                               /* O11 or no gate */
             }
             if (e < 0 || e >= n_experts || oracle_expert_ffn(arena, &experts[e], hidden, ffn,
                                                              xhat, NULL, NULL, NULL, NULL,

@@ -522,3 +522,79 @@ def test_generator_q5_1_blocks():
             W, _ = oracle.dequant_matrix(synth.Q5_1, mat.ravel(), rows, st, nb)
             lo = np.repeat(m, 32, axis=1)
             assert (W >= lo).all() and (W <= lo + 31 * np.repeat(d, 32, axis=1)).all()
+
+
+# ------------------------------------------------------------------ O10-O11 router and gate
+
+
+def test_router_one_hot_rows_pick_the_inputs():
+    rng = np.random.default_rng(21)
+    T, H, E = 5, 64, 16
+    x = rng.standard_normal((T, H)).astype(np.float32)
+    pick = rng.permutation(H)[:E]
+    Wr = np.zeros((E, H), np.float32)
+    Wr[np.arange(E), pick] = 1.0
+    l32, l64 = oracle.router(x, Wr)
+    assert np.array_equal(l32, x[:, pick])            # one nonzero product per sum: exact
+    l32q, _ = oracle.router(x, Wr * np.float32(0.25))
+    assert np.array_equal(l32q, x[:, pick] * np.float32(0.25))
+
+
+def test_router_matches_dense_fp64_matmul():
+    rng = np.random.default_rng(22)
+    T, H, E = 7, 2048, 64
+    x = rng.standard_normal((T, H)).astype(np.float32)
+    Wr = (rng.standard_normal((E, H)) * 0.02).astype(np.float32)
+    l32, l64 = oracle.router(x, Wr)
+    ref = x.astype(np.float64) @ Wr.astype(np.float64).T
+    # two fp64 summations of the same 2048 exact products differ by at most ~H ulp of sum|p|
+    bound = 4e-13 * (np.abs(x).astype(np.float64) @ np.abs(Wr).astype(np.float64).T)
+    assert (np.abs(l64 - ref) <= bound).all()
+    assert np.array_equal(l32, l64.astype(np.float32))
+
+
+def test_router_then_topk_follows_one_channel():
+    # x one-hot at channel c: every logit is Wr[e][c] exactly, so the top-k are that column's
+    # largest entries
+    rng = np.random.default_rng(23)
+    H, E, k = 32, 40, 6
+    Wr = rng.permutation(E * H).reshape(E, H).astype(np.float32) / np.float32(64.0)
+    for c in (0, 7, 31):
+        x = np.zeros((1, H), np.float32)
+        x[0, c] = 1.0
+        l32, _ = oracle.router(x, Wr)
+        ids, _, _ = oracle.topk(l32, k)
+        assert list(ids[0]) == list(np.argsort(-Wr[:, c], kind="stable")[:k])
+
+
+def test_shared_gate_closed_forms():
+    rng = np.random.default_rng(24)
+    T, H = 6, 256
+    x = rng.standard_normal((T, H)).astype(np.float32)
+    assert (oracle.shared_gate(x, np.zeros(H, np.float32)) == 0.5).all()
+    wg = (rng.standard_normal(H) * 0.05).astype(np.float32)
+    g = oracle.shared_gate(x, wg)
+    ref = scipy.special.expit(x.astype(np.float64) @ wg.astype(np.float64))
+    assert np.allclose(g, ref, rtol=1e-14, atol=0)
+    big = oracle.shared_gate(x[:1], (x[0] * np.float32(1e4)).astype(np.float32))
+    assert big[0] == 1.0                                # exp(-large) underflows: gate fully open
+
+
+def test_gated_forward_is_routed_plus_gated_shared():
+    w = _tiny(((synth.Q4_K, 0.5), (synth.Q5_1, 1.0)), 256, 160, 6, 2, 4, True, 7)
+    arena, lay = synth.host_arena(w, 0)
+    x = synth.activations(w, 0)
+    ids, wt, _ = oracle.topk(synth.router_logits(w, 0), w.k)
+    ex = oracle.experts_table(lay.fmts, lay.offs, lay.strides)
+    rng = np.random.default_rng(25)
+    g = oracle.shared_gate(x, (rng.standard_normal(w.hidden) * 0.1).astype(np.float32))
+    assert (g > 0.05).all() and (g < 0.95).all()
+    _, routed = oracle.forward(arena, ex, -1, w.hidden, w.ffn, x, ids, wt)
+    _, gated = oracle.forward(arena, ex, lay.shared, w.hidden, w.ffn, x, ids, wt, gate=g)
+    for t in range(w.tokens):
+        y_s = oracle.expert_ffn(arena, ex[lay.shared], w.hidden, w.ffn, _q8_1_values(x[t]))["y"]
+        assert np.allclose(gated[t], routed[t] + g[t] * y_s, rtol=1e-12, atol=1e-12)
+    _, ungated = oracle.forward(arena, ex, lay.shared, w.hidden, w.ffn, x, ids, wt)
+    _, ones = oracle.forward(arena, ex, lay.shared, w.hidden, w.ffn, x, ids, wt,
+                             gate=np.ones(w.tokens))
+    assert np.array_equal(ones, ungated)
