@@ -33,7 +33,8 @@ F_KEEP_H = 8
 EXPORTED = ["moe_arena_create", "moe_arena_destroy", "moe_workspace_size", "moe_quantize_act",
             "moe_route_workspace_size", "moe_route_topk", "moe_forward", "moe_ws_views",
             "moe_read_status", "moe_debug_dequant", "moe_status_string",
-            "moe_kernels_enqueued", "moe_forward_noalloc", "moe_set_timing_events"]
+            "moe_kernels_enqueued", "moe_forward_noalloc", "moe_set_timing_events",
+            "moe_router_logits", "moe_shared_gate"]
 
 
 class ExpertDesc(ctypes.Structure):
@@ -70,6 +71,8 @@ _lib.moe_read_status.argtypes = [_P, _P, _I, ctypes.POINTER(_I)]
 _lib.moe_debug_dequant.argtypes = [_P, _I, _I, _P, _P]
 _lib.moe_forward_noalloc.argtypes = [_P, _P, _P, _I, _I, _P, _P, _P]
 _lib.moe_set_timing_events.argtypes = [_P, _P, _P, _P]
+_lib.moe_router_logits.argtypes = [_P, _I, _I, _P, _I, _P, _P]
+_lib.moe_shared_gate.argtypes = [_P, _I, _I, _P, _P, _P]
 _lib.moe_kernels_enqueued.argtypes = []
 _lib.moe_kernels_enqueued.restype = ctypes.c_uint64
 
@@ -130,6 +133,19 @@ def route_workspace_size(T: int, E: int, k: int) -> int:
     n = _S()
     _check(_lib.moe_route_workspace_size(T, E, k, ctypes.byref(n)), "moe_route_workspace_size")
     return n.value
+
+
+def router_logits(d_x: int, T: int, H: int, d_router: int, E: int, d_logits: int,
+                  stream=None) -> None:
+    _check(_lib.moe_router_logits(d_x, T, H, d_router, E, d_logits, stream), "moe_router_logits")
+
+
+def router_logits_status(d_x, T, H, d_router, E, d_logits, stream=None) -> int:
+    return _lib.moe_router_logits(d_x, T, H, d_router, E, d_logits, stream)
+
+
+def shared_gate(d_x: int, T: int, H: int, d_gate_row: int, d_gate: int, stream=None) -> None:
+    _check(_lib.moe_shared_gate(d_x, T, H, d_gate_row, d_gate, stream), "moe_shared_gate")
 
 
 def route_topk(d_logits: int, T: int, E: int, k: int, d_ids: int, d_w: int, d_counts: int,

@@ -110,6 +110,21 @@ moe_status moe_workspace_size(const moe_arena *arena, int max_tokens, int k, uin
 moe_status moe_quantize_act(const float *d_x, int T, int H, int8_t *d_q, uint16_t *d_d,
                             uint16_t *d_s, uint32_t *d_status, void *stream);
 
+/* The router: d_logits fp32 [T][E] = d_x fp32 [T][H] times d_router fp32 [E][H] (row e holds
+ * expert e's weights), each logit summed in fp32 in a fixed order.  The pages keep the routers
+ * on the GPU in the per-token path ("Strata: a 125B MoE at 94 tok/s on a 12 GB Card", "Three
+ * architecture facts").  H multiple of 4; d_x and d_router 16-byte aligned, d_logits 4-byte
+ * aligned.  Returns MOE_ERR_INVALID_ARG / MOE_ERR_ALIGNMENT before enqueueing anything.      */
+moe_status moe_router_logits(const float *d_x, int T, int H, const float *d_router, int E,
+                             float *d_logits, void *stream);
+
+/* An optional gate on the shared expert: d_gate fp32 [T] = 1 / (1 + exp(-x[t] . gate_row)),
+ * from d_x fp32 [T][H] and d_gate_row fp32 [H].  The pages describe no such gate; models of
+ * the Qwen-Next family scale their shared expert by it.  Same argument rules as
+ * moe_router_logits.                                                                         */
+moe_status moe_shared_gate(const float *d_x, int T, int H, const float *d_gate_row,
+                           float *d_gate, void *stream);
+
 /* Bytes of workspace moe_route_topk needs for T tokens, E experts, k per token. */
 moe_status moe_route_workspace_size(int T, int E, int k, size_t *bytes);
 

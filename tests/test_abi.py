@@ -74,6 +74,17 @@ def test_arena_create_rejects_bad_arguments(moe):
     assert L.moe_arena_create(FAKE, 1, 256, 256, 1, -1, None, ctypes.byref(h)) == moe.ERR_INVALID_ARG
 
 
+def test_router_and_gate_reject_bad_arguments(moe):
+    L = moe.library()
+    assert L.moe_router_logits(None, 1, 64, FAKE, 8, FAKE, None) == moe.ERR_INVALID_ARG
+    assert L.moe_router_logits(FAKE, 0, 64, FAKE, 8, FAKE, None) == moe.ERR_INVALID_ARG
+    assert L.moe_router_logits(FAKE, 1, 66, FAKE, 8, FAKE, None) == moe.ERR_INVALID_ARG  # H % 4
+    assert L.moe_router_logits(FAKE + 4, 1, 64, FAKE, 8, FAKE, None) == moe.ERR_ALIGNMENT
+    assert L.moe_router_logits(FAKE, 1, 64, FAKE, 8, FAKE + 2, None) == moe.ERR_ALIGNMENT
+    assert L.moe_shared_gate(FAKE, 1, 64, None, FAKE, None) == moe.ERR_INVALID_ARG
+    assert L.moe_shared_gate(FAKE, 1, 64, FAKE + 8, FAKE, None) == moe.ERR_ALIGNMENT
+
+
 def test_entry_points_reject_null_arguments(moe):
     L = moe.library()
     n = ctypes.c_size_t()
