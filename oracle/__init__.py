@@ -238,6 +238,30 @@ def forward(arena: np.ndarray, experts: np.ndarray, shared: int, hidden: int, ff
     return out, out64
 
 
+def chain(layers, x0: np.ndarray, k: int, lookahead: bool = False):
+    """O12: a chain of MoE layers with a residual stream, as in a decoder: for each layer l,
+    logits = router(x_l, Wr_l) (O10), top-k (O3), out_l = O1-O9 (gated by O11 when the layer
+    has a gate row), and x_{l+1} = fp32(x_l + out_l).  `layers` is a sequence of dicts with
+    keys arena, experts, shared, hidden, ffn, router (Wr [E][H]) and optionally gate (wg [H]).
+
+    Returns (x_L fp32 [T][H], per-layer ids).  With lookahead=True it also returns, for every
+    layer l >= 1, the ids that layer l's router picks from x_{l-1} (before layer l-1 has
+    run): the experts a prefetch one layer ahead would fetch."""
+    x = np.ascontiguousarray(x0, dtype=np.float32)
+    all_ids, early = [], []
+    for l, L in enumerate(layers):
+        logits, _ = router(x, L["router"])
+        ids, w, _ = topk(logits, k)
+        g = shared_gate(x, L["gate"]) if L.get("gate") is not None else None
+        out, _ = forward(L["arena"], L["experts"], L["shared"], L["hidden"], L["ffn"], x, ids, w,
+                         gate=g)
+        if lookahead and l + 1 < len(layers):
+            early.append(topk(router(x, layers[l + 1]["router"])[0], k)[0])
+        x = (x + out).astype(np.float32)
+        all_ids.append(ids)
+    return (x, all_ids, early) if lookahead else (x, all_ids)
+
+
 def set_threads(n: int) -> int:
     """OpenMP threads for oracle_forward (0 keeps the default); returns the count in use."""
     return lib().oracle_set_threads(n)

@@ -598,3 +598,60 @@ def test_gated_forward_is_routed_plus_gated_shared():
     _, ones = oracle.forward(arena, ex, lay.shared, w.hidden, w.ffn, x, ids, wt,
                              gate=np.ones(w.tokens))
     assert np.array_equal(ones, ungated)
+
+
+# ------------------------------------------------------------------ O12 layer chain
+
+
+def _chain_layer(w, layer, seed, zero=False, gate=False):
+    arena, lay = synth.host_arena(w, layer)
+    if zero:                       # every block's d and dmin 0: every expert outputs 0
+        arena = arena.copy()
+        for e in range(lay.n):
+            for t in range(3):
+                rows, width = synth.tensor_shape(w, t)
+                fmt = int(lay.fmts[e])
+                nb, bb = synth.row_blocks(fmt, width), synth.BLOCK_BYTES[fmt]
+                st = int(lay.strides[e, t])
+                m = arena[lay.offs[e, t]:lay.offs[e, t] + rows * st].reshape(rows, st)
+                for b in range(nb):
+                    m[:, b * bb:b * bb + (2 if fmt == synth.Q8_0 else 4)] = 0
+    rng = np.random.default_rng(seed)
+    return {"arena": arena, "experts": oracle.experts_table(lay.fmts, lay.offs, lay.strides),
+            "shared": lay.shared, "hidden": w.hidden, "ffn": w.ffn,
+            "router": (rng.standard_normal((w.n_experts, w.hidden)) * 0.05).astype(np.float32),
+            "gate": (rng.standard_normal(w.hidden) * 0.05).astype(np.float32) if gate else None}
+
+
+def test_chain_of_one_layer_is_the_layer_plus_residual():
+    w = _tiny(None, 256, 256, 8, 2, 3, True, 8)
+    L = _chain_layer(w, 0, 31, gate=True)
+    x0 = synth.activations(w, 0)
+    xL, ids = oracle.chain([L], x0, w.k)
+    logits, _ = oracle.router(x0, L["router"])
+    rid, rw, _ = oracle.topk(logits, w.k)
+    out, _ = oracle.forward(L["arena"], L["experts"], L["shared"], w.hidden, w.ffn, x0, rid, rw,
+                            gate=oracle.shared_gate(x0, L["gate"]))
+    assert np.array_equal(ids[0], rid)
+    assert np.array_equal(xL, (x0 + out).astype(np.float32))
+
+
+def test_chain_of_silent_layers_keeps_the_residual():
+    w = _tiny(None, 256, 256, 8, 2, 3, True, 9)
+    layers = [_chain_layer(w, l, 40 + l, zero=True) for l in range(3)]
+    x0 = synth.activations(w, 0)
+    xL, ids = oracle.chain(layers, x0, w.k)
+    assert np.array_equal(xL, x0) and len(ids) == 3
+
+
+def test_chain_lookahead_with_identical_routers_predicts_from_the_previous_input():
+    # layers that share one router: the early pick for layer l is the routing of x_{l-1}, which
+    # is exactly what layer l-1 chose
+    w = _tiny(None, 256, 256, 8, 2, 3, False, 10)
+    base = _chain_layer(w, 0, 50)
+    layers = [dict(base, arena=_chain_layer(w, l, 50)["arena"]) for l in range(3)]
+    x0 = synth.activations(w, 0)
+    _, ids, early = oracle.chain(layers, x0, w.k, lookahead=True)
+    assert len(early) == 2
+    for l in range(2):
+        assert np.array_equal(early[l], ids[l])
