@@ -21,7 +21,7 @@ _HERE = Path(__file__).resolve().parent
 _SRC = _HERE / "moe_oracle.c"
 _LIB = _HERE / "liboracle.so"
 
-FMT_Q4_K, FMT_Q5_K, FMT_Q8_0, FMT_Q5_1 = 0, 1, 2, 3
+FMT_Q4_K, FMT_Q5_K, FMT_Q8_0, FMT_Q5_1, FMT_Q6_K = 0, 1, 2, 3, 4
 
 _lib = None
 

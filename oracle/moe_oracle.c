@@ -12,8 +12,9 @@
  * Q4_K, Q5_K, Q5_1 and Q8_0 experts whose dequantizers follow llama.cpp's bit for bit; the q8_1
  * activations of the "Strata v0.1.39" release notes, fixes list, #606):
  *
- *   O1  block decode (Q4_K, Q5_K, Q5_1, Q8_0) to exact fp64 and to the fp32 value
- *       RN32( RN32(d*sc)*q - RN32(dmin*m) )             (Q8_0: RN32(d*q); Q5_1: RN32(d*q + m))
+ *   O1  block decode (Q4_K, Q5_K, Q5_1, Q8_0, Q6_K) to exact fp64 and to the fp32 value
+ *       RN32( RN32(d*sc)*q - RN32(dmin*m) )             (Q8_0: RN32(d*q); Q5_1: RN32(d*q + m);
+ *       Q6_K: RN32(RN32(d*sc)*q) -- the format real Q4_K_M model files mix in)
  *   O2  Q8_1 quantization of 32-value blocks: amax, d = amax/127 (fp32 division),
  *       q = round-half-away(x/d) clamped to [-127,127], stored d16 = fp16(d),
  *       s16 = fp16(d * sum(q)); a block holding a non-finite value becomes all zero
@@ -46,16 +47,16 @@
 #include <omp.h>
 #endif
 
-enum { ORC_Q4_K = 0, ORC_Q5_K = 1, ORC_Q8_0 = 2, ORC_Q5_1 = 3 };
+enum { ORC_Q4_K = 0, ORC_Q5_K = 1, ORC_Q8_0 = 2, ORC_Q5_1 = 3, ORC_Q6_K = 4 };
 
 /* weights and bytes per block of each format */
 static int orc_block_weights(int fmt) { return fmt == ORC_Q8_0 || fmt == ORC_Q5_1 ? 32 : 256; }
 static int orc_block_bytes(int fmt) {
-    return fmt == ORC_Q4_K ? 144 : fmt == ORC_Q5_K ? 176 : fmt == ORC_Q8_0 ? 34 : 24;
+    return fmt == ORC_Q4_K ? 144 : fmt == ORC_Q5_K ? 176 : fmt == ORC_Q8_0 ? 34 : fmt == ORC_Q5_1 ? 24 : 210;
 }
 
-int oracle_block_weights(int fmt) { return fmt >= 0 && fmt <= 3 ? orc_block_weights(fmt) : -1; }
-int oracle_block_bytes(int fmt) { return fmt >= 0 && fmt <= 3 ? orc_block_bytes(fmt) : -1; }
+int oracle_block_weights(int fmt) { return fmt >= 0 && fmt <= 4 ? orc_block_weights(fmt) : -1; }
+int oracle_block_bytes(int fmt) { return fmt >= 0 && fmt <= 4 ? orc_block_bytes(fmt) : -1; }
 
 /* ---------------------------------------------------------------- IEEE binary16 <-> binary64 */
 
@@ -120,8 +121,29 @@ static void orc_kquant_scale_min(const uint8_t *S, int j, int *sc, int *m) {
  * Q5_1 (24 B): d, m (fp16, bytes 0-3), qh (32 bits, little endian, bytes 4-7), qs[16] (8-23);
  *   element n < 16: q = low nibble of qs[n], n >= 16: high nibble of qs[n-16]; bit n of qh is
  *   the fifth bit of element n; w = d*q + m (d*q has <= 16 significant bits, so the fp32 value
- *   is RN32(d*q + m) whether or not the multiply-add is fused).                               */
+ *   is RN32(d*q + m) whether or not the multiply-add is fused).
+ * Q6_K (210 B): ql[128] (bytes 0-127, low 4 bits), qh[64] (128-191, high 2 bits), sc[16]
+ *   (192-207, int8, one per 16 weights), d (fp16, 208-209).  Element n: half h = n / 128,
+ *   i = n % 128, quarter g = i / 32, l = i % 32; low bits = nibble of ql[64h + l + 32(g & 1)]
+ *   (low nibble for g < 2, high for g >= 2); high bits = bits 2g, 2g+1 of qh[32h + l];
+ *   q = low + 16 high - 32; scale sc[8h + 2g + l / 16]; w = RN32( RN32(d*sc) * q ), where
+ *   d*sc is exact (11 x 8 bits) and the product with q rounds once.                           */
 static void orc_decode_block(int fmt, const uint8_t *b, double *w64, float *w32) {
+    if (fmt == ORC_Q6_K) {
+        double d = orc_half_to_double((uint16_t)(b[208] | (b[209] << 8)));
+        for (int n = 0; n < 256; n++) {
+            int h = n / 128, i = n % 128, g = i / 32, l = i % 32;
+            int lo = b[64 * h + l + 32 * (g & 1)];
+            lo = g < 2 ? (lo & 15) : (lo >> 4);
+            int hi = (b[128 + 32 * h + l] >> (2 * g)) & 3;
+            int q = lo + 16 * hi - 32;
+            int sc = (int8_t)b[192 + 8 * h + 2 * g + l / 16];
+            float d1 = (float)(d * sc);             /* exact */
+            w64[n] = (double)d1 * q;
+            if (w32) w32[n] = d1 * (float)q;
+        }
+        return;
+    }
     if (fmt == ORC_Q5_1) {
         double d = orc_half_to_double((uint16_t)(b[0] | (b[1] << 8)));
         double m = orc_half_to_double((uint16_t)(b[2] | (b[3] << 8)));
@@ -171,7 +193,7 @@ static void orc_decode_block(int fmt, const uint8_t *b, double *w64, float *w32)
 
 /* O1 over a packed row of nblocks blocks.  Returns 0, or -1 for an unknown format. */
 int oracle_dequant_row(int fmt, const uint8_t *row, int64_t nblocks, double *w64, float *w32) {
-    if (fmt < 0 || fmt > 3) return -1;
+    if (fmt < 0 || fmt > 4) return -1;
     int bw = orc_block_weights(fmt), bb = orc_block_bytes(fmt);
     for (int64_t i = 0; i < nblocks; i++)
         orc_decode_block(fmt, row + i * bb, w64 + i * bw, w32 ? w32 + i * bw : NULL);
@@ -291,7 +313,7 @@ int oracle_group(const int32_t *ids, int T, int k, int E, int32_t *counts, int32
 
 /* ------------------------------------------------------------------------ O5-O9: the FFN */
 
-/* One expert's three matrices inside a host arena.  fmt: 0 Q4_K, 1 Q5_K, 2 Q8_0, 3 Q5_1.
+/* One expert's three matrices inside a host arena.  fmt: 0 Q4_K, 1 Q5_K, 2 Q8_0, 3 Q5_1, 4 Q6_K.
  * gate, up: ffn rows of hidden weights; down: hidden rows of ffn weights (padded to whole
  * blocks).  Offsets and row strides are in bytes.                                             */
 typedef struct {
@@ -329,7 +351,7 @@ int oracle_expert_ffn(const uint8_t *arena, const oracle_expert *ex, int hidden,
                       const double *xhat, double *g, double *u, double *h, int8_t *hq,
                       uint16_t *hd, uint16_t *hs, double *y) {
     int fmt = ex->fmt;
-    if (fmt < 0 || fmt > 3) return -1;
+    if (fmt < 0 || fmt > 4) return -1;
     int bw = orc_block_weights(fmt);
     if (hidden % bw) return -1;
     int64_t fp = orc_padded(fmt, ffn);

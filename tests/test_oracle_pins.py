@@ -126,6 +126,72 @@ def test_q5_1_offset_rounds_once_in_fp32():
     assert (w64 == -1.0).all()
 
 
+def _q6_k_block(d16, scales, ql=None, qh=None):
+    b = bytearray(210)
+    for i, v in (ql or {}).items():
+        b[i] = v
+    for i, v in (qh or {}).items():
+        b[128 + i] = v
+    b[192:208] = np.array(scales, np.int8).tobytes()
+    b[208:210] = d16.to_bytes(2, "little")
+    return np.frombuffer(bytes(b), np.uint8)
+
+
+def test_q6_k_hand_decoded_block():
+    g = _load("q6_k_e6.json")
+    blk = _q6_k_block(int(g["block"]["d"], 16), g["block"]["scales"],
+                      {int(i): int(v, 16) for i, v in g["block"]["ql_nonzero"].items()},
+                      {int(i): int(v, 16) for i, v in g["block"]["qh_nonzero"].items()})
+    w64, w32 = oracle.dequant_row(oracle.FMT_Q6_K, blk)
+    for n, v in g["expected"].items():
+        assert w64[int(n)] == v and w32[int(n)] == np.float32(v), n
+
+
+def test_q6_k_bit_positions_every_element():
+    # d = 1, every scale 1: all quants are -32 until one low nibble or one pair of high bits
+    # is set, which moves exactly one element
+    base = _q6_k_block(0x3C00, [1] * 16)
+    w0, _ = oracle.dequant_row(oracle.FMT_Q6_K, base)
+    assert (w0 == -32).all()
+    for byte in range(128):
+        for hi in (0, 1):
+            w, _ = oracle.dequant_row(oracle.FMT_Q6_K,
+                                      _q6_k_block(0x3C00, [1] * 16, {byte: 0x30 if hi else 0x03}))
+            (nz,) = np.nonzero(w != -32)
+            h, rest = divmod(byte, 64)
+            n = 128 * h + 32 * (2 * hi + rest // 32) + rest % 32
+            assert list(nz) == [n] and w[n] == -29
+    for byte in range(64):
+        for g in range(4):
+            w, _ = oracle.dequant_row(oracle.FMT_Q6_K,
+                                      _q6_k_block(0x3C00, [1] * 16, qh={byte: 1 << (2 * g + 1)}))
+            (nz,) = np.nonzero(w != -32)
+            h, l = divmod(byte, 32)
+            n = 128 * h + 32 * g + l
+            assert list(nz) == [n] and w[n] == 0       # high bits 2 -> q = 32 - 32
+
+
+def test_q6_k_scales_every_group_and_single_rounding():
+    rng = np.random.default_rng(26)
+    for _ in range(200):
+        sc = rng.integers(-128, 128, size=16)
+        raw = bytearray(rng.integers(0, 256, size=210, dtype=np.uint8).tobytes())
+        raw[192:208] = np.array(sc, np.int8).tobytes()
+        d = np.float16(rng.uniform(1e-3, 1e-2) * (1 if rng.random() < 0.8 else 1000))
+        raw[208:210] = np.array([d]).view(np.uint8).tobytes()
+        blk = np.frombuffer(bytes(raw), np.uint8)
+        w64, w32 = oracle.dequant_row(oracle.FMT_Q6_K, blk)
+        assert np.array_equal(w32, w64.astype(np.float32))
+        dq = Fraction(float(d))
+        for n in range(0, 256, 7):
+            h, i = divmod(n, 128)
+            g, l = divmod(i, 32)
+            lo = raw[64 * h + l + 32 * (g & 1)]
+            lo = lo & 15 if g < 2 else lo >> 4
+            q = lo + 16 * ((raw[128 + 32 * h + l] >> (2 * g)) & 3) - 32
+            assert Fraction(float(w64[n])) == dq * int(sc[8 * h + 2 * g + l // 16]) * q, n
+
+
 def _pack_scales(sc, m):
     """Inverse of the 6-bit scale/min unpacking: 8 (sc, m) pairs -> 12 bytes."""
     S = [0] * 12
