@@ -721,3 +721,57 @@ def test_chain_lookahead_with_identical_routers_predicts_from_the_previous_input
     assert len(early) == 2
     for l in range(2):
         assert np.array_equal(early[l], ids[l])
+
+
+def test_forward_q6_k_experts_match_dense_fp64():
+    # a tiny layer of Q6_K experts built here (the generator does not draw Q6_K): random quants,
+    # int8 scales in [-16, 16], d ~ U(1e-3, 1e-2); down rows of width 160 stored as one block
+    rng = np.random.default_rng(27)
+    H, F, E, k, T = 256, 160, 4, 2, 3
+    n = E + 1
+    shapes = ((F, H), (F, H), (H, F))
+    offs = np.zeros((n, 3), np.int64)
+    strides = np.zeros((n, 3), np.int64)
+    chunks, pos = [], 0
+    for e in range(n):
+        for t, (rows, width) in enumerate(shapes):
+            nb = -(-width // 256)
+            st = -(-nb * 210 // 16) * 16
+            m = rng.integers(0, 256, size=(rows, st), dtype=np.uint8)
+            for b in range(nb):
+                m[:, b * 210 + 192:b * 210 + 208] = rng.integers(-16, 17, size=(rows, 16)).astype(np.int8).view(np.uint8)
+                d = rng.uniform(1e-3, 1e-2, size=rows).astype(np.float16)
+                m[:, b * 210 + 208:b * 210 + 210] = d.view(np.uint8).reshape(rows, 2)
+            m[:, nb * 210:] = 0
+            pad = -pos % 256
+            chunks.append(np.zeros(pad, np.uint8))
+            pos += pad
+            offs[e, t], strides[e, t] = pos, st
+            chunks.append(m.ravel())
+            pos += m.size
+    arena = np.concatenate(chunks)
+    ex = oracle.experts_table(np.full(n, oracle.FMT_Q6_K, np.int32), offs, strides)
+    x = rng.standard_normal((T, H)).astype(np.float32)
+    logits = (np.arange(E)[None, :] * 0.25 + rng.permutation(E * T).reshape(T, E)).astype(np.float32)
+    ids, wt, _ = oracle.topk(logits, k)
+    out, out64 = oracle.forward(arena, ex, E, H, F, x, ids, wt)
+    dense = []
+    for e in range(n):
+        mats = []
+        for t, (rows, width) in enumerate(shapes):
+            nb = -(-width // 256)
+            W, _ = oracle.dequant_matrix(oracle.FMT_Q6_K, arena[offs[e, t]:], rows, int(strides[e, t]), nb)
+            mats.append(W)
+        dense.append(mats)
+    for t in range(T):
+        xh = _q8_1_values(x[t])
+        acc = np.zeros(H)
+        for e, wj in [(int(a), float(b)) for a, b in zip(ids[t], wt[t])] + [(E, 1.0)]:
+            Wg, Wu, Wd = dense[e]
+            g = Wg @ xh
+            u = Wu @ xh
+            hp = np.zeros(Wd.shape[1], np.float32)
+            hp[:F] = g * scipy.special.expit(g) * u
+            acc += wj * (Wd @ _q8_1_values(hp))
+        assert np.allclose(out64[t], acc, rtol=1e-12, atol=1e-9)
+        assert np.array_equal(out[t], out64[t].astype(np.float32))
