@@ -410,7 +410,25 @@ def oracle_sample(w, seconds, max_layers=None):
     used = min(threads, sample_tokens)
     return {"value": done_tokens / t_total, "unit": "tokens/s", "cores": used, "kind": "oracle",
             "sample": f"{layers} layer(s) x {sample_tokens} token(s) of the workload "
-                      f"({t_total:.1f} s on {used} thread(s); OpenMP over tokens)"}
+                      f"({t_total:.1f} s on {used} thread(s) of {host_cpu()}; OpenMP over tokens)"}
+
+
+def host_cpu() -> str:
+    """The host CPU's model name and the cores this process may use."""
+    name = "unknown CPU"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    name = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    try:
+        n = len(os.sched_getaffinity(0))
+    except (AttributeError, OSError):
+        n = os.cpu_count() or 1
+    return f"{name}, {n} usable cores"
 
 
 def run_reference(args):

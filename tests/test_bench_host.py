@@ -45,6 +45,7 @@ def test_oracle_sample_runs_at_least_one_layer():
     w = bench.workload("decode")
     s = bench.oracle_sample(w, 0.0, max_layers=1)
     assert s["value"] > 0 and s["sample"].startswith("1 layer(s)")
+    assert "usable cores" in s["sample"]
 
 
 def test_job_throughput_counts_every_rank():
