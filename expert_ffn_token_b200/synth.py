@@ -24,6 +24,9 @@ Weight tensors of expert e in layer l (tensor t: 0 gate, 1 up, 2 down), rows of 
         d    = fp16(fp32(1e-3 + 9e-3 * uniform(key(seed, l, e, t, 1), i)))   bytes 0-1
         dmin = fp16(fp32(1e-3 + 9e-3 * uniform(key(seed, l, e, t, 2), i)))   bytes 2-3 (K-quants)
         m    = -16 * dmin (exact in fp16)                                  bytes 2-3 (Q5_1)
+    Q6_K blocks keep d at bytes 208-209 instead (the scale bytes 192-207 are raw int8 draws);
+    their 16-weight groups past the row's logical width get scale 0.  Q6_K is drawn on the
+    host only: the device fill refuses it.
     K-quant blocks that run past the row's logical width (down rows of width 640 stored as
     768) get scale and min 0 for the sub-blocks past the width, so those weights are exactly 0.
     Pad bytes after the last block of a row are 0.
@@ -43,10 +46,10 @@ from dataclasses import dataclass, field
 
 import numpy as np
 
-Q4_K, Q5_K, Q8_0, Q5_1 = 0, 1, 2, 3
-FMT_NAMES = {Q4_K: "Q4_K", Q5_K: "Q5_K", Q8_0: "Q8_0", Q5_1: "Q5_1"}
-BLOCK_WEIGHTS = {Q4_K: 256, Q5_K: 256, Q8_0: 32, Q5_1: 32}
-BLOCK_BYTES = {Q4_K: 144, Q5_K: 176, Q8_0: 34, Q5_1: 24}
+Q4_K, Q5_K, Q8_0, Q5_1, Q6_K = 0, 1, 2, 3, 4
+FMT_NAMES = {Q4_K: "Q4_K", Q5_K: "Q5_K", Q8_0: "Q8_0", Q5_1: "Q5_1", Q6_K: "Q6_K"}
+BLOCK_WEIGHTS = {Q4_K: 256, Q5_K: 256, Q8_0: 32, Q5_1: 32, Q6_K: 256}
+BLOCK_BYTES = {Q4_K: 144, Q5_K: 176, Q8_0: 34, Q5_1: 24, Q6_K: 210}
 TENSOR_ALIGN = 256
 
 G = np.uint64(0x9E3779B97F4A7C15)
@@ -246,7 +249,16 @@ def tensor_bytes(w: Workload, layer: int, e: int, t: int, fmt: int) -> np.ndarra
     d = scale_to_half(uniform(key(w.seed, layer, e, t, 1), 0, nblk)).reshape(rows, nb)
     blocks[:, :, 0] = (d & 0xFF).astype(np.uint8)
     blocks[:, :, 1] = (d >> 8).astype(np.uint8)
-    if fmt == Q5_1:
+    if fmt == Q6_K:
+        # d lives at the end of a Q6_K block; the first two bytes are quants like the rest
+        raw_first = m[:, :nb * bb].reshape(rows, nb, bb)[:, :, 0:2].copy()
+        blocks[:, :, 0:2] = raw_first
+        blocks[:, :, 208] = (d & 0xFF).astype(np.uint8)
+        blocks[:, :, 209] = (d >> 8).astype(np.uint8)
+        valid = width - (nb - 1) * 256
+        if valid < 256:
+            blocks[:, nb - 1, 192 + valid // 16:208] = 0
+    elif fmt == Q5_1:
         dm = scale_to_half(uniform(key(w.seed, layer, e, t, 2), 0, nblk)).reshape(rows, nb)
         mm = (dm + np.uint16(4 << 10)) | np.uint16(0x8000)      # -16 * dmin: exponent + 4, sign
         blocks[:, :, 2] = (mm & 0xFF).astype(np.uint8)
@@ -404,6 +416,8 @@ def device_fill_layer(w: Workload, layer: int, d_base: int, stream=None) -> Aren
                     ("kquant", ctypes.c_int32), ("valid_last", ctypes.c_int32)]
 
     fmts = layer_formats(w, layer)
+    if (fmts == Q6_K).any():
+        raise NotImplementedError("the device fill does not draw Q6_K blocks (host_arena does)")
     lay = arena_layout(w, fmts)
     tab = (_T * (lay.n * 3))()
     for e in range(lay.n):

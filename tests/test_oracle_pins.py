@@ -469,6 +469,8 @@ def _q8_1_values(v):
     (4, ((synth.Q5_1, 1.0),), 256, 160, 5, 2, 3, True),      # Q5_1, width 160
     (5, ((synth.Q4_K, 0.25), (synth.Q5_K, 0.5), (synth.Q8_0, 0.75), (synth.Q5_1, 1.0)),
      512, 640, 12, 4, 5, True),
+    (6, ((synth.Q6_K, 1.0),), 256, 160, 5, 2, 3, True),      # Q6_K, down rows padded
+    (7, ((synth.Q4_K, 0.5), (synth.Q6_K, 1.0)), 512, 640, 8, 3, 4, True),
 ])
 def test_forward_matches_dense_fp64(case):
     idx, mix, H, F, E, k, T, shared = case
@@ -775,3 +777,23 @@ def test_forward_q6_k_experts_match_dense_fp64():
             acc += wj * (Wd @ _q8_1_values(hp))
         assert np.allclose(out64[t], acc, rtol=1e-12, atol=1e-9)
         assert np.array_equal(out[t], out64[t].astype(np.float32))
+
+
+def test_generator_q6_k_blocks_and_padding():
+    # Q6_K tensors: d from the scale draw at the end of each block; the down rows' weights past
+    # the logical width 160 (groups 10-15 of the one block) are exactly 0
+    w = _tiny(((synth.Q6_K, 1.0),), 256, 160, 3, 1, 2, False, 11)
+    arena, lay = synth.host_arena(w, 0)
+    assert (lay.fmts == synth.Q6_K).all() and lay.strides[0, 0] == 224
+    for e in range(lay.n):
+        for t in range(3):
+            rows, width = synth.tensor_shape(w, t)
+            st = int(lay.strides[e, t])
+            mat = arena[lay.offs[e, t]:lay.offs[e, t] + rows * st].reshape(rows, st)
+            assert not mat[:, 210:].any()
+            d = mat[:, 208:210].copy().view(np.float16)[:, 0].astype(np.float64)
+            assert (d >= 1e-3 * 0.999).all() and (d <= 1e-2 * 1.001).all()
+            W, _ = oracle.dequant_matrix(synth.Q6_K, mat.ravel(), rows, st, 1)
+            assert not W[:, width:].any() and W[:, :width].any()
+    with pytest.raises(NotImplementedError):
+        synth.device_fill_layer(w, 0, 0)
