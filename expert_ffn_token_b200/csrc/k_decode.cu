@@ -523,7 +523,8 @@ __device__ __forceinline__ void prologue(const DecParams &P, Ctx &C, uint8_t *sm
             }
         }
         __syncthreads();
-        if (cta0) {   // the intermediates of a1-a3 in the workspace
+        if (cta0) {   // the intermediates of a1-a3 in the workspace (from outside the stage
+                      // ring: this CTA's producer may already be filling it)
             const int U = C.s_misc[0];
 #pragma unroll 1
             for (int i = tid; i < H / 16; i += kThreads)
@@ -533,7 +534,7 @@ __device__ __forceinline__ void prologue(const DecParams &P, Ctx &C, uint8_t *sm
                 int c = 0, o = 0;
 #pragma unroll 1
                 for (int i = 0; i < k; i++) {
-                    const int x = s_ids[i];
+                    const int x = C.s_jobs[i].expert;
                     c += x == e ? 1 : 0;
                     o += x < e ? 1 : 0;
                 }
