@@ -116,3 +116,24 @@ def test_product_path_does_not_import_the_oracle():
                     text = fh.read()
                 assert "import oracle" not in text and "from oracle" not in text, f
                 assert "moe_oracle" not in text and "liboracle" not in text, f
+
+
+def _declared_arity():
+    """Parameter count of every moe_* function declared in include/moe.h."""
+    with open(os.path.join(ROOT, "include", "moe.h")) as f:
+        text = re.sub(r"/\*.*?\*/", "", f.read(), flags=re.S)
+    out = {}
+    for m in re.finditer(r"\b(moe_[a-z_]+)\s*\(([^)]*)\)\s*;", text):
+        params = m.group(2).strip()
+        out[m.group(1)] = 0 if params in ("", "void") else params.count(",") + 1
+    return out
+
+
+def test_binding_signatures_match_the_header(moe):
+    arity = _declared_arity()
+    assert set(moe.EXPORTED) <= set(arity)
+    for name in moe.EXPORTED:
+        fn = getattr(moe.library(), name)
+        if fn.argtypes is None:
+            continue
+        assert len(fn.argtypes) == arity[name], (name, len(fn.argtypes), arity[name])
