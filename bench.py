@@ -1,27 +1,33 @@
 #!/usr/bin/env python
 """Throughput of the quantized MoE layer on B200 (one JSON line on stdout, rank 0).
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode|mtp_verify|prefill|
-                    mixed_prefill] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload all|decode|mtp_verify|
+                    prefill|mixed_prefill] [--impl ours|reference]
 
-A step is one pass of the whole layer (a1-a7) over one batch of synthetic input:
-  decode       48 independent layers (hidden 2048, 256 experts, top-8, width 512, Q4_K), one
-               token each -- the default workload; one CUDA graph of 48 moe_forward calls
-  mtp_verify   48 layers (hidden 2560, 512 experts, top-10 + shared, width 640), 3 tokens each
-  prefill      one 4096-token chunk of the 512-expert layer (rotating over 4 layers)
+A step is one pass of the whole layer (a1-a7) over one batch of synthetic input of a workload:
+  decode        48 independent layers (hidden 2048, 256 experts, top-8, width 512, Q4_K), one
+                token each; one CUDA graph of 48 moe_forward calls -- the headline workload
+  mtp_verify    48 layers (hidden 2560, 512 experts, top-10 + shared, width 640), 3 tokens each
+  prefill       one 4096-token chunk of the 512-expert layer (rotating over 4 layers)
   mixed_prefill one 8192-token chunk, per-expert Q4_K / Q5_K / Q8_0, Zipf(1.3) routing
-The metric is MoE-layer tokens/s (tokens x layers / time); expert bytes read per step (the stored
-bytes of every distinct expert that received a token, plus the shared expert) give the HBM
-fraction; algorithmic int8 ops (2 * 3 * H * F per assignment) give TOPS.  The roofline object
-describes the dominant kernel: for decode the fused layer kernel against HBM bandwidth (expert
-bytes per launch / layer time); for prefill the gate/up grouped GEMM against the tensor-core
-peak (2 * assignments * 2F * H flops per launch / its own duration, timed with CUDA events that
-the library records around it in every timed step).
+The default (`all`) times every workload one after the other (each arena freed before the next)
+and reports the decode workload as the line's headline value, the others under "workloads".
+The metric is MoE-layer tokens/s (tokens x layers / time).  Per workload:
+  - expert bytes read (stored bytes of every distinct expert that received a token, plus the
+    shared expert) give the HBM fraction; algorithmic int8 ops (2 * 3 * H * F per assignment,
+    unpadded) give TOPS; the layer's binding roofline is max(bytes / HBM, ops / int8 peak);
+  - `roofline` describes the dominant kernel: decode -- the fused layer kernel against HBM
+    bandwidth (expert bytes per launch / layer time); prefill -- the gate/up grouped GEMM against
+    the fp16 tensor-core peak (2 * assignments * 2F * H flops per launch / its own duration, from
+    CUDA events the library records around it in every timed step);
+  - `e2e` goes through the C ABI eagerly (moe_forward per layer) with the inputs copied from
+    pinned host memory and the outputs copied back inside the timed region;
+  - `cpu_baseline` is the plain fp64 C oracle (oracle/) timed on the host's cores on a bounded
+    sample of the same workload, all cores and one thread.
 
---impl reference times the CPU oracle (the plain fp64 C implementation under oracle/) on the
-same workload, a bounded sample per step, on the host cores: the reference arm of this
-comparison.  With torchrun (N > 1) every rank runs its own replica of the workload (no data
-exchange: the layer needs none), timed with CUDA events and reduced as the max over ranks.
+--impl reference times that oracle alone on the headline workload (the reference arm).  With
+torchrun (N > 1) every rank runs its own replica of the workloads (no data exchange: the layer
+needs none), timed with CUDA events and reduced as the max over ranks.
 """
 from __future__ import annotations
 
@@ -41,26 +47,29 @@ sys.path.insert(0, ROOT)
 METRIC = "MoE-layer tokens/s; decode expert-weight GB/s and prefill int8 TOPS vs B200 peak"
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
+INT8_NOMINAL_TOPS = 4500.0          # B200 dense int8, datasheet figure
+ALL = ("decode", "mtp_verify", "prefill", "mixed_prefill")
+HEADLINE = "decode"
 
 
-def parse():
+def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=None)
     ap.add_argument("--warmup", type=int, default=None)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="decode",
-                    choices=["decode", "mtp_verify", "prefill", "mixed_prefill"])
-    ap.add_argument("--cpu-seconds", type=float, default=15.0,
-                    help="target CPU time of the oracle baseline sample")
+    ap.add_argument("--workload", default="all", choices=["all", *ALL])
+    ap.add_argument("--cpu-seconds", type=float, default=8.0,
+                    help="target CPU time of each oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--layers", type=int, default=None,
                     help="layers per step (default: 48 decode / 4 prefill / 2 mixed_prefill); "
                          "fewer layers make a smaller case for profilers")
-    return ap.parse_args()
+    return ap.parse_args(argv)
 
 
 def peaks():
+    """(HBM GB/s, bf16 dense TFLOP/s, source): the driver's measured figures, else fallback."""
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         with open(p) as f:
@@ -75,6 +84,7 @@ class Clocks:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
     def __init__(self, gpu):
         self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
@@ -86,38 +96,53 @@ class Clocks:
             self.p = None
 
     def stop(self):
+        """Rows sampled so far: [(sm_mhz, max_mhz, reasons set)]."""
         if self.p is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+            return None
         time.sleep(0.25)
         self.p.terminate()
         self.p.wait()
         self.f.seek(0)
         rows = [r.split(",") for r in self.f.read().strip().splitlines() if r.count(",") >= 8]
         os.unlink(self.f.name)
+        out = []
+        for r in rows:
+            try:
+                out.append((float(r[1]), float(r[2]),
+                            {self.NAMES[i] for i in range(4) if r[5 + i].strip() == "Active"}))
+            except ValueError:
+                pass
+        return out
+
+    @staticmethod
+    def summary(rows):
+        if rows is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].strip() == "Active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+        return {"sm_mhz": statistics.median(r[0] for r in rows),
+                "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": sorted(set().union(*(r[2] for r in rows))), "samples": len(rows)}
 
 
 def traffic_for(kernel: str, workload: str):
-    """dram bytes per launch from the committed ncu summary (profiles/traffic.json), or None when
+    """DRAM bytes per launch from the committed ncu summary (profiles/traffic.json), or None when
     that capture was of another workload or the kernel's sources changed since it was taken."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
-        d = json.load(f).get(kernel)
-    if not d or d.get("workload", "decode") != workload:
+        table = json.load(f)
+    d = table.get(f"{kernel}@{workload}")
+    if not d:
         return None
     h = hashlib.sha256()
-    for s in d.get("source_files", []):
-        with open(os.path.join(ROOT, s), "rb") as f:
-            h.update(f.read())
+    try:
+        for s in d.get("source_files", []):
+            with open(os.path.join(ROOT, s), "rb") as f:
+                h.update(f.read())
+    except OSError:           # a source of that capture no longer exists
+        return None
     return d["bytes_per_launch"] if d.get("source_sha256") == h.hexdigest() else None
 
 
@@ -168,35 +193,31 @@ def expert_bytes_and_ops(w, lay, logits):
     return nbytes, ops, len(used)
 
 
-def run_ours(args, rank, world):
+def run_workload(name, args, world, dev):
+    """Time one workload on this rank's GPU; returns its result dict (every rank, same keys)."""
     import numpy as np
     import torch
 
     from expert_ffn_token_b200 import moe, synth
 
-    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
-    torch.cuda.set_device(dev)
-    w = workload(args.workload, args.layers)
-    decode = args.workload in ("decode", "mtp_verify")
+    w = workload(name, args.layers)
+    decode = name in ("decode", "mtp_verify")
     K = args.steps if args.steps is not None else (200 if decode else 20)
     W = args.warmup if args.warmup is not None else (10 if decode else 3)
     stream = torch.cuda.current_stream().cuda_stream
 
     # arenas: one tensor holding every layer, drawn on the device
-    fmts0 = synth.layer_formats(w, 0)
     lays = [synth.arena_layout(w, synth.layer_formats(w, l)) for l in range(w.layers)]
     offs = [0]
     for lay in lays[:-1]:
         offs.append(offs[-1] + lay.nbytes)
     total = offs[-1] + lays[-1].nbytes
     arena = torch.empty(total, dtype=torch.uint8, device=dev)
-    for l, lay in enumerate(lays):
+    for l in range(w.layers):
         synth.device_fill_layer(w, l, arena.data_ptr() + offs[l], stream)
-    handles = []
-    for l, lay in enumerate(lays):
-        handles.append(moe.arena_create(arena.data_ptr() + offs[l], lay.nbytes, w.hidden, w.ffn,
-                                        w.n_experts, w.n_experts if w.shared else -1,
-                                        synth.layout_descs(lay)))
+    handles = [moe.arena_create(arena.data_ptr() + offs[l], lay.nbytes, w.hidden, w.ffn,
+                                w.n_experts, w.n_experts if w.shared else -1,
+                                synth.layout_descs(lay)) for l, lay in enumerate(lays)]
     T = w.tokens
     ws_bytes = moe.workspace_size(handles[0], T, w.k, 0)
     ws = torch.zeros(ws_bytes, dtype=torch.uint8, device=dev)
@@ -214,7 +235,6 @@ def run_ours(args, rank, world):
         step_bytes += b
         step_ops += o
         distinct.append(u)
-    del fmts0
 
     def one_step(events=None):
         for l in range(w.layers):
@@ -224,8 +244,8 @@ def run_ours(args, rank, world):
                         out_d[l].data_ptr(), ws.data_ptr(), ws_bytes, 0,
                         torch.cuda.current_stream().cuda_stream)
 
-    # decode: one step (48 layers x one launch) captured in a CUDA graph.  Prefill: eager steps
-    # (about ten launches per ~5 ms layer), with CUDA events around the grouped-GEMM kernels of
+    # decode: one step (the layers' single launches) captured in a CUDA graph.  Prefill: eager
+    # steps (about ten launches per layer) with CUDA events around the grouped-GEMM kernels of
     # every layer of every timed step.
     graph = None
     kernels_per_step = 0
@@ -268,8 +288,9 @@ def run_ours(args, rank, world):
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    clocks = Clocks(os.environ.get("CUDA_VISIBLE_DEVICES", str(dev.index)).split(",")[dev.index]
-                    if "CUDA_VISIBLE_DEVICES" in os.environ else dev.index)
+    gpu_id = (os.environ["CUDA_VISIBLE_DEVICES"].split(",")[dev.index]
+              if "CUDA_VISIBLE_DEVICES" in os.environ else dev.index)
+    clocks = Clocks(gpu_id)
     n0 = moe.kernels_enqueued()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
@@ -278,111 +299,143 @@ def run_ours(args, rank, world):
     e1.record()
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1)
+    gateup_ms = down_ms = None
     if not decode:
         kernels_per_step = (moe.kernels_enqueued() - n0) // K
         for h in handles:
             moe.set_timing_events(h)
         gateup_ms = statistics.mean(t[0].elapsed_time(t[1]) for row in step_events for t in row)
         down_ms = statistics.mean(t[1].elapsed_time(t[2]) for row in step_events for t in row)
+    ms = max_over_ranks(ms, world, dev)
     if world > 1:
-        ms = max_over_ranks(ms, world, dev)
         dist.barrier()
-    clk = clocks.stop()
+    clock_rows = clocks.stop()
 
-    # end to end through the C ABI: pinned host inputs in, result out, every step
+    # end to end through the C ABI, eagerly: pinned host inputs in, every layer's moe_forward,
+    # the result out, every step
     x_h = torch.from_numpy(xs).pin_memory()
     lg_h = torch.from_numpy(lgs).pin_memory()
     out_h = torch.empty(out_d.shape, dtype=torch.float32).pin_memory()
-    for _ in range(2):
+
+    def e2e_step(graphed):
         x_d.copy_(x_h, non_blocking=True)
         lg_d.copy_(lg_h, non_blocking=True)
-        run()
+        if graphed:
+            graph.replay()
+        else:
+            one_step()
         out_h.copy_(out_d, non_blocking=True)
-    torch.cuda.synchronize()
-    K2 = max(3, K // 4)
-    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    f0.record()
-    for _ in range(K2):
-        x_d.copy_(x_h, non_blocking=True)
-        lg_d.copy_(lg_h, non_blocking=True)
-        run()
-        out_h.copy_(out_d, non_blocking=True)
-    f1.record()
-    torch.cuda.synchronize()
-    ms_e2e = f0.elapsed_time(f1)
-    ms_e2e = max_over_ranks(ms_e2e, world, dev)
+
+    def time_e2e(graphed):
+        for _ in range(2):
+            e2e_step(graphed)
+        torch.cuda.synchronize()
+        k2 = max(3, K // 4)
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record()
+        for _ in range(k2):
+            e2e_step(graphed)
+        f1.record()
+        torch.cuda.synchronize()
+        return k2, max_over_ranks(f0.elapsed_time(f1), world, dev)
+
+    k2, ms_e2e = time_e2e(False)
+    graph_e2e = time_e2e(True) if graph is not None else None
     assert np.isfinite(out_h.numpy()).all()
 
     st = moe.read_status(ws.data_ptr(), stream)   # status word sits at workspace offset 0
     if st != 0:
-        raise RuntimeError(f"device status {moe.status_string(st)}")
+        raise RuntimeError(f"{name}: device status {moe.status_string(st)}")
     graph = None
     for h in handles:
         moe.arena_destroy(h)
+    del arena, ws, x_d, lg_d, out_d
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
 
     tok_per_step = T * w.layers
     ms_step = ms / K
+    layer_s = ms_step / 1e3 / w.layers
     hbm, bf16, src = peaks()
+    bytes_per_layer = step_bytes / w.layers
+    ops_per_layer = step_ops / w.layers
+    int8_meas = 2.0 * bf16           # the int8 tensor rate is twice the fp16/bf16 rate
+    t_hbm = bytes_per_layer / (hbm * 1e9)
+    t_tensor = ops_per_layer / (int8_meas * 1e12)
+    layer_roof = {"t_min_us": 1e6 * max(t_hbm, t_tensor),
+                  "binding": "hbm" if t_hbm >= t_tensor else "int8 tensor",
+                  "t_hbm_us": 1e6 * t_hbm, "t_int8_us": 1e6 * t_tensor,
+                  "frac": max(t_hbm, t_tensor) / layer_s,
+                  "int8_peak_tops": int8_meas,
+                  "int8_peak_source": f"2 x {src} bf16 dense ({bf16:.1f} TFLOP/s)"}
     if decode:
-        per_launch_s = ms_step / 1e3 / w.layers
-        bytes_per_launch = step_bytes / w.layers
-        achieved_gbs = bytes_per_launch / per_launch_s / 1e9
-        roofline = {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm, "unit": "GB/s",
-                    "frac": achieved_gbs / hbm,
-                    "traffic": traffic_for("k_decode_fused", args.workload),
+        achieved = bytes_per_layer / layer_s / 1e9
+        roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                    "frac": achieved / hbm, "traffic": traffic_for("k_decode_fused", name),
                     "kernel": "k_decode_fused (one launch per layer)",
-                    "peak_source": src, "bytes_per_launch": bytes_per_launch}
+                    "peak_source": f"{src} HBM copy", "bytes_per_launch": bytes_per_layer}
     else:
         # dominant kernel: the gate/up grouped GEMM (k_gemm_tc<0>); 2 flops per multiply-add
         assign = T * (w.k + (1 if w.shared else 0))
         flops = 2.0 * assign * 2 * w.ffn * w.hidden
         achieved = flops / (gateup_ms / 1e3) / 1e12
         roofline = {"bound": "tensor", "achieved": achieved, "peak": bf16, "unit": "TFLOP/s",
-                    "frac": achieved / bf16,
-                    "traffic": traffic_for("k_gemm_tc<0>", args.workload),
-                    "kernel": "k_gemm_tc<0> (gate/up grouped GEMM, kind::f16 with exact integer "
-                              "operands), one launch per layer",
-                    "peak_source": f"{src} bf16 dense (same rate as f16)",
+                    "frac": achieved / bf16, "traffic": traffic_for("k_gemm_tc<0>", name),
+                    "kernel": "k_gemm_tc<0> (gate/up grouped GEMM, tcgen05 kind::f16 with whole "
+                              "fp16 weights), one launch per layer",
+                    "peak_source": f"{src} bf16 dense (fp16 runs at the same rate)",
                     "flops_per_launch": flops, "ms_per_launch": gateup_ms,
-                    "frac_of_int8_peak": achieved / (2 * bf16),
-                    "down_kernel_ms_per_launch": down_ms}
-    value = job_throughput(tok_per_step, K, world, ms)
-    result = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
-        "warmup": W, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "int8", "data": "synthetic",
-        "config": {"workload": w.note, "layers": w.layers, "tokens_per_layer": T,
-                   "hidden": w.hidden, "experts": w.n_experts, "top_k": w.k,
-                   "shared_expert": w.shared, "ffn": w.ffn,
-                   "l2": f"inputs larger than L2: {step_bytes / 1e6:.0f} MB of distinct expert "
-                         f"bytes per step (L2 126 MB)",
-                   "parallelism": f"replicas x{world}" if world > 1 else "1 GPU"},
+                    "frac_of_int8_peak": achieved / int8_meas,
+                    "down_ms_per_launch": down_ms}
+    res = {
+        "workload": w.note, "value": job_throughput(tok_per_step, K, world, ms),
+        "unit": "tokens/s", "steps": K, "warmup": W, "ms_per_step": ms_step,
+        "us_per_layer": 1e6 * layer_s, "layers": w.layers, "tokens_per_layer": T,
+        "hidden": w.hidden, "experts": w.n_experts, "top_k": w.k, "shared_expert": w.shared,
+        "ffn": w.ffn,
+        "l2": f"inputs larger than L2: {step_bytes / 1e6:.0f} MB of distinct expert bytes per "
+              f"step (L2 126 MB)",
         "expert_bytes_per_step": step_bytes,
         "distinct_experts_per_layer": statistics.mean(distinct),
         "expert_gbs": step_bytes / (ms_step / 1e3) / 1e9,
         "int8_tops": step_ops / (ms_step / 1e3) / 1e12,
+        "int8_frac_of_nominal": step_ops / (ms_step / 1e3) / 1e12 / INT8_NOMINAL_TOPS,
+        "layer_roofline": layer_roof,
         "roofline": roofline,
-        "e2e": {"value": job_throughput(tok_per_step, K2, world, ms_e2e), "unit": "tokens/s",
+        "e2e": {"value": job_throughput(tok_per_step, k2, world, ms_e2e), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(xs.nbytes + lgs.nbytes),
-                "d2h_bytes_per_step": int(out_h.numel() * 4)},
+                "d2h_bytes_per_step": int(out_h.numel() * 4),
+                "mode": "eager moe_forward per layer through the C ABI"},
         "gpu_launches": int(kernels_per_step * K),
         "kernels_per_step": int(kernels_per_step),
-        "clocks": clk,
+        "clock_rows": clock_rows,
     }
-    return result
+    if graph_e2e is not None:
+        res["e2e_graph"] = {"value": job_throughput(tok_per_step, graph_e2e[0], world,
+                                                    graph_e2e[1]),
+                            "unit": "tokens/s", "mode": "the captured graph of moe_forward calls"}
+    return res
 
 
 # ------------------------------------------------------------------ oracle (CPU baseline)
 
 
-def oracle_sample(w, seconds, max_layers=None):
-    """Time the oracle on successive layers of the workload until ~`seconds` of CPU time."""
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except (AttributeError, OSError):
+        return os.cpu_count() or 1
+
+
+def oracle_sample(w, seconds, max_layers=None, threads=None):
+    """Time the oracle on successive layers of the workload until ~`seconds` of CPU time, on
+    `threads` OpenMP threads (default: every usable core)."""
     import numpy as np
 
     import oracle
     from expert_ffn_token_b200 import synth
     oracle.build()
-    threads = oracle.set_threads(0)
+    used = oracle.set_threads(threads if threads else host_cores())
     done_tokens = 0
     t_total = 0.0
     layers = 0
@@ -407,10 +460,11 @@ def oracle_sample(w, seconds, max_layers=None):
         done_tokens += sample_tokens
         layers += 1
         l += 1
-    used = min(threads, sample_tokens)
+    what = "all tokens" if sample_tokens == w.tokens else f"{sample_tokens} of {w.tokens} tokens"
     return {"value": done_tokens / t_total, "unit": "tokens/s", "cores": used, "kind": "oracle",
-            "sample": f"{layers} layer(s) x {sample_tokens} token(s) of the workload "
-                      f"({t_total:.1f} s on {used} thread(s) of {host_cpu()}; OpenMP over tokens)"}
+            "sample": f"{layers} layer(s) x {sample_tokens} token(s) of the workload ({what} "
+                      f"per layer; {t_total:.1f} s on {used} thread(s) of {host_cpu()}; OpenMP "
+                      f"over the rows of each expert matrix)"}
 
 
 def host_cpu() -> str:
@@ -424,15 +478,12 @@ def host_cpu() -> str:
                     break
     except OSError:
         pass
-    try:
-        n = len(os.sched_getaffinity(0))
-    except (AttributeError, OSError):
-        n = os.cpu_count() or 1
-    return f"{name}, {n} usable cores"
+    return f"{name}, {host_cores()} usable cores"
 
 
 def run_reference(args):
-    w = workload(args.workload, args.layers)
+    name = HEADLINE if args.workload == "all" else args.workload
+    w = workload(name, args.layers)
     K = args.steps if args.steps is not None else 5
     W = args.warmup if args.warmup is not None else 1
     per_step = max(1.0, args.cpu_seconds / max(1, K))
@@ -464,18 +515,52 @@ def main():
         if rank == 0:
             print(json.dumps(run_reference(args)), flush=True)
         return
+    import torch
     if world > 1:
         import datetime
 
-        import torch
         import torch.distributed as dist
         torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
-    res = run_ours(args, rank, world)
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    names = ALL if args.workload == "all" else (args.workload,)
+    results = {n: run_workload(n, args, world, dev) for n in names}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        res["cpu_baseline"] = oracle_sample(workload(args.workload, args.layers), args.cpu_seconds)
+        for n in names:
+            w = workload(n, args.layers)
+            results[n]["cpu_baseline"] = oracle_sample(w, args.cpu_seconds)
+            results[n]["cpu_baseline_1_thread"] = oracle_sample(w, args.cpu_seconds / 2,
+                                                                threads=1)
+    head_name = HEADLINE if HEADLINE in results else names[0]
+    all_rows = []
+    for r in results.values():
+        rows = r.pop("clock_rows")
+        r["clocks"] = Clocks.summary(rows)
+        all_rows.extend(rows or [])
+    head = results[head_name]
+    line = {
+        "metric": METRIC, "value": head["value"], "unit": "tokens/s", "n_gpus": world,
+        "steps": head["steps"], "warmup": head["warmup"], "ms_per_step": head["ms_per_step"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
+        "data": "synthetic (seeded generator; random-init Q4_K/Q5_K/Q8_0 experts)",
+        "config": {"workload": head["workload"], "layers": head["layers"],
+                   "tokens_per_layer": head["tokens_per_layer"], "hidden": head["hidden"],
+                   "experts": head["experts"], "top_k": head["top_k"],
+                   "shared_expert": head["shared_expert"], "ffn": head["ffn"],
+                   "l2": head["l2"],
+                   "parallelism": f"replicas x{world}" if world > 1 else "1 GPU"},
+        "expert_gbs": head["expert_gbs"], "int8_tops": head["int8_tops"],
+        "roofline": head["roofline"], "layer_roofline": head["layer_roofline"],
+        "e2e": head["e2e"],
+        "gpu_launches": sum(r["gpu_launches"] for r in results.values()),
+        "clocks": Clocks.summary(all_rows if all_rows else None),
+        "workloads": results,
+    }
+    if "cpu_baseline" in head:
+        line["cpu_baseline"] = head["cpu_baseline"]
     if rank == 0:
-        print(json.dumps(res), flush=True)
+        print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()

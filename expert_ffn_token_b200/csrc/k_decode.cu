@@ -42,7 +42,6 @@ constexpr int kThreads = (kCW + 1) * 32;     // + one producer warp
 constexpr int kRG = 2;                       // gate/up rows per warp per unit
 constexpr int kUnitPairs = kRG * kCW / 2;    // 16 gate + 16 up rows per unit
 constexpr int kDownRowsMax = 2 * kCW;        // down rows per unit: 1 or 2 per warp
-constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s: far beyond any legitimate wait
 
 enum { ST_END = 0, ST_GU = 1, ST_DOWN = 2 };
 
@@ -67,10 +66,17 @@ struct DecParams {
     int T, H, F, E, k, shared, hpad;
     int stage_bytes, nstages, max_jobs, slots;
     int keep_h;            // also store fp32 h
+    uint64_t wait_ns;      // limit of every bounded wait
     int o_bar, o_meta, o_xq, o_xd, o_xs, o_jobs, o_stok, o_sw, o_hq, o_hd, o_hs, o_gu, o_h,
         o_acc, o_misc;
     int smem_bytes;
 };
+
+// The descriptor table is a copy of the arena's own table into this CTA's shared memory: it
+// depends on no other CTA, so its wait keeps a long bound whatever the caller's wait limit.
+__device__ __forceinline__ uint64_t desc_wait_ns(const DecParams &P) {
+    return P.wait_ns > 50000000ull ? P.wait_ns : 50000000ull;
+}
 
 // ------------------------------------------------------------------ chunk-level math
 //
@@ -507,8 +513,12 @@ __device__ __forceinline__ void prologue(const DecParams &P, Ctx &C, uint8_t *sm
                 C.s_misc[0] = U;
             }
             __syncwarp();
-            if (!ptx::mbar_wait_bounded(C.desc_bar, 0, kWaitNs) && lane == 0)
-                set_status(status, MOE_ERR_TIMEOUT);
+            if (!ptx::mbar_wait_bounded(C.desc_bar, 0, desc_wait_ns(P))) {
+                if (lane == 0) {   // the table is not there: this CTA does no work
+                    set_status(status, MOE_ERR_TIMEOUT);
+                    C.s_misc[3] = 1;
+                }
+            } else
 #pragma unroll 1
             for (int u = lane; u < U; u += 32) {
                 JobX &J = jobs[u];
@@ -634,9 +644,14 @@ __device__ __forceinline__ void prologue(const DecParams &P, Ctx &C, uint8_t *sm
         C.s_stok[A + t] = t;
         C.s_sw[A + t] = 1.0f;
     }
-    if (tid < U && !ptx::mbar_wait_bounded(C.desc_bar, 0, kWaitNs)) set_status(status, MOE_ERR_TIMEOUT);
+    bool desc_ok = true;
+    if (tid < U && !ptx::mbar_wait_bounded(C.desc_bar, 0, desc_wait_ns(P))) {
+        desc_ok = false;   // the table is not there: this CTA does no work
+        set_status(status, MOE_ERR_TIMEOUT);
+        C.s_misc[3] = 1;
+    }
 #pragma unroll 1
-    for (int u = tid; u < U; u += kThreads) {
+    for (int u = tid; u < U && desc_ok; u += kThreads) {
         JobX &J = s_jobs[u];
         const ExpertDev &ex = s_ex[J.expert];
         J.m[0] = ex.m[0];
@@ -677,7 +692,7 @@ struct Ring {
 };
 
 __device__ __forceinline__ bool ring_acquire(const DecParams &P, const Ctx &C, Ring &R, int &st) {
-    if (!ptx::mbar_wait_bounded(&C.empty[R.s], R.ph ^ 1u, kWaitNs)) return false;
+    if (!ptx::mbar_wait_bounded(&C.empty[R.s], R.ph ^ 1u, P.wait_ns)) return false;
     st = R.s;
     if (++R.s == P.nstages) {
         R.s = 0;
@@ -750,6 +765,19 @@ __device__ __forceinline__ void producer(const DecParams &P, const Ctx &C) {
     } else {
         set_status(C.status, MOE_ERR_TIMEOUT);
     }
+    // After a wait that ran out the consumers may have left without taking every stage.  The
+    // bulk copies already issued land before the CTA leaves: wait (bounded) for the stages
+    // filled last, one ring's worth (older stages were consumed, so their phases are complete;
+    // after a normal run every one of these waits returns at once).
+    Ring B = R;
+#pragma unroll 1
+    for (int q = 0; q < P.nstages; q++) {
+        if (--B.s < 0) {
+            B.s = P.nstages - 1;
+            B.ph ^= 1u;
+        }
+        ptx::mbar_wait_bounded(&C.full[B.s], B.ph, 20000000ull);
+    }
 }
 
 // Q8_1 of a completed 32-row block of h (s_h [32][16]) for every slot of job J.
@@ -802,7 +830,7 @@ __device__ __forceinline__ bool wait_and_stage_h(const DecParams &P, const Ctx &
         int to = 0;
 #pragma unroll 1
         while (ptx::ld_acquire_u32(&C.ctr[1]) < (uint32_t)C.n_blk) {
-            if (ptx::globaltimer() - t0 > kWaitNs) {
+            if (ptx::globaltimer() - t0 > P.wait_ns) {
                 to = 1;
                 break;
             }
@@ -944,7 +972,7 @@ __device__ __forceinline__ void consumer(const DecParams &P, const Ctx &C) {
     float dacc[2][TT];   // down sums of this warp's rows (warp, warp + 16) per token
 #pragma unroll 1
     while (true) {
-        if (!ptx::mbar_wait_bounded(&C.full[s], ph, kWaitNs)) {
+        if (!ptx::mbar_wait_bounded(&C.full[s], ph, P.wait_ns)) {
             if (lane == 0) set_status(C.status, MOE_ERR_TIMEOUT);
             break;
         }
@@ -1082,6 +1110,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_fused(const DecParams P)
         ptx::mbar_init(C.desc_bar, 1);
         ptx::fence_barrier_init();
         C.s_misc[2] = 0;
+        C.s_misc[3] = 0;
         C.s_misc[5] = 0;
         // the descriptor table is the arena's (not written by the previous kernel): fetch it
         // now, in the background, before waiting for the previous grid
@@ -1102,7 +1131,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_fused(const DecParams P)
     C.i_lo = (int)((long long)P.H * cta / G);
     C.i_hi = (int)((long long)P.H * (cta + 1) / G);
 
-    if (warp == kCW) {
+    if (C.s_misc[3]) {
+        // the descriptor table did not arrive in time: no work here (this CTA's blocks are never
+        // published, so the grid-wide waits of the others give up too); the copy lands first
+        if (tid == 0) ptx::mbar_wait_bounded(C.desc_bar, 0, 50000000ull);
+    } else if (warp == kCW) {
         if ((tid & 31) == 0) producer(P, C);
     } else {
         consumer<NT, TT, FK>(P, C);
@@ -1184,6 +1217,7 @@ cudaError_t launch_decode_fused(const FfnArgs &a, int E, int shared, const float
     P.max_jobs = a.max_jobs;
     P.slots = a.T * a.k + a.T;
     P.keep_h = a.h != nullptr;
+    P.wait_ns = a.wait_ns;
     auto al = [](int v, int q) { return (v + q - 1) / q * q; };
     const int fk = a.fmt_mask == (1 << MOE_FMT_Q4_K) ? FK_Q4K
                    : a.fmt_mask == (1 << MOE_FMT_Q5_K) ? FK_Q5K : FK_ANY;

@@ -4,6 +4,8 @@
 // the workspace layout, and the choice of kernels.  All arithmetic of the layer runs in the
 // kernels of k_route.cu, k_ffn.cu and k_gemm_tc.cu.
 #include <algorithm>
+#include <cstdio>
+#include <cstdlib>
 #include <atomic>
 #include <cstring>
 #include <map>
@@ -24,6 +26,7 @@ struct moe_arena {
     void *d_wmaps;            // tensor maps of the packed matrices (tensor-core path) or null
     bool tc_ok;               // large batches may run on the tensor cores
     cudaEvent_t ev[3];        // optional timing events around the tensor-core phases
+    uint64_t wait_ns;         // limit of every bounded wait inside the kernels
     std::vector<moe_expert_desc> descs;
 };
 
@@ -89,22 +92,30 @@ WsLayout ws_layout(const moe_arena *A, int T, int k, uint32_t flags, bool allow_
     L.h = take((size_t)L.slots * F * 4);
     (void)flags;
     L.y = (flags & MOE_F_DETERMINISTIC) ? take((size_t)L.slots * H * 4) : 0;
-    // the tensor-core operands come last, so that a workspace without them keeps every other
-    // offset (moe_forward then runs the CUDA-core grouped kernels)
+    // the tensor-core operands come last
     L.tc = allow_tc && A->tc_ok && ((flags & MOE_F_FORCE_PREFILL) || T > kDecodeMaxT) &&
            !(flags & MOE_F_FORCE_DECODE);
+    L.kd = ((F + 63) / 64) * 64;
     if (L.tc) {
-        L.xg = take((size_t)L.slots * H * 2);
-        L.xgd = take((size_t)L.slots * (H / 32) * 4);
-        L.xgsh = take((size_t)L.slots * (H / 32) * 4);
-        L.xgsl = take((size_t)L.slots * (H / 32) * 4);
-        L.hg = take((size_t)L.slots * L.hpad * 2);
-        L.hgd = take((size_t)L.slots * (L.hpad / 32) * 4);
-        L.hgsh = take((size_t)L.slots * (L.hpad / 32) * 4);
-        L.hgsl = take((size_t)L.slots * (L.hpad / 32) * 4);
+        L.xh = take((size_t)T * H * 2);
+        L.xl = take((size_t)T * H * 2);
+        L.xsh = take((size_t)T * (H / 32) * 4);
+        L.xsl = take((size_t)T * (H / 32) * 4);
+        L.xscale = take((size_t)T * 4);
+        L.hh = take((size_t)L.slots * L.kd * 2);
+        L.hscale = take((size_t)L.slots * 4);
     }
     L.total = p;
     return L;
+}
+
+moe_status check_forward_args(const moe_arena *arena, const float *d_x, const float *d_logits,
+                              int T, int k, const float *d_out, uint32_t flags) {
+    if (!arena || !d_x || !d_logits || !d_out) return MOE_ERR_INVALID_ARG;
+    if (T <= 0 || k <= 0 || k > kMaxK || k > arena->E) return MOE_ERR_INVALID_ARG;
+    if ((flags & MOE_F_FORCE_DECODE) && (flags & MOE_F_FORCE_PREFILL)) return MOE_ERR_INVALID_ARG;
+    if (!aligned(d_x, 16) || !aligned(d_out, 16) || !aligned(d_logits, 4)) return MOE_ERR_ALIGNMENT;
+    return MOE_OK;
 }
 
 }  // namespace moe
@@ -183,6 +194,7 @@ moe_status moe_arena_create(const void *d_arena, size_t arena_bytes, int hidden,
     A->d_wmaps = nullptr;
     A->tc_ok = false;
     A->ev[0] = A->ev[1] = A->ev[2] = nullptr;
+    A->wait_ns = 2000000000ull;
     if (cudaMalloc(&A->d_experts, sizeof(ExpertDev) * n) != cudaSuccess ||
         cudaMemcpy(A->d_experts, dev.data(), sizeof(ExpertDev) * n, cudaMemcpyHostToDevice) !=
             cudaSuccess) {
@@ -197,7 +209,7 @@ moe_status moe_arena_create(const void *d_arena, size_t arena_bytes, int hidden,
         const bool fits = cudaGetDevice(&dev_id) == cudaSuccess &&
                           cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin,
                                                  dev_id) == cudaSuccess &&
-                          tc_smem_bytes(fmt_mask) <= (size_t)optin;
+                          tc_smem_bytes(fmt_mask) <= (size_t)optin && ffn % 64 == 0;
         if (fits && tc_build_weight_maps(A->base, host_descs, n, hidden, ffn, maps)) {
             if (cudaMalloc(&A->d_wmaps, maps.size()) != cudaSuccess ||
                 cudaMemcpy(A->d_wmaps, maps.data(), maps.size(), cudaMemcpyHostToDevice) !=
@@ -305,6 +317,7 @@ moe_status moe_ws_views(const moe_arena *arena, void *d_ws, int T, int k, uint32
     out->h = (flags & MOE_F_KEEP_H) ? reinterpret_cast<float *>(ws + L.h) : nullptr;
     out->slots = L.slots;
     out->hpad = L.hpad;
+    out->counters = reinterpret_cast<uint32_t *>(ws + L.sync);
     return MOE_OK;
 }
 
@@ -324,13 +337,12 @@ moe_status moe_read_status(uint32_t *d_status_word, void *stream, int clear,
 moe_status moe_forward(const moe_arena *arena, const float *d_x, const float *d_logits, int T,
                        int k, float *d_out, void *d_ws, size_t ws_bytes, uint32_t flags,
                        void *stream) {
-    if (!arena || !d_x || !d_logits || !d_out || !d_ws) return MOE_ERR_INVALID_ARG;
-    if (T <= 0 || k <= 0 || k > kMaxK || k > arena->E) return MOE_ERR_INVALID_ARG;
-    if ((flags & MOE_F_FORCE_DECODE) && (flags & MOE_F_FORCE_PREFILL)) return MOE_ERR_INVALID_ARG;
-    if (!aligned(d_x, 16) || !aligned(d_out, 16) || !aligned(d_logits, 4) || !aligned(d_ws, 256))
-        return MOE_ERR_ALIGNMENT;
-    WsLayout L = ws_layout(arena, T, k, flags);
-    if (ws_bytes < L.total && L.tc) L = ws_layout(arena, T, k, flags, false);
+    const moe_status chk = check_forward_args(arena, d_x, d_logits, T, k, d_out, flags);
+    if (chk != MOE_OK) return chk;
+    if (!d_ws) return MOE_ERR_INVALID_ARG;
+    if (!aligned(d_ws, 256)) return MOE_ERR_ALIGNMENT;
+    if ((flags & MOE_F_FORCE_PREFILL) && !arena->tc_ok) return MOE_ERR_UNSUPPORTED;
+    const WsLayout L = ws_layout(arena, T, k, flags);
     if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
     cudaStream_t st = (cudaStream_t)stream;
     uint8_t *ws = static_cast<uint8_t *>(d_ws);
@@ -368,6 +380,7 @@ moe_status moe_forward(const moe_arena *arena, const float *d_x, const float *d_
         a.max_stride01 = arena->max_stride01;
         a.max_stride2 = arena->max_stride2;
         a.h = (flags & MOE_F_KEEP_H) ? reinterpret_cast<float *>(ws + L.h) : nullptr;
+        a.wait_ns = arena->wait_ns;
         bool taken = false;
         cudaError_t e = launch_decode_fused(a, E, shared, d_x, d_logits, ws, L, L.sync, L.blkcnt,
                                             true, st, &taken);
@@ -377,18 +390,31 @@ moe_status moe_forward(const moe_arena *arena, const float *d_x, const float *d_
     // a1-a3
     const bool small_route = T <= kDecodeMaxT && T * k <= kDecodeMaxT * kMaxK &&
                              ((size_t)T * E + E) * 4 <= 96 * 1024;
+    const bool tc = L.tc && !(decode && T <= kDecodeMaxT);
     cudaError_t err;
-    if (small_route) {
+    if (small_route && !tc) {
         err = launch_route_small(d_x, d_logits, T, H, E, k, shared, L, ws, st);
     } else {
-        err = launch_quantize(d_x, (int64_t)T * H / 32, xq, xd, xs, xsum, status, st);
+        if (tc)
+            err = launch_quant_rows(d_x, T, H, xq, xd, xs, xsum,
+                                    reinterpret_cast<__half *>(ws + L.xh),
+                                    reinterpret_cast<__half *>(ws + L.xl),
+                                    reinterpret_cast<float *>(ws + L.xsh),
+                                    reinterpret_cast<float *>(ws + L.xsl),
+                                    reinterpret_cast<float *>(ws + L.xscale), status, st);
+        else
+            err = launch_quantize(d_x, (int64_t)T * H / 32, xq, xd, xs, xsum, status, st);
         if (err == cudaSuccess) err = launch_topk(d_logits, T, E, k, ids, w, status, st);
         if (err == cudaSuccess)
             err = launch_group(ids, T, k, E, shared, counts, offsets, perm, inv_perm,
                                reinterpret_cast<int32_t *>(ws + L.chunk_counts),
                                reinterpret_cast<int32_t *>(ws + L.chunk_base), jobs, njobs, st);
     }
-    if (err != cudaSuccess) return MOE_ERR_CUDA;
+    if (err != cudaSuccess) {
+        if (std::getenv("MOE_DEBUG"))
+            std::fprintf(stderr, "moe: routing failed: %s\n", cudaGetErrorString(err));
+        return MOE_ERR_CUDA;
+    }
 
     FfnArgs a{};
     a.experts = arena->d_experts;
@@ -417,28 +443,26 @@ moe_status moe_forward(const moe_arena *arena, const float *d_x, const float *d_
     a.fmt_mask = arena->fmt_mask;
     a.max_stride01 = arena->max_stride01;
     a.max_stride2 = arena->max_stride2;
+    a.wait_ns = arena->wait_ns;
 
-    if (L.tc && !(decode && T <= kDecodeMaxT)) {
+    if (tc) {
         // a4-a7 on the tensor cores
         TcPhaseArgs p{};
         p.ffn = a;
         p.wmaps = arena->d_wmaps;
         p.slots = L.slots;
         p.keep_h = (flags & MOE_F_KEEP_H) ? 1 : 0;
-        p.xg = reinterpret_cast<__half *>(ws + L.xg);
-        p.xgd = reinterpret_cast<float *>(ws + L.xgd);
-        p.xgsh = reinterpret_cast<float *>(ws + L.xgsh);
-        p.xgsl = reinterpret_cast<float *>(ws + L.xgsl);
-        p.hg = reinterpret_cast<__half *>(ws + L.hg);
-        p.hgd = reinterpret_cast<float *>(ws + L.hgd);
-        p.hgsh = reinterpret_cast<float *>(ws + L.hgsh);
-        p.hgsl = reinterpret_cast<float *>(ws + L.hgsl);
+        p.Kd = L.kd;
+        p.xh = reinterpret_cast<const __half *>(ws + L.xh);
+        p.xl = reinterpret_cast<const __half *>(ws + L.xl);
+        p.xsh = reinterpret_cast<const float *>(ws + L.xsh);
+        p.xsl = reinterpret_cast<const float *>(ws + L.xsl);
+        p.xscale = reinterpret_cast<const float *>(ws + L.xscale);
+        p.hh = reinterpret_cast<const __half *>(ws + L.hh);
+        p.hscale = reinterpret_cast<const float *>(ws + L.hscale);
+        p.wait_ns = arena->wait_ns;
         const int used = T * k + (shared ? T : 0);
-        err = launch_act_gather(xq, xd, xsum, perm, T, k, H, used, p.xg, p.xgd, p.xgsh, p.xgsl,
-                                st);
-        if (err == cudaSuccess)
-            err = launch_hg_tail_zero(p.hg, p.hgd, p.hgsh, p.hgsl, L.slots, arena->F, L.hpad, st);
-        if (err == cudaSuccess && p.keep_h) err = launch_hpad_zero(a, st);
+        if (p.keep_h) err = launch_hpad_zero(a, st);
         if (err == cudaSuccess && !(flags & MOE_F_DETERMINISTIC))
             err = cudaMemsetAsync(d_out, 0, (size_t)T * H * sizeof(float), st);
         if (err == cudaSuccess && arena->ev[0]) err = cudaEventRecord(arena->ev[0], st);
@@ -447,6 +471,10 @@ moe_status moe_forward(const moe_arena *arena, const float *d_x, const float *d_
             err = launch_gemm_tc(p, st);
         }
         if (err == cudaSuccess && arena->ev[1]) err = cudaEventRecord(arena->ev[1], st);
+        if (err == cudaSuccess)
+            err = launch_h_rows(a.hq, a.hd, used, arena->F, L.hpad, L.kd,
+                                reinterpret_cast<__half *>(ws + L.hh),
+                                reinterpret_cast<float *>(ws + L.hscale), st);
         if (err == cudaSuccess) {
             p.phase = 1;
             err = launch_gemm_tc(p, st);
@@ -454,6 +482,8 @@ moe_status moe_forward(const moe_arena *arena, const float *d_x, const float *d_
         if (err == cudaSuccess && arena->ev[2]) err = cudaEventRecord(arena->ev[2], st);
         if (err == cudaSuccess && (flags & MOE_F_DETERMINISTIC))
             err = launch_combine(a, shared != 0, st);
+        if (err != cudaSuccess && std::getenv("MOE_DEBUG"))
+            std::fprintf(stderr, "moe: tensor-core path failed: %s\n", cudaGetErrorString(err));
         return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
     }
     // a4 + a5
@@ -479,6 +509,12 @@ moe_status moe_set_timing_events(moe_arena *arena, void *ev_begin, void *ev_mid,
     arena->ev[0] = static_cast<cudaEvent_t>(ev_begin);
     arena->ev[1] = static_cast<cudaEvent_t>(ev_mid);
     arena->ev[2] = static_cast<cudaEvent_t>(ev_end);
+    return MOE_OK;
+}
+
+moe_status moe_set_wait_limit(moe_arena *arena, uint64_t ns) {
+    if (!arena || ns == 0) return MOE_ERR_INVALID_ARG;
+    arena->wait_ns = ns;
     return MOE_OK;
 }
 

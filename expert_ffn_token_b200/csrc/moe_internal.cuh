@@ -74,14 +74,20 @@ struct moe_arena_impl;
 struct WsLayout {
     size_t status, sync, blkcnt, njobs, jobs, xq, xd, xs, xsum, ids, w, counts, offsets, perm,
         inv_perm, chunk_counts, chunk_base, hq, hd, hs, hsum, h, y, total;
-    // tensor-core path: slot-ordered fp16 operands and fp32 scales (absent when tc == 0)
-    size_t xg, xgd, xgsh, xgsl, hg, hgd, hgsh, hgsl;
-    int slots, hpad, max_jobs, n_chunks, tc;
+    // tensor-core path (absent when tc == 0): fp16 activation rows with their power-of-two
+    // scales, per token (gate/up) and per slot (down)
+    size_t xh, xl, xsh, xsl, xscale, hh, hscale;
+    int slots, hpad, max_jobs, n_chunks, tc, kd;
 };
 
 // Workspace layout of one moe_forward call (moe_api.cu).  Without allow_tc the tensor-core
 // operands are left out.
 WsLayout ws_layout(const moe_arena *A, int T, int k, uint32_t flags, bool allow_tc = true);
+
+// The host checks moe_forward makes on its arguments other than the workspace (null pointers,
+// sizes, flag combinations, alignment), before anything is enqueued.
+moe_status check_forward_args(const moe_arena *arena, const float *d_x, const float *d_logits,
+                              int T, int k, const float *d_out, uint32_t flags);
 
 // ------------------------------------------------------------------ device helpers
 
@@ -159,6 +165,7 @@ struct FfnArgs {
     uint32_t *status;
     int T, k, H, F, hpad, max_jobs, fmt_mask;
     int max_stride01, max_stride2;   // largest gate/up and down row strides in the arena
+    uint64_t wait_ns;                // limit of every bounded wait in the kernels
 };
 
 cudaError_t launch_gateup_gemv(const FfnArgs &a, cudaStream_t st);
@@ -178,28 +185,39 @@ cudaError_t launch_hpad_zero(const FfnArgs &a, cudaStream_t st);
 
 // ---- tensor-core path for large batches (k_gemm_tc.cu)
 
-// One projection phase: 0 = gate/up over the gathered activations, 1 = down over Q8_1(h).
+// One projection phase: 0 = gate/up over the token rows x^, 1 = down over the slot rows h^.
 struct TcPhaseArgs {
     FfnArgs ffn;
     const void *wmaps;          // device array of the experts' weight tensor maps
     int phase, slots, keep_h;
-    __half *xg;
-    float *xgd, *xgsh, *xgsl;
-    __half *hg;
-    float *hgd, *hgsh, *hgsl;
+    int Kd;                     // down contraction length: ffn rounded up to 64
+    const __half *xh, *xl;      // [T][H] fp16 planes, x^ * 2^-e = hi + lo exactly
+    const float *xsh, *xsl;     // [T][H/32] block sums xd * sum(q) * 2^-e, tf32 hi + lo
+    const float *xscale;        // [T] 2^e
+    const __half *hh;           // [slots][Kd] fp16 rows of Q8_1(h) * 2^-e
+    const float *hscale;        // [slots] 2^e
+    uint64_t wait_ns;           // limit of every wait inside the kernels
 };
 
 // Host encoding of every expert's weight tensor maps into `out` (bytes to copy to the device);
 // false when the shape or a map is not supported.
 bool tc_build_weight_maps(const uint8_t *d_base, const moe_expert_desc *descs, int n, int H,
                           int F, std::vector<uint8_t> &out);
+// Dynamic shared memory the tensor-core kernels need for the formats present ((size_t)-1: no
+// plan fits); the gate/up kernel's alone.
 size_t tc_smem_bytes(int fmt_mask);
+size_t tc_gateup_smem_bytes(int fmt_mask);
+// One tensor-core phase (phase 0: k_gateup_tc, phase 1: k_down_tc).
 cudaError_t launch_gemm_tc(const TcPhaseArgs &p, cudaStream_t st);
-cudaError_t launch_act_gather(const int8_t *xq, const uint16_t *xd, const float *xsum,
-                              const int32_t *perm, int T, int k, int H, int slots, __half *xg,
-                              float *xgd, float *xgsh, float *xgsl, cudaStream_t st);
-cudaError_t launch_hg_tail_zero(__half *hg, float *hgd, float *hgsh, float *hgsl, int slots,
-                                int F, int hpad, cudaStream_t st);
+cudaError_t launch_gateup_tc(const TcPhaseArgs &p, int grid, cudaStream_t st);
+// a1 per token for the tensor-core path: the Q8_1 blocks (as moe_quantize_act) plus the gate/up
+// operand planes, the block sums and 2^e.
+cudaError_t launch_quant_rows(const float *x, int T, int H, int8_t *xq, uint16_t *xd,
+                              uint16_t *xs, float *xsum, __half *xh, __half *xl, float *xsh,
+                              float *xsl, float *xscale, uint32_t *status, cudaStream_t st);
+// The down operand of every used slot from its Q8_1(h) blocks.
+cudaError_t launch_h_rows(const int8_t *hq, const uint16_t *hd, int slots, int F, int hpad, int Kd,
+                          __half *hh, float *hscale, cudaStream_t st);
 
 cudaError_t launch_dequant(const uint8_t *m, int fmt, int rows, int nblocks, int stride,
                            float *out, cudaStream_t st);

@@ -42,18 +42,20 @@ moe_status scratch_for_current_device(uint8_t **out) {
 extern "C" moe_status moe_forward_noalloc(const moe_arena *arena, const float *d_x,
                                           const float *d_logits, int T, int k, float *d_out,
                                           uint32_t *d_status, void *stream) {
-    if (!arena || !d_x || !d_logits || !d_out) return MOE_ERR_INVALID_ARG;
-    if (T <= 0 || T > moe::kDecodeMaxT || k <= 0 || k > moe::kMaxK) return MOE_ERR_INVALID_ARG;
+    // every check moe_forward would make, before anything is enqueued
+    moe_status st = moe::check_forward_args(arena, d_x, d_logits, T, k, d_out, 0);
+    if (st != MOE_OK) return st;
+    if (T > moe::kDecodeMaxT) return MOE_ERR_INVALID_ARG;
+    if (d_status && (reinterpret_cast<uintptr_t>(d_status) & 3)) return MOE_ERR_ALIGNMENT;
     const moe::WsLayout L = moe::ws_layout(arena, T, k, 0);
     if (L.total > kNoallocScratchBytes) return MOE_ERR_UNSUPPORTED;
     uint8_t *ws = nullptr;
-    moe_status st = scratch_for_current_device(&ws);
+    st = scratch_for_current_device(&ws);
     if (st != MOE_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    // the status word and the kernel's counters must start at zero; the previous call's
-    // contents are otherwise left as they are
-    if (cudaMemsetAsync(ws + L.status, 0, sizeof(uint32_t), s) != cudaSuccess ||
-        cudaMemsetAsync(ws + L.sync, 0, 4 * sizeof(uint32_t), s) != cudaSuccess)
+    // the status word and the kernel's counters (the first bytes of the layout) must start at
+    // zero; the previous call's contents are otherwise left as they are
+    if (cudaMemsetAsync(ws, 0, L.sync + 4 * sizeof(uint32_t), s) != cudaSuccess)
         return MOE_ERR_CUDA;
     st = moe_forward(arena, d_x, d_logits, T, k, d_out, ws, kNoallocScratchBytes, 0, stream);
     if (st != MOE_OK) return st;

@@ -34,7 +34,7 @@ EXPORTED = ["moe_arena_create", "moe_arena_destroy", "moe_workspace_size", "moe_
             "moe_route_workspace_size", "moe_route_topk", "moe_forward", "moe_ws_views",
             "moe_read_status", "moe_debug_dequant", "moe_status_string",
             "moe_kernels_enqueued", "moe_forward_noalloc", "moe_set_timing_events",
-            "moe_router_logits", "moe_shared_gate"]
+            "moe_router_logits", "moe_shared_gate", "moe_set_wait_limit"]
 
 
 class ExpertDesc(ctypes.Structure):
@@ -48,7 +48,8 @@ class WsView(ctypes.Structure):
                 ("counts", ctypes.c_void_p), ("offsets", ctypes.c_void_p),
                 ("perm", ctypes.c_void_p), ("inv_perm", ctypes.c_void_p),
                 ("hq", ctypes.c_void_p), ("hd", ctypes.c_void_p), ("hs", ctypes.c_void_p),
-                ("h", ctypes.c_void_p), ("slots", ctypes.c_int32), ("hpad", ctypes.c_int32)]
+                ("h", ctypes.c_void_p), ("slots", ctypes.c_int32), ("hpad", ctypes.c_int32),
+                ("counters", ctypes.c_void_p)]
 
 
 _P = ctypes.c_void_p
@@ -73,6 +74,7 @@ _lib.moe_forward_noalloc.argtypes = [_P, _P, _P, _I, _I, _P, _P, _P]
 _lib.moe_set_timing_events.argtypes = [_P, _P, _P, _P]
 _lib.moe_router_logits.argtypes = [_P, _I, _I, _P, _I, _P, _P]
 _lib.moe_shared_gate.argtypes = [_P, _I, _I, _P, _P, _P]
+_lib.moe_set_wait_limit.argtypes = [_P, ctypes.c_uint64]
 _lib.moe_kernels_enqueued.argtypes = []
 _lib.moe_kernels_enqueued.restype = ctypes.c_uint64
 
@@ -168,6 +170,11 @@ def forward_noalloc(arena: int, d_x: int, d_logits: int, T: int, k: int, d_out: 
            "moe_forward_noalloc")
 
 
+def forward_noalloc_status(arena, d_x, d_logits, T, k, d_out, d_status=None, stream=None) -> int:
+    """moe_forward_noalloc returning its status code instead of raising."""
+    return _lib.moe_forward_noalloc(arena, d_x, d_logits, T, k, d_out, d_status, stream)
+
+
 def forward_status(arena, d_x, d_logits, T, k, d_out, d_ws, ws_bytes, flags=0, stream=None) -> int:
     """moe_forward returning its status code instead of raising (for error-path tests)."""
     return _lib.moe_forward(arena, d_x, d_logits, T, k, d_out, d_ws, ws_bytes, flags, stream)
@@ -190,6 +197,11 @@ def set_timing_events(arena: int, ev_begin=None, ev_mid=None, ev_end=None) -> No
     """moe_set_timing_events: cudaEvent_t handles (ints) recorded around the tensor-core phases
     of later forwards on this arena, or None to stop."""
     _check(_lib.moe_set_timing_events(arena, ev_begin, ev_mid, ev_end), "moe_set_timing_events")
+
+
+def set_wait_limit(arena: int, ns: int) -> None:
+    """moe_set_wait_limit: limit of every bounded device wait of later calls on this arena."""
+    _check(_lib.moe_set_wait_limit(arena, ns), "moe_set_wait_limit")
 
 
 def kernels_enqueued() -> int:

@@ -95,7 +95,10 @@ void moe_arena_destroy(moe_arena *arena);
 /* Forward flags. */
 #define MOE_F_DETERMINISTIC 1u   /* prefill: combine by gathering per-token sums (no atomics) */
 #define MOE_F_FORCE_DECODE 2u    /* use the grouped dequant-GEMV path whatever T is          */
-#define MOE_F_FORCE_PREFILL 4u   /* use the grouped tensor-core GEMM path whatever T is      */
+#define MOE_F_FORCE_PREFILL 4u   /* use the grouped tensor-core GEMM path whatever T is; the
+                                    workspace must be sized with this flag (else
+                                    MOE_ERR_WORKSPACE); MOE_ERR_UNSUPPORTED when the arena's
+                                    shape has no tensor-core plan (hidden % 256 or ffn % 64)   */
 #define MOE_F_KEEP_H 8u          /* also store fp32 h (SwiGLU output) in the workspace       */
 
 /* Bytes of device workspace moe_forward needs for up to max_tokens tokens, k routed experts
@@ -145,7 +148,13 @@ moe_status moe_route_topk(const float *d_logits, int T, int E, int k, int32_t *d
  * Q8_1 of h, optional fp32 h) are left in the workspace; moe_ws_views locates them.  They
  * equal what moe_quantize_act / moe_route_topk produce for the same inputs.
  * The grouped dequant-GEMV path (decode) is taken for T <= 16 unless a FORCE flag says
- * otherwise.  The workspace's status word collects device-side errors (moe_read_status).   */
+ * otherwise; larger batches take the tensor-core path when the arena allows it (hidden a
+ * multiple of 256, ffn a multiple of 64, stored weights and Q8_1 values of magnitude below
+ * 65504, which fp16 operands hold) and CUDA-core grouped kernels otherwise (or with
+ * MOE_F_FORCE_DECODE).  The decode kernel is one persistent CTA per SM whose CTAs wait for
+ * one another (bounded): it needs every SM free for the duration of the call; if other work
+ * keeps SMs busy the wait gives up after the arena's wait limit with MOE_ERR_TIMEOUT in the
+ * status word.  The workspace's status word collects device-side errors (moe_read_status).  */
 moe_status moe_forward(const moe_arena *arena, const float *d_x, const float *d_logits, int T,
                        int k, float *d_out, void *d_ws, size_t ws_bytes, uint32_t flags,
                        void *stream);
@@ -166,6 +175,8 @@ typedef struct {
     uint16_t *hd, *hs;         /* [slots][hpad/32] fp16 bits                           */
     float *h;                  /* [slots][ffn] fp32 (MOE_F_KEEP_H only, else NULL)     */
     int32_t slots, hpad;
+    uint32_t *counters;        /* 4 words: the decode kernel's grid-wide counters (zero
+                                  between calls; diagnostics and failure tests only)     */
 } moe_ws_view;
 
 moe_status moe_ws_views(const moe_arena *arena, void *d_ws, int T, int k, uint32_t flags,
@@ -206,6 +217,13 @@ moe_status moe_forward_noalloc(const moe_arena *arena, const float *d_x, const f
  * arena keeps the handles (not owned); calls that use them must not overlap.  The pages have
  * no counterpart; it serves the measurement of the grouped GEMM alone.                       */
 moe_status moe_set_timing_events(moe_arena *arena, void *ev_begin, void *ev_mid, void *ev_end);
+
+/* Limit, in nanoseconds, of every bounded wait inside the kernels of later calls on this arena
+ * (default 2 s).  A wait that runs out ends its kernel with MOE_ERR_TIMEOUT in the status word
+ * after the copies it had in flight have landed; the next call starts clean.  The pages'
+ * counterpart is the engine's stall watchdog ("Strata - the details", "Troubleshooting").
+ * ns > 0; MOE_ERR_INVALID_ARG otherwise.                                                      */
+moe_status moe_set_wait_limit(moe_arena *arena, uint64_t ns);
 
 /* Number of kernels this library has enqueued (or recorded into a CUDA graph under stream
  * capture) in this process since it was loaded.  Counting a captured forward gives the

@@ -56,6 +56,8 @@ def lib():
                                            ctypes.c_int, P, P, P, ctypes.c_int, ctypes.c_int, P,
                                            ctypes.c_int, P, P, P]
         L.oracle_router.argtypes = [P, P, ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P]
+        L.oracle_down_combine.argtypes = [P, P, ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P,
+                                          ctypes.c_int, P, P, P, ctypes.c_int, ctypes.c_int, P]
         L.oracle_shared_gate.argtypes = [P, P, ctypes.c_int, ctypes.c_int, P]
         L.oracle_set_threads.argtypes = [ctypes.c_int]
         L.oracle_half_to_double.argtypes = [ctypes.c_uint16]
@@ -176,6 +178,26 @@ def expert_ffn(arena: np.ndarray, expert: np.ndarray, hidden: int, ffn: int, xha
                                  _p(out["hs"]), _p(out["y"]))
     if rc != 0:
         raise ValueError("bad expert")
+    return out
+
+
+def down_combine(arena: np.ndarray, experts: np.ndarray, hidden: int, ffn: int, hq: np.ndarray,
+                 hd: np.ndarray, slot_tok, slot_exp, slot_w, T: int) -> np.ndarray:
+    """O8-O9 from given Q8_1(h) rows: out fp64 [T][hidden] = sum over slots s of
+    slot_w[s] * W_down(slot_exp[s]) * dequant(hq[s], hd[s]), added to token slot_tok[s]."""
+    arena = np.ascontiguousarray(arena, dtype=np.uint8)
+    experts = np.ascontiguousarray(experts, dtype=EXPERT_DTYPE)
+    hq = np.ascontiguousarray(hq, dtype=np.int8)
+    hd = np.ascontiguousarray(hd, dtype=np.uint16)
+    n, hpad = hq.shape
+    assert hd.shape == (n, hpad // 32)
+    st = np.ascontiguousarray(slot_tok, dtype=np.int32)
+    se = np.ascontiguousarray(slot_exp, dtype=np.int32)
+    sw = np.ascontiguousarray(slot_w, dtype=np.float64)
+    out = np.empty((T, hidden), np.float64)
+    if lib().oracle_down_combine(_p(arena), _p(experts), len(experts), hidden, ffn, _p(hq), _p(hd),
+                                 hpad, _p(st), _p(se), _p(sw), n, T, _p(out)) != 0:
+        raise ValueError("oracle_down_combine: bad arguments")
     return out
 
 

@@ -32,8 +32,9 @@
  *   O11 optional shared-expert gate: g[t] = 1 / (1 + exp(-sum_h x[t][h] * wg[h])) in fp64;
  *       with it, O9's shared term is g[t] * y[t][shared]
  *
- * Nothing here is blocked, fused or reordered beyond these definitions.  Per-token work may run
- * on several OpenMP threads; every token's arithmetic is the same whatever the thread count.
+ * Nothing here is blocked, fused or reordered beyond these definitions.  The rows of one expert
+ * matrix may be computed on several OpenMP threads; every sum runs in the same order whatever
+ * the thread count.
  *
  * Pinned by tests/test_oracle_pins.py (hand-computed blocks, a 64x64 scale pack/unpack round
  * trip, exact-rational rounding, Q8_1 closed forms, brute-force top-k, grouping invariants and
@@ -356,7 +357,6 @@ int oracle_expert_ffn(const uint8_t *arena, const oracle_expert *ex, int hidden,
     if (hidden % bw) return -1;
     int64_t fp = orc_padded(fmt, ffn);
     int64_t nb_in = hidden / bw, nb_down = fp / bw;
-    double *scratch = (double *)malloc(sizeof(double) * (size_t)(hidden > fp ? hidden : fp));
     double *hh = (double *)calloc((size_t)ffn, sizeof(double));
     float *hf = (float *)calloc((size_t)fp, sizeof(float));
     int8_t *q = (int8_t *)malloc((size_t)fp);
@@ -364,14 +364,22 @@ int oracle_expert_ffn(const uint8_t *arena, const oracle_expert *ex, int hidden,
     uint16_t *ss = (uint16_t *)malloc(sizeof(uint16_t) * (size_t)(fp / 32));
     double *hhat = (double *)malloc(sizeof(double) * (size_t)fp);
 
-    for (int r = 0; r < ffn; r++) {
-        double gr = orc_row_dot(fmt, arena + ex->off[0] + r * ex->stride[0], nb_in, xhat, scratch);
-        double ur = orc_row_dot(fmt, arena + ex->off[1] + r * ex->stride[1], nb_in, xhat, scratch);
-        double hr = gr / (1.0 + exp(-gr)) * ur;                     /* O6 */
-        if (g) g[r] = gr;
-        if (u) u[r] = ur;
-        hh[r] = hr;
-        hf[r] = (float)hr;
+    /* rows are independent: the row loops may run on several threads (each row's sum is the
+     * same sequential loop whatever the thread count) */
+#pragma omp parallel
+    {
+        double *sc = (double *)malloc(sizeof(double) * (size_t)(hidden > fp ? hidden : fp));
+#pragma omp for schedule(static)
+        for (int r = 0; r < ffn; r++) {
+            double gr = orc_row_dot(fmt, arena + ex->off[0] + r * ex->stride[0], nb_in, xhat, sc);
+            double ur = orc_row_dot(fmt, arena + ex->off[1] + r * ex->stride[1], nb_in, xhat, sc);
+            double hr = gr / (1.0 + exp(-gr)) * ur;                 /* O6 */
+            if (g) g[r] = gr;
+            if (u) u[r] = ur;
+            hh[r] = hr;
+            hf[r] = (float)hr;
+        }
+        free(sc);
     }
     if (h) memcpy(h, hh, sizeof(double) * (size_t)ffn);
     oracle_quantize_q8_1(hf, fp / 32, q, dd, ss);                   /* O7 (tail stays zero) */
@@ -379,11 +387,57 @@ int oracle_expert_ffn(const uint8_t *arena, const oracle_expert *ex, int hidden,
     if (hq) memcpy(hq, q, (size_t)fp);
     if (hd) memcpy(hd, dd, sizeof(uint16_t) * (size_t)(fp / 32));
     if (hs) memcpy(hs, ss, sizeof(uint16_t) * (size_t)(fp / 32));
-    for (int i = 0; i < hidden; i++)                                 /* O8 */
-        y[i] = orc_row_dot(fmt, arena + ex->off[2] + i * ex->stride[2], nb_down, hhat, scratch);
+#pragma omp parallel
+    {
+        double *sc = (double *)malloc(sizeof(double) * (size_t)(hidden > fp ? hidden : fp));
+#pragma omp for schedule(static)
+        for (int i = 0; i < hidden; i++)                             /* O8 */
+            y[i] = orc_row_dot(fmt, arena + ex->off[2] + i * ex->stride[2], nb_down, hhat, sc);
+        free(sc);
+    }
 
-    free(scratch); free(hh); free(hf); free(q); free(dd); free(ss); free(hhat);
+    free(hh); free(hf); free(q); free(dd); free(ss); free(hhat);
     return 0;
+}
+
+/* O8-O9 from Q8_1(h) rows given from outside (the reading that checks a layer whose h was
+ * computed elsewhere in two parts: h itself, and everything after it).  Slot s belongs to token
+ * slot_tok[s] and expert slot_exp[s] with routing weight slot_w[s]; its h^ is the dequantized
+ * Q8_1 row hq [s][0..fp), hd [s][0..fp/32) (fp = the expert's stored down width, <= hpad).
+ * y = W_down h^ (exact weights, fp64) and out64[tok] += w * y, slot after slot in the order
+ * given.  out64 [T][hidden] is overwritten.  Returns 0, or -1 for bad arguments.             */
+int oracle_down_combine(const uint8_t *arena, const oracle_expert *experts, int n_experts,
+                        int hidden, int ffn, const int8_t *hq, const uint16_t *hd, int hpad,
+                        const int32_t *slot_tok, const int32_t *slot_exp, const double *slot_w,
+                        int n_slots, int T, double *out64) {
+    if (!arena || !experts || !hq || !hd || !slot_tok || !slot_exp || !slot_w || !out64) return -1;
+    if (hidden <= 0 || ffn <= 0 || hpad % 32 || n_slots < 0 || T <= 0) return -1;
+    memset(out64, 0, sizeof(double) * (size_t)T * (size_t)hidden);
+    double *hhat = (double *)malloc(sizeof(double) * (size_t)hpad);
+    double *y = (double *)malloc(sizeof(double) * (size_t)hidden);
+    int err = 0;
+    for (int s = 0; s < n_slots && !err; s++) {
+        const int t = slot_tok[s], e = slot_exp[s];
+        if (t < 0 || t >= T || e < 0 || e >= n_experts) { err = -1; break; }
+        const oracle_expert *ex = &experts[e];
+        const int64_t fp = orc_padded(ex->fmt, ffn);
+        if (fp > hpad) { err = -1; break; }
+        orc_q8_1_values(hq + (int64_t)s * hpad, hd + (int64_t)s * (hpad / 32), fp, hhat);
+        const int64_t nb_down = fp / orc_block_weights(ex->fmt);
+#pragma omp parallel
+        {
+            double *sc = (double *)malloc(sizeof(double) * (size_t)fp);
+#pragma omp for schedule(static)
+            for (int i = 0; i < hidden; i++)                                     /* O8 */
+                y[i] = orc_row_dot(ex->fmt, arena + ex->off[2] + i * ex->stride[2], nb_down, hhat,
+                                   sc);
+            free(sc);
+        }
+        for (int i = 0; i < hidden; i++) out64[(int64_t)t * hidden + i] += slot_w[s] * y[i];   /* O9 */
+    }
+    free(hhat);
+    free(y);
+    return err;
 }
 
 /* O10: logits [T][E] (fp32, and the fp64 sums when l64 is not NULL) of x [T][H] and the
@@ -447,7 +501,7 @@ static int orc_forward(const uint8_t *arena, const oracle_expert *experts, int n
     if (hidden % 32 || n_tokens < 0) return -1;
     if (!tokens) n_tokens = T;
     int err = 0;
-#pragma omp parallel for schedule(dynamic, 1)
+    /* tokens in order; the threads work inside each expert's row loops (oracle_expert_ffn) */
     for (int it = 0; it < n_tokens; it++) {
         int t = tokens ? tokens[it] : it;
         if (t < 0 || t >= T) { err = -1; continue; }

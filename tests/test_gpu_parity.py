@@ -9,8 +9,8 @@ import pytest
 import oracle
 from expert_ffn_token_b200 import synth
 
-from gpu_helpers import (REL_TOL, W_TOL, device_layer, inputs, oracle_layer, rel_err,
-                         run_forward, torch_cuda, ws_array)
+from gpu_helpers import (W_TOL, check_parity, device_layer, inputs, run_forward, torch_cuda,
+                         ws_array)
 
 pytestmark = pytest.mark.gpu
 
@@ -144,21 +144,22 @@ def test_route_bit_exact(torch, T, E, k, ties):
 # ------------------------------------------------------------------ a1-a7 the layer
 
 
-def _check_layer(torch, w, layer, x, logits, flags=0, tokens=None, L=None, keep_h=False):
+def _check_layer(torch, w, layer, x, logits, flags=0, tokens=None, L=None, name=""):
+    """One forward through the C ABI on any path (flags), checked against the oracle: the
+    intermediates left in the workspace bit for bit, the Q8_1 of the GPU's own h bit for bit,
+    and the outputs through gpu_helpers.check_parity (h, the chain after h, end to end)."""
     from expert_ffn_token_b200 import moe
     T = x.shape[0]
+    fl = flags | moe.F_KEEP_H
     own = L is None
     if own:
-        L, _, _ = device_layer(w, layer, max_tokens=T, flags=flags | (moe.F_KEEP_H if keep_h else 0))
-    gpu = run_forward(L, x, logits, flags=flags | (moe.F_KEEP_H if keep_h else 0))
+        L, _, _ = device_layer(w, layer, max_tokens=T, flags=fl)
+    gpu = run_forward(L, x, logits, flags=fl)
     assert L.status() == 0
-    ref, rid, rw = oracle_layer(w, layer, x, logits, tokens)
-    sel = np.arange(T) if tokens is None else np.asarray(tokens)
-    err = rel_err(gpu[sel], ref)
-    assert err.max() <= REL_TOL, (err.max(), int(sel[err.argmax()]))
     # intermediates left in the workspace equal the standalone steps
-    v = L.views(T, flags | (moe.F_KEEP_H if keep_h else 0))
+    v = L.views(T, fl)
     k, E, H = w.k, w.n_experts, w.hidden
+    rid, rw, _ = oracle.topk(logits, k)
     assert np.array_equal(ws_array(L, v["ids"], T * k, np.int32).reshape(T, k), rid)
     assert np.abs(ws_array(L, v["w"], T * k, np.float32).reshape(T, k) - rw).max() <= W_TOL
     rq, rd, rs, _ = oracle.quantize_q8_1(x)
@@ -169,20 +170,21 @@ def _check_layer(torch, w, layer, x, logits, flags=0, tokens=None, L=None, keep_
     assert np.array_equal(ws_array(L, v["counts"], E, np.int32), rc)
     assert np.array_equal(ws_array(L, v["offsets"], E + 1, np.int32), ro)
     assert np.array_equal(ws_array(L, v["perm"], T * k, np.int32), rp)
-    if keep_h:
-        # the quantizer applied to the GPU's own h is bit-exact; h itself is within tolerance
-        hp, F = v["hpad"], w.ffn
-        n_slots = T * k + (T if w.shared else 0)
-        h = ws_array(L, v["h"], n_slots * F, np.float32).reshape(n_slots, F)
-        hq = ws_array(L, v["hq"], n_slots * hp, np.int8).reshape(n_slots, hp)
-        hd = ws_array(L, v["hd"], n_slots * hp // 32, np.uint16).reshape(n_slots, hp // 32)
-        hs = ws_array(L, v["hs"], n_slots * hp // 32, np.uint16).reshape(n_slots, hp // 32)
-        pad = np.zeros((n_slots, hp), np.float32)
-        pad[:, :F] = h
-        q2, d2, s2, _ = oracle.quantize_q8_1(pad)
-        assert np.array_equal(hq.ravel(), q2)
-        assert np.array_equal(hd.ravel(), d2)
-        assert np.array_equal(hs.ravel(), s2)
+    # the quantizer applied to the GPU's own h is bit-exact (every slot)
+    hp, F = v["hpad"], w.ffn
+    n_slots = T * k + (T if w.shared else 0)
+    h = ws_array(L, v["h"], n_slots * F, np.float32).reshape(n_slots, F)
+    hq = ws_array(L, v["hq"], n_slots * hp, np.int8).reshape(n_slots, hp)
+    hd = ws_array(L, v["hd"], n_slots * hp // 32, np.uint16).reshape(n_slots, hp // 32)
+    hs = ws_array(L, v["hs"], n_slots * hp // 32, np.uint16).reshape(n_slots, hp // 32)
+    pad = np.zeros((n_slots, hp), np.float32)
+    pad[:, :F] = h
+    q2, d2, s2, _ = oracle.quantize_q8_1(pad)
+    assert np.array_equal(hq.ravel(), q2)
+    assert np.array_equal(hd.ravel(), d2)
+    assert np.array_equal(hs.ravel(), s2)
+    check_parity(L, w, layer, x, logits, gpu, fl, tokens=tokens,
+                 name=name or f"{w.name} T={T} flags={flags}")
     if own:
         L.close()
     return gpu
@@ -192,21 +194,21 @@ def _check_layer(torch, w, layer, x, logits, flags=0, tokens=None, L=None, keep_
 def test_layer_tiny_all_paths(torch, flags):
     w = W["tiny"]
     x, logits = inputs(w, 0)
-    _check_layer(torch, w, 0, x, logits, flags=flags, keep_h=True)
+    _check_layer(torch, w, 0, x, logits, flags=flags)
 
 
 @pytest.mark.parametrize("layer", [0, 23, 47])
 def test_layer_decode_full_size(torch, layer):
     w = W["decode"]
     x, logits = inputs(w, layer)
-    _check_layer(torch, w, layer, x, logits, keep_h=True)
+    _check_layer(torch, w, layer, x, logits)
 
 
 @pytest.mark.parametrize("layer", [0, 47])
 def test_layer_mtp_verify_full_size(torch, layer):
     w = W["mtp_verify"]
     x, logits = inputs(w, layer)
-    _check_layer(torch, w, layer, x, logits, keep_h=True)
+    _check_layer(torch, w, layer, x, logits)
 
 
 def _sample_tokens(T, ids, n=24, seed=0):
@@ -240,20 +242,22 @@ def test_layer_ragged_batches(torch, T):
     if T > 64:
         ids, _, _ = oracle.topk(logits, w.k)
         tokens = _sample_tokens(T, ids, n=20, seed=T)
-    _check_layer(torch, w, 5, x, logits, keep_h=T <= 17, tokens=tokens)
+    _check_layer(torch, w, 5, x, logits, tokens=tokens)
 
 
 def test_decode_and_prefill_paths_agree(torch):
+    # both paths against the oracle on the same 12 tokens; each path repeats bit for bit
     from expert_ffn_token_b200 import moe
     w = synth.with_tokens(W["mtp_verify"], 12, layers=1)
     x, logits = inputs(w, 2)
-    L, _, _ = device_layer(w, 2, max_tokens=12, flags=moe.F_DETERMINISTIC)
-    a = run_forward(L, x, logits, flags=moe.F_FORCE_DECODE)
-    b = run_forward(L, x, logits, flags=moe.F_FORCE_PREFILL | moe.F_DETERMINISTIC)
-    c = run_forward(L, x, logits, flags=moe.F_FORCE_PREFILL | moe.F_DETERMINISTIC)
+    fl = moe.F_FORCE_PREFILL | moe.F_DETERMINISTIC | moe.F_KEEP_H
+    L, _, _ = device_layer(w, 2, max_tokens=12, flags=fl)
+    a = _check_layer(torch, w, 2, x, logits, flags=moe.F_FORCE_DECODE, L=L, name="paths: decode")
+    b = _check_layer(torch, w, 2, x, logits, flags=moe.F_FORCE_PREFILL | moe.F_DETERMINISTIC,
+                     L=L, name="paths: tensor cores, deterministic")
+    c = run_forward(L, x, logits, flags=fl)
     assert np.array_equal(b, c)                       # deterministic mode repeats bit for bit
-    assert rel_err(a, b.astype(np.float64)).max() <= REL_TOL
-    a2 = run_forward(L, x, logits, flags=moe.F_FORCE_DECODE)
+    a2 = run_forward(L, x, logits, flags=moe.F_FORCE_DECODE | moe.F_KEEP_H)
     assert np.array_equal(a, a2)                      # decode path is deterministic
     L.close()
 
@@ -298,6 +302,22 @@ def test_host_errors_enqueue_nothing(torch):
                               L.ws.data_ptr(), L.ws_bytes, 0, None) == moe.ERR_INVALID_ARG
     assert moe.forward_status(L.handle, x.data_ptr() + 4, lg.data_ptr(), 4, 2, out.data_ptr(),
                               L.ws.data_ptr(), L.ws_bytes, 0, None) == moe.ERR_ALIGNMENT
+    # the tensor-core path needs a workspace sized for it: no silent switch to other kernels
+    assert moe.forward_status(L.handle, x.data_ptr(), lg.data_ptr(), 4, 2, out.data_ptr(),
+                              L.ws.data_ptr(), L.ws_bytes, moe.F_FORCE_PREFILL,
+                              None) == moe.ERR_WORKSPACE
+    assert moe.forward_status(L.handle, x.data_ptr(), lg.data_ptr(), 4, 2, out.data_ptr(),
+                              L.ws.data_ptr(), L.ws_bytes,
+                              moe.F_FORCE_PREFILL | moe.F_FORCE_DECODE, None) == moe.ERR_INVALID_ARG
+    # the allocation-free entry point makes the same checks before it enqueues anything
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    n0 = moe.kernels_enqueued()
+    for args, code in (((x.data_ptr() + 4, lg.data_ptr(), 4, 2, out.data_ptr()), moe.ERR_ALIGNMENT),
+                       ((x.data_ptr(), lg.data_ptr(), 4, 17, out.data_ptr()), moe.ERR_INVALID_ARG),
+                       ((x.data_ptr(), lg.data_ptr() + 2, 4, 2, out.data_ptr()), moe.ERR_ALIGNMENT),
+                       ((x.data_ptr(), lg.data_ptr(), 4, 2, out.data_ptr() + 8), moe.ERR_ALIGNMENT)):
+        assert moe.forward_noalloc_status(L.handle, *args, st.data_ptr(), None) == code
+    assert moe.kernels_enqueued() == n0
     torch.cuda.synchronize()
     assert (out == 7.0).all()
     L.close()
@@ -307,7 +327,7 @@ def test_decode_large_expert_count_uses_grouped_kernels(torch):
     # 2048 experts exceed the fused decode kernel's plan: the three-kernel decode path runs
     w = synth.Workload("wideE", 70, 256, 256, 2048, 4, 3, True, 1, "normal", sigma=2.0)
     x, logits = inputs(w, 0)
-    _check_layer(torch, w, 0, x, logits, keep_h=True)
+    _check_layer(torch, w, 0, x, logits)
 
 
 # ------------------------------------------------------------------ Q5_1 experts
@@ -351,18 +371,18 @@ def test_q5_1_layer_every_path(torch, T, flags):
     # or to the tensor cores (4), deterministic (5)
     w = synth.with_tokens(Q51, T)
     x, logits = inputs(w, 0)
-    _check_layer(torch, w, 0, x, logits, flags=flags, keep_h=True)
+    _check_layer(torch, w, 0, x, logits, flags=flags)
 
 
 @pytest.mark.parametrize("T,flags", [(2, 0), (12, 0), (150, 2), (150, 4), (150, 5)])
 def test_four_formats_layer_every_path(torch, T, flags):
     w = synth.with_tokens(FOUR, T)
     x, logits = inputs(w, 0)
-    _check_layer(torch, w, 0, x, logits, flags=flags, keep_h=T <= 12)
+    _check_layer(torch, w, 0, x, logits, flags=flags)
 
 
 def test_q5_1_large_expert_count_grouped_decode(torch):
     w = synth.Workload("wideE_q51", 71, 256, 256, 2048, 4, 3, True, 1, "normal", sigma=2.0,
                        mix=((synth.Q5_1, 1.0),))
     x, logits = inputs(w, 0)
-    _check_layer(torch, w, 0, x, logits, keep_h=True)
+    _check_layer(torch, w, 0, x, logits)

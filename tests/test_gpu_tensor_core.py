@@ -7,10 +7,9 @@ deterministic mode repeating bit for bit; and the timing-events hook."""
 import numpy as np
 import pytest
 
-import oracle
 from expert_ffn_token_b200 import synth
 
-from gpu_helpers import REL_TOL, rel_err, torch_cuda
+from gpu_helpers import check_parity, torch_cuda
 
 pytestmark = pytest.mark.gpu
 
@@ -56,13 +55,6 @@ def _layer(torch, w, flags):
     return L, buf, lay
 
 
-def _oracle(w, buf, lay, x, logits):
-    ids, wt, _ = oracle.topk(logits, w.k)
-    ex = oracle.experts_table(lay.fmts, lay.offs, lay.strides)
-    out, _ = oracle.forward(buf, ex, lay.shared, w.hidden, w.ffn, x, ids, wt)
-    return out
-
-
 def _run(torch, L, x, logits, flags):
     xd = torch.from_numpy(x).cuda()
     ld = torch.from_numpy(logits).cuda()
@@ -76,26 +68,25 @@ def test_mixed_formats_and_zero_scales(torch):
     w = MIXED
     fmts = synth.layer_formats(w, 0)
     assert len(set(int(f) for f in fmts)) == 3
-    L, buf, lay = _layer(torch, w, moe.F_FORCE_PREFILL)
+    fl = moe.F_FORCE_PREFILL | moe.F_KEEP_H
+    L, buf, lay = _layer(torch, w, fl)
     x, logits = synth.activations(w, 0), synth.router_logits(w, 0)
-    gpu = _run(torch, L, x, logits, moe.F_FORCE_PREFILL)
+    gpu = _run(torch, L, x, logits, fl)
     assert L.status() == 0
-    ref = _oracle(w, buf, lay, x, logits)
-    err = rel_err(gpu, ref)
-    assert err.max() <= REL_TOL, (err.max(), int(err.argmax()))
+    check_parity(L, w, 0, x, logits, gpu, fl, host=(buf, lay), name="tc: mixed formats, zero scales")
     L.close()
 
 
 def test_deterministic_mode_repeats_bit_for_bit(torch):
     from expert_ffn_token_b200 import moe
     w = MIXED
-    flags = moe.F_FORCE_PREFILL | moe.F_DETERMINISTIC
-    L, buf, lay = _layer(torch, w, flags)
+    fl = moe.F_FORCE_PREFILL | moe.F_DETERMINISTIC | moe.F_KEEP_H
+    L, buf, lay = _layer(torch, w, fl)
     x, logits = synth.activations(w, 0), synth.router_logits(w, 0)
-    a = _run(torch, L, x, logits, flags)
-    b = _run(torch, L, x, logits, flags)
+    a = _run(torch, L, x, logits, fl)
+    b = _run(torch, L, x, logits, fl)
     assert np.array_equal(a, b)
-    assert rel_err(a, _oracle(w, buf, lay, x, logits)).max() <= REL_TOL
+    check_parity(L, w, 0, x, logits, a, fl, host=(buf, lay), name="tc: deterministic mode")
     L.close()
 
 

@@ -797,3 +797,56 @@ def test_generator_q6_k_blocks_and_padding():
             assert not W[:, width:].any() and W[:, :width].any()
     with pytest.raises(NotImplementedError):
         synth.device_fill_layer(w, 0, 0)
+
+
+@pytest.mark.parametrize("case", [
+    (61, None, 256, 256, 6, 2, 3, True),
+    (62, ((synth.Q4_K, 0.25), (synth.Q5_K, 0.5), (synth.Q8_0, 0.75), (synth.Q5_1, 1.0)),
+     512, 320, 8, 3, 4, True),
+])
+def test_down_combine_matches_dense_fp64(case):
+    # O8-O9 from Q8_1(h) rows given from outside, against a dense fp64 matmul of the exact down
+    # weights: random Q8_1 rows (int8 codes, positive fp16 scales), slots in a shuffled order
+    idx, mix, H, F, E, k, T, shared = case
+    w = _tiny(mix, H, F, E, k, T, shared, idx)
+    arena, lay = synth.host_arena(w, 0)
+    ex = oracle.experts_table(lay.fmts, lay.offs, lay.strides)
+    rng = np.random.default_rng(idx)
+    hpad = -(-F // 256) * 256
+    n = 11
+    slot_tok = rng.integers(0, T, n)
+    slot_exp = rng.integers(0, lay.n, n)
+    slot_w = rng.uniform(0.1, 1.0, n)
+    hq = rng.integers(-127, 128, (n, hpad)).astype(np.int8)
+    hd = np.float16(rng.uniform(1e-3, 10.0, (n, hpad // 32))).view(np.uint16)
+    got = oracle.down_combine(arena, ex, H, F, hq, hd, slot_tok, slot_exp, slot_w, T)
+    want = np.zeros((T, H))
+    for s in range(n):
+        _, _, Wd = _dense(arena, lay, int(slot_exp[s]), H, F)
+        fp = Wd.shape[1]
+        hh = hq[s, :fp].astype(np.float64) * np.repeat(hd[s].view(np.float16).astype(np.float64),
+                                                       32)[:fp]
+        want[slot_tok[s]] += slot_w[s] * (Wd @ hh)
+    assert np.allclose(got, want, rtol=1e-12, atol=1e-9 * np.abs(want).max())
+
+
+def test_down_combine_of_the_oracles_own_h_is_the_forward():
+    # with the Q8_1(h) of each (token, expert) as O5-O7 produce it, O8-O9 from outside give the
+    # layer's output exactly as the whole forward does (the same sums in the same order)
+    w = _tiny(None, 256, 256, 6, 2, 3, True, 63)
+    arena, lay = synth.host_arena(w, 0)
+    ex = oracle.experts_table(lay.fmts, lay.offs, lay.strides)
+    x = synth.activations(w, 0)
+    ids, wt, _ = oracle.topk(synth.router_logits(w, 0), 2)
+    _, out64 = oracle.forward(arena, ex, lay.shared, 256, 256, x, ids, wt)
+    rows_q, rows_d, st, se, sw = [], [], [], [], []
+    for t in range(3):
+        for e, wj in [(int(e), float(v)) for e, v in zip(ids[t], wt[t])] + [(6, 1.0)]:
+            r = oracle.expert_ffn(arena, ex[e], 256, 256, _q8_1_values(x[t]))
+            rows_q.append(r["hq"])
+            rows_d.append(r["hd"])
+            st.append(t)
+            se.append(e)
+            sw.append(wj)
+    got = oracle.down_combine(arena, ex, 256, 256, np.stack(rows_q), np.stack(rows_d), st, se, sw, 3)
+    assert np.array_equal(got, out64)
