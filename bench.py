@@ -380,13 +380,14 @@ def run_workload(name, args, world, dev):
         flops = 2.0 * assign * 2 * w.ffn * w.hidden
         achieved = flops / (gateup_ms / 1e3) / 1e12
         roofline = {"bound": "tensor", "achieved": achieved, "peak": bf16, "unit": "TFLOP/s",
-                    "frac": achieved / bf16, "traffic": traffic_for("k_gemm_tc<0>", name),
-                    "kernel": "k_gemm_tc<0> (gate/up grouped GEMM, tcgen05 kind::f16 with whole "
-                              "fp16 weights), one launch per layer",
+                    "frac": achieved / bf16, "traffic": traffic_for("k_gateup_tc", name),
+                    "kernel": "k_gateup_tc (gate/up grouped GEMM, tcgen05 kind::f16: exact integer "
+                              "weight operands, hi/lo activation planes), one launch per layer",
                     "peak_source": f"{src} bf16 dense (fp16 runs at the same rate)",
                     "flops_per_launch": flops, "ms_per_launch": gateup_ms,
                     "frac_of_int8_peak": achieved / int8_meas,
-                    "down_ms_per_launch": down_ms}
+                    "down_ms_per_launch": down_ms,
+                    "down_note": "k_h_rows + k_down_tc, from the events around the down phase"}
     res = {
         "workload": w.note, "value": job_throughput(tok_per_step, K, world, ms),
         "unit": "tokens/s", "steps": K, "warmup": W, "ms_per_step": ms_step,

@@ -108,10 +108,8 @@ __device__ __forceinline__ Smem carve(uint8_t *base, const GemmArgs &a) {
 
 // ---------------------------------------------------------------- warp 0: weight producer
 
-__device__ void role_producer(const GemmArgs &a, const Smem &S, int nj, int (&slot_hist)[kMaxDR],
-                              uint32_t (&ph_hist)[kMaxDR], int &issued) {
+__device__ void role_producer(const GemmArgs &a, const Smem &S, int nj, Ring &rr, int &issued) {
     Cursor cur;
-    Ring rr;
     const int nsb = (a.nst + 3) / 4;
     for (int i = blockIdx.x;; i += gridDim.x) {
         Tile t;
@@ -130,8 +128,6 @@ __device__ void role_producer(const GemmArgs &a, const Smem &S, int nj, int (&sl
                 mbar_arrive_expect_tx(S.raw_full + rr.s, 128u * sbb);
                 tma_load_2d(S.raw + (size_t)rr.s * a.rawb, m, sb * xu, hh ? y1 : y0,
                             S.raw_full + rr.s);
-                slot_hist[issued % kMaxDR] = rr.s;
-                ph_hist[issued % kMaxDR] = rr.ph;
                 issued++;
                 rr.adv(1, a.DR);
             }
@@ -366,8 +362,7 @@ __device__ void role_loader(const GemmArgs &a, const Smem &S, int nj) {
     const int c = lane & 7;                        // 16-byte chunk of a 128-byte row
     const int rg = 4 * wl + (lane >> 3);           // rows rg + 8 j, j = 0..15
     Cursor cur;
-    Ring rb, rt;
-    int pend[8];
+    Ring rb, rt, ob;                               // ob: oldest stage issued, not yet signalled
     int npend = 0;
     bool ok = true;
     for (int i = blockIdx.x; ok; i += gridDim.x) {
@@ -410,15 +405,15 @@ __device__ void role_loader(const GemmArgs &a, const Smem &S, int nj) {
                                col + (size_t)n * a.act_pitch);
             }
             cp_async_commit();
-            pend[npend++] = rb.s;
+            if (npend++ == 0) ob = rb;
             rb.adv(1, a.DB);
             if (npend > a.lag) {
                 if (a.lag >= 3) cp_async_wait<3>();
                 else cp_async_wait<2>();
                 fence_proxy_async_smem();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(S.b_full + pend[0]);
-                for (int q = 0; q + 1 < npend; q++) pend[q] = pend[q + 1];
+                if (lane == 0) mbar_arrive(S.b_full + ob.s);
+                ob.adv(1, a.DB);
                 npend--;
             }
         }
@@ -426,9 +421,10 @@ __device__ void role_loader(const GemmArgs &a, const Smem &S, int nj) {
         cp_async_wait<0>();
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0)
-            for (int q = 0; q < npend; q++) mbar_arrive(S.b_full + pend[q]);
-        npend = 0;
+        for (; npend > 0; npend--) {
+            if (lane == 0) mbar_arrive(S.b_full + ob.s);
+            ob.adv(1, a.DB);
+        }
     }
     cp_async_wait<0>();
 }
@@ -531,16 +527,19 @@ __global__ void __launch_bounds__(kThreads, 1) k_down_tc(const GemmArgs a) {
 
     if (warp == 0) {
         if (lane == 0) {
-            int slot_hist[kMaxDR];
-            uint32_t ph_hist[kMaxDR];
+            Ring rr;
             int issued = 0;
-            role_producer(a, S, nj, slot_hist, ph_hist, issued);
+            role_producer(a, S, nj, rr, issued);
             if (*(volatile int *)S.abort) {
-                // the loads already issued land before the CTA leaves (each wait bounded)
+                // the loads already issued land before the CTA leaves (each wait bounded): walk
+                // back over the last positions filled, one ring's worth at most
                 const int n = issued < a.DR ? issued : a.DR;
-                for (int k = 1; k <= n; k++) {
-                    const int h = (issued - k) % kMaxDR;
-                    mbar_wait_bounded(S.raw_full + slot_hist[h], ph_hist[h], 20000000ull);
+                for (int k = 0; k < n; k++) {
+                    if (--rr.s < 0) {
+                        rr.s = a.DR - 1;
+                        rr.ph ^= 1u;
+                    }
+                    mbar_wait_bounded(S.raw_full + rr.s, rr.ph, 20000000ull);
                 }
             }
         }

@@ -61,8 +61,8 @@ constexpr uint32_t kBStage = 2 * kAtomB;         // hi, lo
 constexpr uint32_t kMinW = 128 * 32;             // 128 rows x 8 tf32 (32-byte swizzle)
 constexpr uint32_t kMinX = kTN * 32;             // 64 token rows x 8 tf32
 constexpr uint32_t kMStage = 4 * kMinW + 2 * kMinX;   // [g hi][g lo][u hi][u lo][x hi][x lo]
-constexpr uint32_t kSStage = 2 * 8 * 128 * 4;    // row scales [matrix][group][row]
-constexpr int kMaxDA = 3, kMaxDB = 4, kMaxDR = 8;
+constexpr uint32_t kSStage = 2 * 8 * 128 * 2;    // row scales (fp16) [matrix][group][row]
+constexpr int kMaxDA = 3, kMaxDB = 6, kMaxDR = 8;
 constexpr uint32_t kTmemCols = 512;              // 2 x (gate | up) group buffers + 2 min buffers
 constexpr size_t kSmemCap = 232448;
 
@@ -75,7 +75,7 @@ struct TileInfo {
 
 struct Smem {
     uint8_t *A, *B, *M, *raw;
-    float *scale;
+    __half *scale;
     TileInfo *ti;
     uint64_t *raw_full, *raw_empty, *a_full, *a_empty, *b_full, *b_empty, *m_full, *m_empty,
         *s_full, *s_empty, *pg_full, *pg_empty, *tm_full, *tm_empty, *ti_full, *ti_empty, *done;
@@ -84,9 +84,9 @@ struct Smem {
 };
 
 __host__ __device__ inline size_t smem_plan(int DA, int DB, int DR, uint32_t rawb) {
-    return 1024 + (size_t)DA * kAStage + (size_t)DB * kBStage + kMStage + 2 * (size_t)kSStage +
+    return 1024 + (size_t)DA * kAStage + (size_t)DB * kBStage + 2 * kMStage + 2 * (size_t)kSStage +
            (size_t)DR * rawb + 2 * sizeof(TileInfo) +
-           8 * (2 * kMaxDR + 2 * kMaxDA + 2 * kMaxDB + 13) + 16;
+           8 * (2 * kMaxDR + 2 * kMaxDA + 2 * kMaxDB + 15) + 16;
 }
 
 __device__ __forceinline__ Smem carve(uint8_t *base, const GemmArgs &a) {
@@ -97,8 +97,8 @@ __device__ __forceinline__ Smem carve(uint8_t *base, const GemmArgs &a) {
     s.B = p;
     p += (size_t)a.DB * kBStage;
     s.M = p;
-    p += kMStage;
-    s.scale = reinterpret_cast<float *>(p);
+    p += 2 * kMStage;
+    s.scale = reinterpret_cast<__half *>(p);
     p += 2 * (size_t)kSStage;
     s.raw = p;
     p += (size_t)a.DR * a.rawb;
@@ -111,8 +111,8 @@ __device__ __forceinline__ Smem carve(uint8_t *base, const GemmArgs &a) {
     s.a_empty = b; b += kMaxDA;
     s.b_full = b; b += kMaxDB;
     s.b_empty = b; b += kMaxDB;
-    s.m_full = b; b += 1;
-    s.m_empty = b; b += 1;
+    s.m_full = b; b += 2;
+    s.m_empty = b; b += 2;
     s.s_full = b; b += 2;
     s.s_empty = b; b += 2;
     s.pg_full = b; b += 2;
@@ -133,10 +133,8 @@ __device__ __forceinline__ bool small_fmt(int fmt) {
 
 // ---------------------------------------------------------------- warp 0: weight producer
 
-__device__ void role_producer(const GemmArgs &a, const Smem &S, int nj, int (&slot_hist)[kMaxDR],
-                              uint32_t (&ph_hist)[kMaxDR], int &issued) {
+__device__ void role_producer(const GemmArgs &a, const Smem &S, int nj, Ring &rr, int &issued) {
     Cursor cur;
-    Ring rr;
     const int nsb = a.H / 256;
     for (int i = blockIdx.x;; i += gridDim.x) {
         Tile t;
@@ -155,8 +153,6 @@ __device__ void role_producer(const GemmArgs &a, const Smem &S, int nj, int (&sl
                 mbar_arrive_expect_tx(S.raw_full + rr.s, 128u * sbb);
                 tma_load_2d(S.raw + (size_t)rr.s * a.rawb, hh ? m1 : m0, sb * xu, y,
                             S.raw_full + rr.s);
-                slot_hist[issued % kMaxDR] = rr.s;
-                ph_hist[issued % kMaxDR] = rr.ph;
                 issued++;
                 rr.adv(1, a.DR);
             }
@@ -306,13 +302,13 @@ __device__ __forceinline__ bool unpack_sb(const GemmArgs &a, const Smem &S, Ring
     row_consts<FMT>(rowu, du, wu, scu, qhu);
     // promotion scales of this super-block's groups
     if (!waitw(a, S.abort, S.s_empty + rs.s, rs.ph ^ 1u)) return false;
-    float *sc = S.scale + (size_t)rs.s * (kSStage / 4);
+    __half *sc = S.scale + (size_t)rs.s * (kSStage / 2);
     const int ng = small_fmt(FMT) ? 8 : 1;
 #pragma unroll
     for (int g = 0; g < 8; g++) {
-        if (g < ng) {
-            sc[(0 * 8 + g) * 128 + r] = dg[g];
-            sc[(1 * 8 + g) * 128 + r] = du[g];
+        if (g < ng) {   // the scales are fp16 values of the blocks: exact as __half
+            sc[(0 * 8 + g) * 128 + r] = __float2half_rn(dg[g]);
+            sc[(1 * 8 + g) * 128 + r] = __float2half_rn(du[g]);
         }
     }
     __syncwarp();
@@ -327,19 +323,20 @@ __device__ __forceinline__ bool unpack_sb(const GemmArgs &a, const Smem &S, Ring
             hi[j] = tf32_round(wg[j]);
             lo[j] = tf32_round(wg[j] - hi[j]);
         }
-        store_min_row(S.M + 0 * kMinW, r, hi);
-        store_min_row(S.M + 1 * kMinW, r, lo);
+        uint8_t *ms = S.M + (size_t)rm.s * kMStage;
+        store_min_row(ms + 0 * kMinW, r, hi);
+        store_min_row(ms + 1 * kMinW, r, lo);
 #pragma unroll
         for (int j = 0; j < 8; j++) {
             hi[j] = tf32_round(wu[j]);
             lo[j] = tf32_round(wu[j] - hi[j]);
         }
-        store_min_row(S.M + 2 * kMinW, r, hi);
-        store_min_row(S.M + 3 * kMinW, r, lo);
+        store_min_row(ms + 2 * kMinW, r, hi);
+        store_min_row(ms + 3 * kMinW, r, lo);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(S.m_full + rm.s);
-        rm.adv(1, 1);
+        rm.adv(1, 2);
     }
     // the four 64-wide stages
 #pragma unroll 1
@@ -411,25 +408,6 @@ __device__ void role_mma(const GemmArgs &a, const Smem &S, int nj, uint32_t tbas
         tc_fence_after();
         const uint32_t dmin = tbase + 256 + (uint32_t)rt.s * 128;   // gate min, up min at +64
         for (int sb = 0; sb < nsb; sb++) {
-            if (mn) {   // the min term of this super-block, before its main products
-                if (!wait1(a, S.abort, S.m_full + rm.s, rm.ph)) return;
-                tc_fence_after();
-                const uint64_t wgh = smem_desc(m_base + 0 * kMinW, 256, 6);
-                const uint64_t wgl = smem_desc(m_base + 1 * kMinW, 256, 6);
-                const uint64_t wuh = smem_desc(m_base + 2 * kMinW, 256, 6);
-                const uint64_t wul = smem_desc(m_base + 3 * kMinW, 256, 6);
-                const uint64_t xh = smem_desc(m_base + 4 * kMinW, 256, 6);
-                const uint64_t xl = smem_desc(m_base + 4 * kMinW + kMinX, 256, 6);
-                const uint32_t acc0 = sb > 0 ? 1u : 0u;
-                umma_tf32(dmin, wgh, xh, idt, acc0);
-                umma_tf32(dmin, wgh, xl, idt, 1u);
-                umma_tf32(dmin, wgl, xh, idt, 1u);
-                umma_tf32(dmin + 64, wuh, xh, idt, acc0);
-                umma_tf32(dmin + 64, wuh, xl, idt, 1u);
-                umma_tf32(dmin + 64, wul, xh, idt, 1u);
-                umma_commit(S.m_empty + rm.s);
-                rm.adv(1, 1);
-            }
             for (int st = 0; st < 4; st++) {
                 if (!wait1(a, S.abort, S.a_full + ra.s, ra.ph)) return;
                 if (!wait1(a, S.abort, S.b_full + rb.s, rb.ph)) return;
@@ -464,6 +442,27 @@ __device__ void role_mma(const GemmArgs &a, const Smem &S, int nj, uint32_t tbas
                 ra.adv(1, a.DA);
                 rb.adv(1, a.DB);
             }
+            if (mn) {   // the min term of this super-block, after its main products (its operands
+                        // came with the super-block's first stage, so they have landed by now)
+                if (!wait1(a, S.abort, S.m_full + rm.s, rm.ph)) return;
+                tc_fence_after();
+                const uint32_t mb = m_base + (uint32_t)rm.s * kMStage;
+                const uint64_t wgh = smem_desc(mb + 0 * kMinW, 256, 6);
+                const uint64_t wgl = smem_desc(mb + 1 * kMinW, 256, 6);
+                const uint64_t wuh = smem_desc(mb + 2 * kMinW, 256, 6);
+                const uint64_t wul = smem_desc(mb + 3 * kMinW, 256, 6);
+                const uint64_t xh = smem_desc(mb + 4 * kMinW, 256, 6);
+                const uint64_t xl = smem_desc(mb + 4 * kMinW + kMinX, 256, 6);
+                const uint32_t acc0 = sb > 0 ? 1u : 0u;
+                umma_tf32(dmin, wgh, xh, idt, acc0);
+                umma_tf32(dmin, wgh, xl, idt, 1u);
+                umma_tf32(dmin, wgl, xh, idt, 1u);
+                umma_tf32(dmin + 64, wuh, xh, idt, acc0);
+                umma_tf32(dmin + 64, wuh, xl, idt, 1u);
+                umma_tf32(dmin + 64, wul, xh, idt, 1u);
+                umma_commit(S.m_empty + rm.s);
+                rm.adv(1, 2);
+            }
         }
         umma_commit(S.tm_full + rt.s);
         rt.adv(1, 2);
@@ -479,8 +478,9 @@ __device__ void role_loader(const GemmArgs &a, const Smem &S, int nj) {
     const int rg = lt >> 3;                      // rows rg + 8 j, j = 0..7
     Cursor cur;
     Ring rb, rt, rm;
-    int pend_b[4], pend_m[4];
-    int npend = 0;
+    // stages issued but not yet signalled are consecutive: the oldest one's B and M positions
+    Ring ob, om;
+    int og = 0, npend = 0;
     bool ok = true;
     const int nsb = a.H / 256;
     const int H32 = a.H / 32;
@@ -519,23 +519,36 @@ __device__ void role_loader(const GemmArgs &a, const Smem &S, int nj) {
         if (lane == 0) mbar_arrive(S.ti_full + rt.s);
         rt.adv(1, 2);
         const bool mn = has_min(t.fmt);
+        ob = rb;
+        om = rm;
+        og = 0;
+        // signal the oldest issued stage (its copies have landed): B, and the block sums it
+        // carried at a super-block's first stage
+        auto signal_oldest = [&]() {
+            if (lane == 0) {
+                mbar_arrive(S.b_full + ob.s);
+                if (mn && (og & 3) == 0) mbar_arrive(S.m_full + om.s);
+            }
+            if (mn && (og & 3) == 0) om.adv(1, 2);
+            ob.adv(1, a.DB);
+            og++;
+            npend--;
+        };
         for (int sb = 0; sb < nsb && ok; sb++) {
             for (int st = 0; st < 4; st++) {
-                int mslot = -1;
                 if (st == 0 && mn) {   // the block sums of this super-block (min-term operand)
                     if (!(ok = waitw(a, S.abort, S.m_empty + rm.s, rm.ph ^ 1u))) break;
                     if (my_tok >= 0) {
                         const int sw = (lt >> 2) & 1;
                         const float *hs = a.xs_hi + (size_t)my_tok * H32 + 8 * sb;
                         const float *ls = a.xs_lo + (size_t)my_tok * H32 + 8 * sb;
-                        uint8_t *xh = S.M + 4 * kMinW + lt * 32;
+                        uint8_t *xh = S.M + (size_t)rm.s * kMStage + 4 * kMinW + lt * 32;
                         cp_async16(xh + ((0 ^ sw) << 4), hs);
                         cp_async16(xh + ((1 ^ sw) << 4), hs + 4);
                         cp_async16(xh + kMinX + ((0 ^ sw) << 4), ls);
                         cp_async16(xh + kMinX + ((1 ^ sw) << 4), ls + 4);
                     }
-                    mslot = rm.s;
-                    rm.adv(1, 1);
+                    rm.adv(1, 2);
                 }
                 if (!(ok = waitw(a, S.abort, S.b_empty + rb.s, rb.ph ^ 1u))) break;
                 uint8_t *bs = S.B + (size_t)rb.s * kBStage;
@@ -552,24 +565,16 @@ __device__ void role_loader(const GemmArgs &a, const Smem &S, int nj) {
                     }
                 }
                 cp_async_commit();
-                pend_b[npend] = rb.s;
-                pend_m[npend] = mslot;
                 npend++;
                 rb.adv(1, a.DB);
                 if (npend > a.lag) {
-                    if (a.lag >= 2) cp_async_wait<2>();
+                    if (a.lag >= 4) cp_async_wait<4>();
+                    else if (a.lag == 3) cp_async_wait<3>();
+                    else if (a.lag == 2) cp_async_wait<2>();
                     else cp_async_wait<1>();
                     fence_proxy_async_smem();
                     __syncwarp();
-                    if (lane == 0) {
-                        mbar_arrive(S.b_full + pend_b[0]);
-                        if (pend_m[0] >= 0) mbar_arrive(S.m_full + pend_m[0]);
-                    }
-                    for (int q = 0; q + 1 < npend; q++) {
-                        pend_b[q] = pend_b[q + 1];
-                        pend_m[q] = pend_m[q + 1];
-                    }
-                    npend--;
+                    signal_oldest();
                 }
             }
         }
@@ -577,12 +582,7 @@ __device__ void role_loader(const GemmArgs &a, const Smem &S, int nj) {
         cp_async_wait<0>();
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0)
-            for (int q = 0; q < npend; q++) {
-                mbar_arrive(S.b_full + pend_b[q]);
-                if (pend_m[q] >= 0) mbar_arrive(S.m_full + pend_m[q]);
-            }
-        npend = 0;
+        while (npend > 0) signal_oldest();
     }
     cp_async_wait<0>();
 }
@@ -608,9 +608,10 @@ __device__ void role_epilogue(const GemmArgs &a, const Smem &S, int nj, uint32_t
         for (int j = 0; j < 32; j++) tg[j] = tu[j] = 0.0f;
         for (int sb = 0; sb < nsb; sb++) {
             if (!waitw(a, S.abort, S.s_full + rs.s, rs.ph)) return;
-            const float *sc = S.scale + (size_t)rs.s * (kSStage / 4);
+            const __half *sc = S.scale + (size_t)rs.s * (kSStage / 2);
             for (int g = 0; g < ng; g++) {
-                const float dg = sc[(0 * 8 + g) * 128 + r], du = sc[(1 * 8 + g) * 128 + r];
+                const float dg = __half2float(sc[(0 * 8 + g) * 128 + r]);
+                const float du = __half2float(sc[(1 * 8 + g) * 128 + r]);
                 if (!waitw(a, S.abort, S.pg_full + rg.s, rg.ph)) return;
                 tc_fence_after();
                 const uint32_t col = tbase + lane_addr + (uint32_t)rg.s * 128 + 32 * ch;
@@ -700,9 +701,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_gateup_tc(const GemmArgs a) {
             mbar_init(S.b_full + i, kLoadWarps);
             mbar_init(S.b_empty + i, 1);
         }
-        mbar_init(S.m_full, kUnpackWarps + kLoadWarps);
-        mbar_init(S.m_empty, 1);
         for (int i = 0; i < 2; i++) {
+            mbar_init(S.m_full + i, kUnpackWarps + kLoadWarps);
+            mbar_init(S.m_empty + i, 1);
             mbar_init(S.s_full + i, kUnpackWarps);
             mbar_init(S.s_empty + i, kEpiWarps);
             mbar_init(S.pg_full + i, 1);
@@ -728,16 +729,19 @@ __global__ void __launch_bounds__(kThreads, 1) k_gateup_tc(const GemmArgs a) {
 
     if (warp == 0) {
         if (lane == 0) {
-            int slot_hist[kMaxDR];
-            uint32_t ph_hist[kMaxDR];
+            Ring rr;
             int issued = 0;
-            role_producer(a, S, nj, slot_hist, ph_hist, issued);
+            role_producer(a, S, nj, rr, issued);
             if (*(volatile int *)S.abort) {
-                // the loads already issued land before the CTA leaves (each wait bounded)
+                // the loads already issued land before the CTA leaves (each wait bounded): walk
+                // back over the last positions filled, one ring's worth at most
                 const int n = issued < a.DR ? issued : a.DR;
-                for (int k = 1; k <= n; k++) {
-                    const int h = (issued - k) % kMaxDR;
-                    mbar_wait_bounded(S.raw_full + slot_hist[h], ph_hist[h], 20000000ull);
+                for (int k = 0; k < n; k++) {
+                    if (--rr.s < 0) {
+                        rr.s = a.DR - 1;
+                        rr.ph ^= 1u;
+                    }
+                    mbar_wait_bounded(S.raw_full + rr.s, rr.ph, 20000000ull);
                 }
             }
         }
@@ -774,18 +778,21 @@ uint32_t raw_bytes(int fmt_mask) {
     return ((128u * sbb_max) + 1023u) & ~1023u;
 }
 
-// Ring depths that fit the shared memory: two integer-operand stages, three or two activation
-// stages, and as many packed stages (two per super-block, at least two super-blocks when the
-// formats allow) as the rest holds.
+// Ring depths that fit the shared memory: two integer-operand stages, the deepest activation
+// ring (five down to two stages: the gathers come from L2 and want several stages in flight)
+// that leaves room for three packed half-stages (one and a half super-blocks), else the deepest
+// one with one super-block of packed rows (the 272-byte Q8_0 super-blocks need that).
 bool ring_plan(int fmt_mask, int &DA, int &DB, int &DR) {
     const uint32_t rawb = raw_bytes(fmt_mask);
     DA = 2;
-    for (DB = 3; DB >= 2; DB--) {
-        const size_t fixed = smem_plan(DA, DB, 0, rawb);
-        if (fixed >= kSmemCap) continue;
-        DR = (int)((kSmemCap - fixed) / rawb);
-        if (DR > kMaxDR) DR = kMaxDR;
-        if (DR >= 4 || (DB == 2 && DR >= 2)) return true;
+    for (int need = 3; need >= 2; need--) {
+        for (DB = 5; DB >= 2; DB--) {
+            const size_t fixed = smem_plan(DA, DB, 0, rawb);
+            if (fixed >= kSmemCap) continue;
+            DR = (int)((kSmemCap - fixed) / rawb);
+            if (DR > kMaxDR) DR = kMaxDR;
+            if (DR >= need) return true;
+        }
     }
     return false;
 }
