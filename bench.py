@@ -10,6 +10,9 @@ A step is one pass of the whole layer (a1-a7) over one batch of synthetic input 
   mtp_verify    48 layers (hidden 2560, 512 experts, top-10 + shared, width 640), 3 tokens each
   prefill       one 4096-token chunk of the 512-expert layer (rotating over 4 layers)
   mixed_prefill one 8192-token chunk, per-expert Q4_K / Q5_K / Q8_0, Zipf(1.3) routing
+  chain         one token through 48 chained decode-shaped layers on a residual stream
+                (moe_chain_forward: router in front of every layer, residual add, and the
+                next layer's expert prediction prefetched into L2), one CUDA graph per step
 The default (`all`) times every workload one after the other (each arena freed before the next)
 and reports the decode workload as the line's headline value, the others under "workloads".
 The metric is MoE-layer tokens/s (tokens x layers / time).  Per workload:
@@ -48,7 +51,7 @@ METRIC = "MoE-layer tokens/s; decode expert-weight GB/s and prefill int8 TOPS vs
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 INT8_NOMINAL_TOPS = 4500.0          # B200 dense int8, datasheet figure
-ALL = ("decode", "mtp_verify", "prefill", "mixed_prefill")
+ALL = ("decode", "mtp_verify", "prefill", "mixed_prefill", "chain")
 HEADLINE = "decode"
 
 
@@ -418,7 +421,199 @@ def run_workload(name, args, world, dev):
     return res
 
 
+def run_chain(name, args, world, dev):
+    """One token through 48 chained decode-shaped layers (moe_chain_forward with the lookahead),
+    one CUDA graph per step; the same chain without the lookahead timed beside it."""
+    import numpy as np
+    import torch
+
+    from expert_ffn_token_b200 import moe, synth
+
+    w = workload("decode", args.layers)
+    K = args.steps if args.steps is not None else 50
+    W = args.warmup if args.warmup is not None else 5
+    stream = torch.cuda.current_stream().cuda_stream
+    lays = [synth.arena_layout(w, synth.layer_formats(w, l)) for l in range(w.layers)]
+    offs = [0]
+    for lay in lays[:-1]:
+        offs.append(offs[-1] + lay.nbytes)
+    arena = torch.empty(offs[-1] + lays[-1].nbytes, dtype=torch.uint8, device=dev)
+    for l in range(w.layers):
+        synth.device_fill_layer(w, l, arena.data_ptr() + offs[l], stream)
+    handles = [moe.arena_create(arena.data_ptr() + offs[l], lay.nbytes, w.hidden, w.ffn,
+                                w.n_experts, -1, synth.layout_descs(lay))
+               for l, lay in enumerate(lays)]
+    # router rows: N(0, 0.05^2) fp32, drawn on the device from a seeded generator
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(w.seed)
+    routers = torch.randn((w.layers, w.n_experts, w.hidden), generator=gen, device=dev) * 0.05
+    # RMSNorm weight 1/32: keeps the random (not zero-mean) experts' h inside the fp16 range of
+    # its Q8_1 scales along the chain
+    gamma = torch.full((w.hidden,), 2.0 ** -5, dtype=torch.float32, device=dev)
+    layers = [(handles[l], routers[l].data_ptr(), None, gamma.data_ptr())
+              for l in range(w.layers)]
+    T, k, H = w.tokens, w.k, w.hidden
+    x0 = synth.activations(w, 0)
+    x_d = torch.from_numpy(x0).to(dev)
+    xo_d = torch.empty_like(x_d)
+    fl_on, fl_off = moe.F_LOOKAHEAD, 0
+    ws_bytes = moe.chain_workspace_size(layers, T, k, fl_on)
+    ws = torch.zeros(ws_bytes, dtype=torch.uint8, device=dev)
+
+    # one traced run: the ids of every layer (expert bytes per step) and the lookahead's hits
+    ids_t = torch.empty((w.layers, T, k), dtype=torch.int32, device=dev)
+    early_t = torch.full((w.layers, T, k), -1, dtype=torch.int32, device=dev)
+    moe.chain_forward(layers, x_d.data_ptr(), T, k, xo_d.data_ptr(), ws.data_ptr(), ws_bytes,
+                      fl_on, {"ids": ids_t.data_ptr(), "early": early_t.data_ptr()}, stream)
+    torch.cuda.synchronize()
+    ids = ids_t.cpu().numpy()
+    early = early_t.cpu().numpy()
+    hits = sum(len(set(ids[l].ravel()) & set(early[l].ravel())) for l in range(1, w.layers))
+    picks = sum(len(set(ids[l].ravel())) for l in range(1, w.layers))
+    step_bytes = sum(sum(lays[l].expert_bytes(int(e)) for e in set(ids[l].ravel()))
+                     for l in range(w.layers))
+
+    def capture(flags):
+        def one():
+            moe.chain_forward(layers, x_d.data_ptr(), T, k, xo_d.data_ptr(), ws.data_ptr(),
+                              ws_bytes, flags, None, torch.cuda.current_stream().cuda_stream)
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            one()
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        n0 = moe.kernels_enqueued()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            one()
+        n = moe.kernels_enqueued() - n0
+        torch.cuda.synchronize()
+        return g, n, one
+
+    g_on, kern_on, eager_on = capture(fl_on)
+    g_off, _, _ = capture(fl_off)
+
+    def timed(fn, steps):
+        for _ in range(W):
+            fn()
+        torch.cuda.synchronize()
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(steps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return max_over_ranks(e0.elapsed_time(e1), world, dev)
+
+    gpu_id = (os.environ["CUDA_VISIBLE_DEVICES"].split(",")[dev.index]
+              if "CUDA_VISIBLE_DEVICES" in os.environ else dev.index)
+    clocks = Clocks(gpu_id)
+    ms = timed(g_on.replay, K)
+    ms_off = timed(g_off.replay, K)
+    clock_rows = clocks.stop()
+
+    # end to end through the C ABI: x0 from pinned host memory, moe_chain_forward (eager), x_L
+    # back to the host, every step
+    x_h = torch.from_numpy(x0).pin_memory()
+    xo_h = torch.empty(xo_d.shape, dtype=torch.float32).pin_memory()
+
+    def e2e_step():
+        x_d.copy_(x_h, non_blocking=True)
+        eager_on()
+        xo_h.copy_(xo_d, non_blocking=True)
+
+    k2 = max(3, K // 2)
+    ms_e2e = timed(e2e_step, k2)
+    assert np.isfinite(xo_h.numpy()).all()
+    st = moe.read_status(moe.chain_status_word(layers, ws.data_ptr(), T, k, fl_on), stream)
+    if st != 0:
+        raise RuntimeError(f"chain: device status {moe.status_string(st)}")
+    sample = {"w": w, "x0": x0, "ids": ids, "routers": routers.cpu().numpy(),
+              "norm": gamma.cpu().numpy()}
+    g_on = g_off = None
+    for h in handles:
+        moe.arena_destroy(h)
+    del arena, ws, routers
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+
+    hbm, _, src = peaks()
+    ms_step = ms / K
+    layer_s = ms_step / 1e3 / w.layers
+    achieved = step_bytes / w.layers / layer_s / 1e9
+    return {
+        "workload": "one token through 48 chained decode-shaped layers (hidden 2048, 256 "
+                    "experts, top-8, width 512, Q4_K) on a residual stream: RMSNorm (weight "
+                    "1/32) + router (fp32 rows N(0, 0.05^2)) + layer + residual add per layer, "
+                    "lookahead prefetch on",
+        "value": job_throughput(T * w.layers, K, world, ms), "unit": "tokens/s",
+        "steps": K, "warmup": W, "ms_per_step": ms_step, "us_per_layer": 1e6 * layer_s,
+        "layers": w.layers, "tokens_per_layer": T, "hidden": H, "experts": w.n_experts,
+        "top_k": k, "shared_expert": False, "ffn": w.ffn,
+        "chain_tokens_per_s": job_throughput(T, K, world, ms),
+        "lookahead_off": {"ms_per_step": ms_off / K,
+                          "us_per_layer": 1e3 * ms_off / K / w.layers,
+                          "value": job_throughput(T * w.layers, K, world, ms_off)},
+        "lookahead_hit_rate": hits / max(1, picks),
+        "l2": f"{step_bytes / 1e6:.0f} MB of distinct expert bytes per step (L2 126 MB)",
+        "expert_bytes_per_step": step_bytes,
+        "expert_gbs": step_bytes / (ms_step / 1e3) / 1e9,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                     "frac": achieved / hbm, "traffic": None,
+                     "kernel": "the chained layer (k_router_rows + k_lookahead + "
+                               "k_decode_fused per layer): expert bytes per layer / layer time",
+                     "peak_source": f"{src} HBM copy"},
+        "e2e": {"value": job_throughput(T * w.layers, k2, world, ms_e2e), "unit": "tokens/s",
+                "h2d_bytes_per_step": int(x0.nbytes), "d2h_bytes_per_step": int(xo_h.numel() * 4),
+                "mode": "eager moe_chain_forward through the C ABI"},
+        "gpu_launches": int(kern_on * K),
+        "kernels_per_step": int(kern_on),
+        "clock_rows": clock_rows,
+        "_chain_sample": sample,
+    }
+
+
 # ------------------------------------------------------------------ oracle (CPU baseline)
+
+
+def chain_oracle_sample(cs, seconds, threads=None):
+    """The oracle's chain (O10, O3, O1-O9 and the residual add per layer) on the first layers of
+    the chain workload, from the same x0 and router rows, until ~`seconds` of CPU time.  The
+    arenas hold the experts the GPU's chain chose (input generation, not timed); a layer whose
+    oracle ids differ from them ends the sample (its arena would lack those experts)."""
+    import numpy as np
+
+    import oracle
+    from expert_ffn_token_b200 import synth
+    oracle.build()
+    used = oracle.set_threads(threads if threads else host_cores())
+    w = cs["w"]
+    x = cs["x0"]
+    t_total, layers, l = 0.0, 0, 0
+    while layers == 0 or t_total < seconds:
+        if l == len(cs["routers"]):     # the whole chain done: start again from x0
+            l, x = 0, cs["x0"]
+        buf, lay = synth.compact_arena(w, l, set(int(e) for e in cs["ids"][l].ravel()))
+        L = {"arena": buf, "experts": oracle.experts_table(lay.fmts, lay.offs, lay.strides),
+             "shared": -1, "hidden": w.hidden, "ffn": w.ffn, "router": cs["routers"][l],
+             "norm": cs["norm"]}
+        t0 = time.perf_counter()
+        x_next, ids = oracle.chain([L], x, w.k)
+        t_total += time.perf_counter() - t0
+        layers += 1
+        if not np.array_equal(ids[0], cs["ids"][l]):
+            break
+        x = x_next
+        l += 1
+    return {"value": layers * w.tokens / t_total, "unit": "tokens/s", "cores": used,
+            "kind": "oracle",
+            "sample": f"{layers} chained layer(s) x {w.tokens} token(s) (router, top-k, layer, "
+                      f"residual); {t_total:.1f} s on {used} thread(s) of {host_cpu()}"}
+
 
 
 def host_cores() -> int:
@@ -526,13 +721,22 @@ def main():
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
     torch.cuda.set_device(dev)
     names = ALL if args.workload == "all" else (args.workload,)
-    results = {n: run_workload(n, args, world, dev) for n in names}
+    results = {n: (run_chain if n == "chain" else run_workload)(n, args, world, dev)
+               for n in names}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         for n in names:
+            if n == "chain":
+                cs = results[n].pop("_chain_sample")
+                results[n]["cpu_baseline"] = chain_oracle_sample(cs, args.cpu_seconds)
+                results[n]["cpu_baseline_1_thread"] = chain_oracle_sample(cs, args.cpu_seconds / 2,
+                                                                          threads=1)
+                continue
             w = workload(n, args.layers)
             results[n]["cpu_baseline"] = oracle_sample(w, args.cpu_seconds)
             results[n]["cpu_baseline_1_thread"] = oracle_sample(w, args.cpu_seconds / 2,
                                                                 threads=1)
+    for r in results.values():
+        r.pop("_chain_sample", None)
     head_name = HEADLINE if HEADLINE in results else names[0]
     all_rows = []
     for r in results.values():
@@ -551,8 +755,8 @@ def main():
                    "shared_expert": head["shared_expert"], "ffn": head["ffn"],
                    "l2": head["l2"],
                    "parallelism": f"replicas x{world}" if world > 1 else "1 GPU"},
-        "expert_gbs": head["expert_gbs"], "int8_tops": head["int8_tops"],
-        "roofline": head["roofline"], "layer_roofline": head["layer_roofline"],
+        "expert_gbs": head["expert_gbs"], "int8_tops": head.get("int8_tops"),
+        "roofline": head["roofline"], "layer_roofline": head.get("layer_roofline"),
         "e2e": head["e2e"],
         "gpu_launches": sum(r["gpu_launches"] for r in results.values()),
         "clocks": Clocks.summary(all_rows if all_rows else None),

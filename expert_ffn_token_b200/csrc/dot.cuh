@@ -116,6 +116,66 @@ __device__ __forceinline__ float kq_part(uint4 hdr, uint4 qv, uint4 qh, int sb, 
     return kq_dot(w, hh, xa, xb, x.d[bl], x.d[bl + 1], x.s[bl], x.s[bl + 1]);
 }
 
+// ------------------------------------------------------------------ Q6_K
+//
+// A Q6_K super-block (210 B) starts 2-byte aligned inside a 16-byte-aligned row.  Lane part j
+// (c = j/2, hh = j%2; half h = c/2, c1 = c%2) covers, like the other K-quants, elements
+// 64c+16hh+[0,16) and 64c+32+16hh+[0,16).  The first sixteen take their low bits from nibble c1
+// of ql[64h+16hh+i], their high bits from bits 4c1, 4c1+1 of qh[32h+16hh+i] and scale
+// sc[8h+4c1+hh]; the second sixteen nibble c1 of ql[64h+32+16hh+i], bits 4c1+2, 4c1+3 of the
+// same qh bytes and scale sc[8h+4c1+2+hh].  The quants are kept as signed bytes q - 32, so the
+// dot of a 16-weight piece is d*sc*xd*sum((q-32)*qx) with no offset term.
+
+// 16 bytes at a 2-byte-aligned address (global or shared), as four little-endian words.
+__device__ __forceinline__ uint4 ld16_a2(const uint8_t *p) {
+    const uint16_t *h = reinterpret_cast<const uint16_t *>(p);
+    return make_uint4((uint32_t)h[0] | ((uint32_t)h[1] << 16), (uint32_t)h[2] | ((uint32_t)h[3] << 16),
+                      (uint32_t)h[4] | ((uint32_t)h[5] << 16), (uint32_t)h[6] | ((uint32_t)h[7] << 16));
+}
+
+// The quant words of one lane part: lo / hi = q - 32 of the two 16-weight pieces (signed bytes),
+// and the two pieces' scales d*sc (exact in fp32: 11 x 8 bits).
+struct Q6Lane {
+    uint32_t lo[4], hi[4];
+    float dl, dh;
+};
+
+__device__ __forceinline__ Q6Lane q6_unpack(const uint8_t *sbp, int j) {
+    const int c = j >> 1, hh = j & 1, h = c >> 1, c1 = c & 1;
+    const uint4 qa = ld16_a2(sbp + 64 * h + 16 * hh);
+    const uint4 qb = ld16_a2(sbp + 64 * h + 32 + 16 * hh);
+    const uint4 qh = ld16_a2(sbp + 128 + 32 * h + 16 * hh);
+    const float d = half_bits_to_float(*reinterpret_cast<const uint16_t *>(sbp + 208));
+    const int8_t *sc = reinterpret_cast<const int8_t *>(sbp + 192 + 8 * h + 4 * c1 + hh);
+    Q6Lane r;
+    r.dl = d * (float)sc[0];
+    r.dh = d * (float)sc[2];
+    const uint32_t a[4] = {qa.x, qa.y, qa.z, qa.w}, b[4] = {qb.x, qb.y, qb.z, qb.w};
+    const uint32_t hb[4] = {qh.x, qh.y, qh.z, qh.w};
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+        const uint32_t lo6 = ((a[i] >> (4 * c1)) & 0x0F0F0F0Fu) | (((hb[i] >> (4 * c1)) & 0x03030303u) << 4);
+        const uint32_t hi6 = ((b[i] >> (4 * c1)) & 0x0F0F0F0Fu) | (((hb[i] >> (4 * c1 + 2)) & 0x03030303u) << 4);
+        r.lo[i] = __vsub4(lo6, 0x20202020u);
+        r.hi[i] = __vsub4(hi6, 0x20202020u);
+    }
+    return r;
+}
+
+// The lane part's share of sum_k w_k * xhat_k (xa, xb: the activation bytes of the two pieces,
+// xdl / xdh: the Q8_1 scales of their 32-blocks 2c and 2c+1).
+__device__ __forceinline__ float q6_dot(const Q6Lane &w, int4 xa, int4 xb, float xdl, float xdh) {
+    int il = __dp4a((int)w.lo[0], xa.x, 0);
+    il = __dp4a((int)w.lo[1], xa.y, il);
+    il = __dp4a((int)w.lo[2], xa.z, il);
+    il = __dp4a((int)w.lo[3], xa.w, il);
+    int ih = __dp4a((int)w.hi[0], xb.x, 0);
+    ih = __dp4a((int)w.hi[1], xb.y, ih);
+    ih = __dp4a((int)w.hi[2], xb.z, ih);
+    ih = __dp4a((int)w.hi[3], xb.w, ih);
+    return w.dl * xdl * (float)il + w.dh * xdh * (float)ih;
+}
+
 // Q8_0 block b of a row (34-byte blocks, 2-byte aligned): its 32 quants as 8 words and d.
 struct Q80Block {
     uint32_t w[8];
@@ -217,6 +277,20 @@ __device__ __forceinline__ void row_parts(const uint8_t *row, int K, const ActRo
         }
         return;
     }
+    if (FMT == MOE_FMT_Q6_K) {
+        const int j = lane & 7, c = j >> 1, hh = j & 1;
+        for (int sb = lane >> 3; sb < K / 256; sb += 4) {
+            const Q6Lane w = q6_unpack(row + (size_t)sb * kQ6KBytes, j);
+            const int kl = sb * 256 + c * 64 + hh * 16, bl = sb * 8 + 2 * c;
+#pragma unroll
+            for (int t = 0; t < NT; t++)
+                if (t < nt)
+                    acc[t] += q6_dot(w, *reinterpret_cast<const int4 *>(x[t].q + kl),
+                                     *reinterpret_cast<const int4 *>(x[t].q + kl + 32),
+                                     x[t].d[bl], x[t].d[bl + 1]);
+        }
+        return;
+    }
     constexpr int SBB = FMT == MOE_FMT_Q5_K ? kQ5KBytes : kQ4KBytes;
     constexpr int QS = FMT == MOE_FMT_Q5_K ? 48 : 16;
     const int nsb = K / 256;
@@ -253,6 +327,7 @@ __device__ __forceinline__ void row_parts_fmt(int fmt, const uint8_t *row, int K
     if (fmt == MOE_FMT_Q4_K) row_parts<MOE_FMT_Q4_K, NT>(row, K, x, nt, acc);
     else if (fmt == MOE_FMT_Q5_K) row_parts<MOE_FMT_Q5_K, NT>(row, K, x, nt, acc);
     else if (fmt == MOE_FMT_Q8_0) row_parts<MOE_FMT_Q8_0, NT>(row, K, x, nt, acc);
+    else if (fmt == MOE_FMT_Q6_K) row_parts<MOE_FMT_Q6_K, NT>(row, K, x, nt, acc);
     else row_parts<MOE_FMT_Q5_1, NT>(row, K, x, nt, acc);
 }
 

@@ -61,6 +61,7 @@ struct DecParams {
     const float *x;
     const float *logits;
     float *out;
+    const float *gate;     // optional [T]: the shared expert's weight per token (else 1)
     uint8_t *ws;
     WsLayout L;
     int T, H, F, E, k, shared, hpad;
@@ -169,6 +170,23 @@ __device__ __forceinline__ WChunk kq_chunk(const uint8_t *sbp, int j) {
     return w;
 }
 
+// A Q6_K chunk (super-block at a 2-byte-aligned address in shared memory): the signed bytes
+// q - 32 of its two 16-weight pieces and their scales d*sc; no min term (ml = mh = 0), so
+// kq_chunk_dot applies unchanged.
+__device__ __forceinline__ WChunk q6_chunk(const uint8_t *sbp, int j) {
+    const Q6Lane q = q6_unpack(sbp, j);
+    WChunk w;
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+        w.lo[i] = q.lo[i];
+        w.hi[i] = q.hi[i];
+    }
+    w.dl = q.dl;
+    w.dh = q.dh;
+    w.ml = w.mh = 0.f;
+    return w;
+}
+
 // Lane share of sum_k w_k * xhat_k over one chunk.  `mf` is 1 on the lane that adds the two
 // sub-blocks' min terms (hh == 0) and 0 on its partner.
 __device__ __forceinline__ float kq_chunk_dot(const WChunk &w, const ActChunk &a, float mf) {
@@ -236,6 +254,7 @@ __device__ __forceinline__ void rows_dot(int fmt_rt, const uint8_t *const (&rows
     const int nchunk = K / 32;
     const int fmt = FK == FK_Q4K ? MOE_FMT_Q4_K : FK == FK_Q5K ? MOE_FMT_Q5_K : fmt_rt;
     const bool q80 = fmt == MOE_FMT_Q8_0, q51 = fmt == MOE_FMT_Q5_1, q5 = fmt == MOE_FMT_Q5_K;
+    const bool q6 = fmt == MOE_FMT_Q6_K;
     const bool small = q80 || q51;
     const int SBB = q5 ? kQ5KBytes : kQ4KBytes;
 #pragma unroll 2
@@ -265,7 +284,8 @@ __device__ __forceinline__ void rows_dot(int fmt_rt, const uint8_t *const (&rows
             } else {
                 const WChunk w = (FK == FK_Q5K || (FK == FK_ANY && q5))
                                      ? kq_chunk<true>(row + (size_t)sb * SBB, j)
-                                     : kq_chunk<false>(row + (size_t)sb * SBB, j);
+                                 : (FK == FK_ANY && q6) ? q6_chunk(row + (size_t)sb * kQ6KBytes, j)
+                                                        : kq_chunk<false>(row + (size_t)sb * SBB, j);
 #pragma unroll
                 for (int t = 0; t < NT; t++) {
                     if (t < n) {
@@ -509,7 +529,7 @@ __device__ __forceinline__ void prologue(const DecParams &P, Ctx &C, uint8_t *sm
                     J.shared = 1;
                 }
                 C.s_stok[k] = 0;
-                C.s_sw[k] = 1.0f;
+                C.s_sw[k] = P.gate ? P.gate[0] : 1.0f;
                 C.s_misc[0] = U;
             }
             __syncwarp();
@@ -642,7 +662,7 @@ __device__ __forceinline__ void prologue(const DecParams &P, Ctx &C, uint8_t *sm
 #pragma unroll 1
     for (int t = tid; t < T; t += kThreads) {
         C.s_stok[A + t] = t;
-        C.s_sw[A + t] = 1.0f;
+        C.s_sw[A + t] = P.gate ? P.gate[t] : 1.0f;
     }
     bool desc_ok = true;
     if (tid < U && !ptx::mbar_wait_bounded(C.desc_bar, 0, desc_wait_ns(P))) {
@@ -939,7 +959,9 @@ __device__ __forceinline__ void down_stage(const DecParams &P, const Ctx &C, con
                     const int SBB = fmt == MOE_FMT_Q5_K ? kQ5KBytes : kQ4KBytes;
                     const int sb = p >> 3, j = p & 7;
                     const WChunk w = fmt == MOE_FMT_Q5_K ? kq_chunk<true>(row + (size_t)sb * SBB, j)
-                                                         : kq_chunk<false>(row + (size_t)sb * SBB, j);
+                                     : (FK == FK_ANY && fmt == MOE_FMT_Q6_K)
+                                         ? q6_chunk(row + (size_t)sb * kQ6KBytes, j)
+                                         : kq_chunk<false>(row + (size_t)sb * SBB, j);
                     const float mf = (j & 1) ? 0.f : 1.f;
 #pragma unroll 1
                     for (int t = 0; t < J.n; t++) {
@@ -1205,6 +1227,7 @@ cudaError_t launch_decode_fused(const FfnArgs &a, int E, int shared, const float
     P.x = x;
     P.logits = logits;
     P.out = a.out;
+    P.gate = a.gate;
     P.ws = ws;
     P.L = L;
     P.T = a.T;

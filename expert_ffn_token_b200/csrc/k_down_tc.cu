@@ -379,7 +379,7 @@ __device__ void role_loader(const GemmArgs &a, const Smem &S, int nj) {
                 float wt;
                 if (t.shared) {
                     tok = slot - a.T * a.k;
-                    wt = 1.0f;
+                    wt = a.gate ? a.gate[tok] : 1.0f;
                 } else {
                     const int p = a.perm[slot];
                     tok = p / a.k;
@@ -747,6 +747,7 @@ bool tc_build_weight_maps(const uint8_t *d_base, const moe_expert_desc *descs, i
     CUtensorMap *maps = reinterpret_cast<CUtensorMap *>(out.data());
     for (int e = 0; e < n; e++) {
         const moe_expert_desc &d = descs[e];
+        if (d.fmt == MOE_FMT_Q6_K) return false;   // no exact fp16 operand form
         for (int t = 0; t < 3; t++) {
             const int rows = t < 2 ? F : H;
             const int width = t < 2 ? H : F;
@@ -810,6 +811,7 @@ cudaError_t launch_gemm_tc(const TcPhaseArgs &p, cudaStream_t st) {
     a.lag = a.DB - 1;
     a.rawb = raw_bytes(f.fmt_mask);
     a.out = f.out;
+    a.gate = f.gate;
     a.y = f.y;
     a.status = f.status;
     a.wait_ns = p.wait_ns;

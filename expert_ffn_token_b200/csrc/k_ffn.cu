@@ -162,7 +162,7 @@ __global__ void __launch_bounds__(256) k_down_decode(FfnArgs a) {
     }
     for (int t = threadIdx.x; t < a.T; t += blockDim.x) {
         s_tok[a.T * a.k + t] = t;
-        s_w[a.T * a.k + t] = 1.0f;
+        s_w[a.T * a.k + t] = a.gate ? a.gate[t] : 1.0f;
     }
     __syncthreads();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -209,9 +209,31 @@ __global__ void __launch_bounds__(256) k_down_decode(FfnArgs a) {
             }
             continue;
         }
-        const bool q5 = ex.fmt == MOE_FMT_Q5_K;
         const int nsb = (a.F + 255) / 256;
         const int j = lane & 7, c = j >> 1, hh = j & 1;
+        if (ex.fmt == MOE_FMT_Q6_K) {
+            for (int sb = lane >> 3; sb < nsb; sb += 4) {
+                const Q6Lane w = q6_unpack(row + (size_t)sb * kQ6KBytes, j);
+                const int kl = sb * 256 + c * 64 + hh * 16;
+                const int bl = sb * 8 + 2 * c;
+                for (int s = 0; s < job.n; s++) {
+                    const int slot = job.slot0 + s;
+                    const int8_t *hq = a.hq + (size_t)slot * a.hpad;
+                    const size_t hbase = (size_t)slot * hb + bl;
+                    const float v = q6_dot(w, *reinterpret_cast<const int4 *>(hq + kl),
+                                           *reinterpret_cast<const int4 *>(hq + kl + 32),
+                                           half_bits_to_float(a.hd[hbase]),
+                                           half_bits_to_float(a.hd[hbase + 1]));
+                    const int t = s_tok[slot];
+                    const float wv = s_w[slot] * v;
+#pragma unroll
+                    for (int tt = 0; tt < NT; tt++)
+                        if (tt == t) acc[tt] += wv;
+                }
+            }
+            continue;
+        }
+        const bool q5 = ex.fmt == MOE_FMT_Q5_K;
         const int SBB = q5 ? kQ5KBytes : kQ4KBytes;
         for (int sb = lane >> 3; sb < nsb; sb += 4) {
             const uint8_t *p = row + (size_t)sb * SBB;
@@ -294,7 +316,7 @@ __global__ void __launch_bounds__(256) k_down_grouped(FfnArgs a, int determinist
             if ((int)threadIdx.x < nt) {
                 if (job.shared) {
                     t = c0 + threadIdx.x;
-                    wv = 1.0f;
+                    wv = a.gate ? a.gate[t] : 1.0f;
                 } else {
                     const int p = a.perm[slot];
                     t = p / a.k;
@@ -369,7 +391,7 @@ __global__ void k_combine(FfnArgs a, int shared) {
             const int p = t * a.k + j;
             acc = fmaf(a.w[p], a.y[(size_t)a.inv_perm[p] * a.H + i], acc);
         }
-        if (shared) acc += a.y[((size_t)a.T * a.k + t) * a.H + i];
+        if (shared) acc = fmaf(a.gate ? a.gate[t] : 1.0f, a.y[((size_t)a.T * a.k + t) * a.H + i], acc);
         a.out[(size_t)t * a.H + i] = acc;
     }
 }
@@ -384,7 +406,8 @@ cudaError_t launch_combine(const FfnArgs &a, bool shared, cudaStream_t st) {
 // ------------------------------------------------------------------ debug dequant export
 
 // One thread per weight: RN32(RN32(d*sc)*q - RN32(dmin*m)) (K-quants), d*q (Q8_0),
-// RN32(d*q + m) (Q5_1; d*q is exact in fp32, so the fused multiply-add rounds once).
+// RN32(d*q + m) (Q5_1; d*q is exact in fp32, so the fused multiply-add rounds once),
+// RN32(RN32(d*sc)*(q - 32)) (Q6_K; d*sc is exact).
 __global__ void k_dequant(const uint8_t *__restrict__ m, int fmt, int rows, int nblocks,
                           int stride, float *out) {
     const int bw = block_weights(fmt), bb = block_bytes(fmt);
@@ -398,7 +421,14 @@ __global__ void k_dequant(const uint8_t *__restrict__ m, int fmt, int rows, int 
         const uint8_t *p = m + r * stride + (int64_t)b * bb;
         const uint32_t d16 = p[0] | (p[1] << 8);
         float w;
-        if (fmt == MOE_FMT_Q8_0) {
+        if (fmt == MOE_FMT_Q6_K) {
+            const int h = n / 128, i = n % 128, g = i / 32, l = i % 32;
+            const int lo = (p[64 * h + l + 32 * (g & 1)] >> (g < 2 ? 0 : 4)) & 15;
+            const int hi = (p[128 + 32 * h + l] >> (2 * g)) & 3;
+            const int sc = (int8_t)p[192 + 8 * h + 2 * g + l / 16];
+            const float d1 = __fmul_rn(half_bits_to_float(p[208] | (p[209] << 8)), (float)sc);
+            w = __fmul_rn(d1, (float)(lo + 16 * hi - 32));
+        } else if (fmt == MOE_FMT_Q8_0) {
             w = __fmul_rn(half_bits_to_float(d16), (float)(int8_t)p[2 + n]);
         } else if (fmt == MOE_FMT_Q5_1) {
             const uint32_t m16 = p[2] | (p[3] << 8);

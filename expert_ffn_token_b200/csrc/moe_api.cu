@@ -158,7 +158,7 @@ moe_status moe_arena_create(const void *d_arena, size_t arena_bytes, int hidden,
     uint64_t ms01 = 0, ms2 = 0;
     for (int e = 0; e < n; e++) {
         const moe_expert_desc &d = host_descs[e];
-        if (d.fmt < 0 || d.fmt > MOE_FMT_Q5_1 || d.reserved != 0) return MOE_ERR_INVALID_ARG;
+        if (d.fmt < 0 || d.fmt > MOE_FMT_Q6_K || d.reserved != 0) return MOE_ERR_INVALID_ARG;
         const int bw = block_weights(d.fmt), bb = block_bytes(d.fmt);
         if (hidden % bw) return MOE_ERR_UNSUPPORTED;
         const int rows[3] = {ffn, ffn, hidden};
@@ -209,6 +209,7 @@ moe_status moe_arena_create(const void *d_arena, size_t arena_bytes, int hidden,
         const bool fits = cudaGetDevice(&dev_id) == cudaSuccess &&
                           cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin,
                                                  dev_id) == cudaSuccess &&
+                          !(fmt_mask & (1 << MOE_FMT_Q6_K)) &&
                           tc_smem_bytes(fmt_mask) <= (size_t)optin && ffn % 64 == 0;
         if (fits && tc_build_weight_maps(A->base, host_descs, n, hidden, ffn, maps)) {
             if (cudaMalloc(&A->d_wmaps, maps.size()) != cudaSuccess ||
@@ -334,16 +335,30 @@ moe_status moe_read_status(uint32_t *d_status_word, void *stream, int clear,
     return MOE_OK;
 }
 
-moe_status moe_forward(const moe_arena *arena, const float *d_x, const float *d_logits, int T,
-                       int k, float *d_out, void *d_ws, size_t ws_bytes, uint32_t flags,
-                       void *stream) {
+}  // extern "C"
+
+namespace moe {
+
+// Every host-side check of moe_forward, in its order.
+static moe_status forward_checks(const moe_arena *arena, const float *d_x, const float *d_logits,
+                                 int T, int k, const float *d_out, const void *d_ws,
+                                 size_t ws_bytes, uint32_t flags) {
     const moe_status chk = check_forward_args(arena, d_x, d_logits, T, k, d_out, flags);
     if (chk != MOE_OK) return chk;
     if (!d_ws) return MOE_ERR_INVALID_ARG;
     if (!aligned(d_ws, 256)) return MOE_ERR_ALIGNMENT;
     if ((flags & MOE_F_FORCE_PREFILL) && !arena->tc_ok) return MOE_ERR_UNSUPPORTED;
+    if (ws_bytes < ws_layout(arena, T, k, flags).total) return MOE_ERR_WORKSPACE;
+    return MOE_OK;
+}
+
+// moe_forward with an optional per-token weight of the shared expert's output (d_gate [T]).
+static moe_status forward_impl(const moe_arena *arena, const float *d_x, const float *d_logits,
+                               const float *d_gate, int T, int k, float *d_out, void *d_ws,
+                               size_t ws_bytes, uint32_t flags, void *stream) {
+    const moe_status chk = forward_checks(arena, d_x, d_logits, T, k, d_out, d_ws, ws_bytes, flags);
+    if (chk != MOE_OK) return chk;
     const WsLayout L = ws_layout(arena, T, k, flags);
-    if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
     cudaStream_t st = (cudaStream_t)stream;
     uint8_t *ws = static_cast<uint8_t *>(d_ws);
     const int H = arena->H, E = arena->E;
@@ -380,6 +395,7 @@ moe_status moe_forward(const moe_arena *arena, const float *d_x, const float *d_
         a.max_stride01 = arena->max_stride01;
         a.max_stride2 = arena->max_stride2;
         a.h = (flags & MOE_F_KEEP_H) ? reinterpret_cast<float *>(ws + L.h) : nullptr;
+        a.gate = d_gate;
         a.wait_ns = arena->wait_ns;
         bool taken = false;
         cudaError_t e = launch_decode_fused(a, E, shared, d_x, d_logits, ws, L, L.sync, L.blkcnt,
@@ -433,6 +449,7 @@ moe_status moe_forward(const moe_arena *arena, const float *d_x, const float *d_
     a.h = reinterpret_cast<float *>(ws + L.h);
     a.y = (flags & MOE_F_DETERMINISTIC) ? reinterpret_cast<float *>(ws + L.y) : nullptr;
     a.out = d_out;
+    a.gate = d_gate;
     a.status = status;
     a.T = T;
     a.k = k;
@@ -502,6 +519,17 @@ moe_status moe_forward(const moe_arena *arena, const float *d_x, const float *d_
     return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
+}  // namespace moe
+
+extern "C" {
+
+moe_status moe_forward(const moe_arena *arena, const float *d_x, const float *d_logits, int T,
+                       int k, float *d_out, void *d_ws, size_t ws_bytes, uint32_t flags,
+                       void *stream) {
+    return forward_impl(arena, d_x, d_logits, nullptr, T, k, d_out, d_ws, ws_bytes,
+                        flags & ~MOE_F_LOOKAHEAD, stream);
+}
+
 moe_status moe_set_timing_events(moe_arena *arena, void *ev_begin, void *ev_mid, void *ev_end) {
     if (!arena) return MOE_ERR_INVALID_ARG;
     if ((ev_begin == nullptr) != (ev_mid == nullptr) || (ev_mid == nullptr) != (ev_end == nullptr))
@@ -530,6 +558,202 @@ moe_status moe_debug_dequant(const moe_arena *arena, int expert, int which, floa
     if (launch_dequant(arena->base + d.off[which], d.fmt, rows, nb, (int)d.stride[which], d_out,
                        (cudaStream_t)stream) != cudaSuccess)
         return MOE_ERR_CUDA;
+    return MOE_OK;
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------------------ router in front, chains
+
+namespace moe {
+
+// Host checks of one layer's router and gate rows.
+static moe_status check_router_rows(const moe_arena *arena, const float *d_router,
+                                    const float *d_gate_row) {
+    if (!d_router) return MOE_ERR_INVALID_ARG;
+    if (d_gate_row && arena->shared < 0) return MOE_ERR_INVALID_ARG;
+    if (arena->H % 4) return MOE_ERR_INVALID_ARG;
+    if (!aligned(d_router, 16) || (d_gate_row && !aligned(d_gate_row, 16))) return MOE_ERR_ALIGNMENT;
+    return MOE_OK;
+}
+
+// A chain workspace: the largest layer workspace, then the chain's own buffers.
+struct ChainLayout {
+    size_t fwd, xa, xb, xn, out, logits, next, gate, total;
+    int H, Emax;
+};
+
+static moe_status chain_layout(const moe_chain_layer *ls, int n, int T, int k, uint32_t flags,
+                               ChainLayout &C) {
+    if (!ls || n <= 0 || T <= 0 || k <= 0 || k > kMaxK) return MOE_ERR_INVALID_ARG;
+    if ((flags & MOE_F_LOOKAHEAD) && T > kDecodeMaxT) return MOE_ERR_INVALID_ARG;
+    if ((T + 15) / 16 > 65535) return MOE_ERR_UNSUPPORTED;
+    C = ChainLayout{};
+    const uint32_t ff = flags & ~MOE_F_LOOKAHEAD;
+    for (int l = 0; l < n; l++) {
+        const moe_arena *A = ls[l].arena;
+        if (!A || k > A->E) return MOE_ERR_INVALID_ARG;
+        if (l == 0) C.H = A->H;
+        if (A->H != C.H) return MOE_ERR_INVALID_ARG;
+        const moe_status r = check_router_rows(A, ls[l].d_router, ls[l].d_gate_row);
+        if (r != MOE_OK) return r;
+        if (ls[l].d_norm_weight && !aligned(ls[l].d_norm_weight, 16)) return MOE_ERR_ALIGNMENT;
+        if ((ff & MOE_F_FORCE_PREFILL) && !A->tc_ok) return MOE_ERR_UNSUPPORTED;
+        C.fwd = std::max(C.fwd, ws_layout(A, T, k, ff).total);
+        C.Emax = std::max(C.Emax, A->E);
+    }
+    if ((flags & MOE_F_LOOKAHEAD) && lookahead_smem_bytes(C.Emax) > 200 * 1024)
+        return MOE_ERR_UNSUPPORTED;
+    size_t p = align256(C.fwd);
+    auto take = [&](size_t bytes) {
+        const size_t o = p;
+        p = align256(p + bytes);
+        return o;
+    };
+    const size_t xb = (size_t)T * C.H * 4;
+    C.xa = take(xb);
+    C.xb = take(xb);
+    C.xn = take(xb);
+    C.out = take(xb);
+    C.logits = take((size_t)T * C.Emax * 4);
+    C.next = take((size_t)T * C.Emax * 4);
+    C.gate = take((size_t)T * 4);
+    C.total = p;
+    return MOE_OK;
+}
+
+}  // namespace moe
+
+extern "C" {
+
+moe_status moe_forward_routed(const moe_arena *arena, const float *d_x, int T, int k,
+                              const float *d_router, const float *d_gate_row, float *d_logits,
+                              float *d_gate, float *d_out, void *d_ws, size_t ws_bytes,
+                              uint32_t flags, void *stream) {
+    flags &= ~MOE_F_LOOKAHEAD;
+    moe_status r = forward_checks(arena, d_x, d_logits, T, k, d_out, d_ws, ws_bytes, flags);
+    if (r != MOE_OK) return r;
+    if ((r = check_router_rows(arena, d_router, d_gate_row)) != MOE_OK) return r;
+    if (d_gate_row && !d_gate) return MOE_ERR_INVALID_ARG;
+    if (d_gate && !aligned(d_gate, 4)) return MOE_ERR_ALIGNMENT;
+    if ((T + 15) / 16 > 65535) return MOE_ERR_UNSUPPORTED;
+    cudaStream_t st = (cudaStream_t)stream;
+    RouterRowsArgs a{};
+    a.x = d_x;
+    a.Wr = d_router;
+    a.E = arena->E;
+    a.logits = d_logits;
+    a.wg = d_gate_row;
+    a.gate = d_gate_row ? d_gate : nullptr;
+    a.T = T;
+    a.H = arena->H;
+    if (launch_router_rows(a, st) != cudaSuccess) return MOE_ERR_CUDA;
+    return forward_impl(arena, d_x, d_logits, a.gate, T, k, d_out, d_ws, ws_bytes, flags, stream);
+}
+
+moe_status moe_chain_workspace_size(const moe_chain_layer *host_layers, int n_layers,
+                                    int max_tokens, int k, uint32_t flags, size_t *bytes) {
+    if (!bytes) return MOE_ERR_INVALID_ARG;
+    ChainLayout C;
+    const moe_status r = chain_layout(host_layers, n_layers, max_tokens, k, flags, C);
+    if (r != MOE_OK) return r;
+    *bytes = C.total;
+    return MOE_OK;
+}
+
+moe_status moe_chain_status(const moe_chain_layer *host_layers, int n_layers, void *d_ws, int T,
+                            int k, uint32_t flags, uint32_t **d_status_word) {
+    if (!d_ws || !d_status_word) return MOE_ERR_INVALID_ARG;
+    ChainLayout C;
+    const moe_status r = chain_layout(host_layers, n_layers, T, k, flags, C);
+    if (r != MOE_OK) return r;
+    // every layer's workspace layout starts with the status word
+    *d_status_word = reinterpret_cast<uint32_t *>(
+        static_cast<uint8_t *>(d_ws) + ws_layout(host_layers[0].arena, T, k, flags).status);
+    return MOE_OK;
+}
+
+moe_status moe_chain_forward(const moe_chain_layer *host_layers, int n_layers, const float *d_x,
+                             int T, int k, float *d_x_out, void *d_ws, size_t ws_bytes,
+                             uint32_t flags, const moe_chain_trace *host_trace, void *stream) {
+    ChainLayout C;
+    moe_status r = chain_layout(host_layers, n_layers, T, k, flags, C);
+    if (r != MOE_OK) return r;
+    if (!d_x || !d_x_out || !d_ws) return MOE_ERR_INVALID_ARG;
+    if (!aligned(d_x, 16) || !aligned(d_x_out, 16) || !aligned(d_ws, 256)) return MOE_ERR_ALIGNMENT;
+    if (ws_bytes < C.total) return MOE_ERR_WORKSPACE;
+    const moe_chain_trace tr = host_trace ? *host_trace : moe_chain_trace{};
+    const bool look = (flags & MOE_F_LOOKAHEAD) != 0;
+    const uint32_t ff = flags & ~MOE_F_LOOKAHEAD;
+    cudaStream_t st = (cudaStream_t)stream;
+    uint8_t *ws = static_cast<uint8_t *>(d_ws);
+    float *xbuf[2] = {reinterpret_cast<float *>(ws + C.xa), reinterpret_cast<float *>(ws + C.xb)};
+    float *xn = reinterpret_cast<float *>(ws + C.xn);
+    float *out = reinterpret_cast<float *>(ws + C.out);
+    float *logits = reinterpret_cast<float *>(ws + C.logits);
+    float *next = reinterpret_cast<float *>(ws + C.next);
+    float *gate = reinterpret_cast<float *>(ws + C.gate);
+    const int H = C.H;
+    const size_t xbytes = (size_t)T * H * 4;
+    auto copy = [&](void *dst, const void *src, size_t bytes) {
+        return cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToDevice, st) == cudaSuccess;
+    };
+    const float *x = d_x;   // x_l
+    for (int l = 0; l < n_layers; l++) {
+        const moe_chain_layer &Ly = host_layers[l];
+        const moe_arena *A = Ly.arena;
+        const bool ahead = look && l + 1 < n_layers;
+        RouterRowsArgs a{};
+        if (l == 0) {
+            a.x = d_x;
+        } else {   // x_l = x_{l-1} + out_{l-1}, formed and written by the router pass
+            a.x = x;
+            a.res = out;
+            a.x_out = xbuf[l & 1];
+        }
+        a.norm = 1;   // the layer reads RMSNorm(x_l), written to xn
+        a.eps = MOE_CHAIN_RMS_EPS;
+        a.gamma = Ly.d_norm_weight;
+        a.xn_out = xn;
+        a.Wr = Ly.d_router;
+        a.E = A->E;
+        a.logits = logits;
+        if (ahead) {
+            a.Wn = host_layers[l + 1].d_router;
+            a.En = host_layers[l + 1].arena->E;
+            a.logits_next = next;
+        }
+        a.wg = Ly.d_gate_row;
+        a.gate = Ly.d_gate_row ? gate : nullptr;
+        a.T = T;
+        a.H = H;
+        if (launch_router_rows(a, st) != cudaSuccess) return MOE_ERR_CUDA;
+        if (l > 0) x = xbuf[l & 1];
+        if (ahead) {
+            const moe_arena *B = host_layers[l + 1].arena;
+            int32_t *early = tr.early ? tr.early + (size_t)(l + 1) * T * k : nullptr;
+            if (launch_lookahead(next, T, B->E, k, B->shared >= 0 ? 1 : 0, B->d_experts, B->H,
+                                 B->F, early, st) != cudaSuccess)
+                return MOE_ERR_CUDA;
+        }
+        r = forward_impl(A, xn, logits, a.gate, T, k, out, d_ws, C.fwd, ff, stream);
+        if (r != MOE_OK) return r;
+        const WsLayout L = ws_layout(A, T, k, ff);
+        bool ok = true;
+        if (tr.x) ok = ok && copy(tr.x + (size_t)l * T * H, x, xbytes);
+        if (tr.xn) ok = ok && copy(tr.xn + (size_t)l * T * H, xn, xbytes);
+        if (tr.logits)
+            for (int t = 0; t < T && ok; t++)
+                ok = copy(tr.logits + ((size_t)l * T + t) * C.Emax, logits + (size_t)t * A->E,
+                          (size_t)A->E * 4);
+        if (tr.ids) ok = ok && copy(tr.ids + (size_t)l * T * k, ws + L.ids, (size_t)T * k * 4);
+        if (tr.w) ok = ok && copy(tr.w + (size_t)l * T * k, ws + L.w, (size_t)T * k * 4);
+        if (tr.gate && Ly.d_gate_row) ok = ok && copy(tr.gate + (size_t)l * T, gate, (size_t)T * 4);
+        if (tr.out) ok = ok && copy(tr.out + (size_t)l * T * H, out, xbytes);
+        if (!ok) return MOE_ERR_CUDA;
+    }
+    if (launch_residual(x, out, d_x_out, T, H, st) != cudaSuccess) return MOE_ERR_CUDA;
+    if (tr.x && !copy(tr.x + (size_t)n_layers * T * H, d_x_out, xbytes)) return MOE_ERR_CUDA;
     return MOE_OK;
 }
 

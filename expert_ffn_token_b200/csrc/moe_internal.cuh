@@ -9,6 +9,10 @@
 //   Q8_0 34 B / 32 weights: fp16 d, int8 q[32].
 //   Q5_1 24 B / 32 weights: fp16 d, fp16 m, uint32 qh (bit n: fifth bit of element n),
 //        qs[16]: byte i holds element i (low nibble) and element 16+i (high nibble); w = d*q + m.
+//   Q6_K 210 B / 256 weights: ql[128] low 4 bits, qh[64] high 2 bits, int8 sc[16] (one per 16
+//        weights), fp16 d at 208; element n (h = n/128, i = n%128, g = i/32, l = i%32): low bits
+//        = nibble (g >= 2) of ql[64h + l + 32(g&1)], high bits = bits 2g, 2g+1 of qh[32h + l],
+//        w = d*sc[8h + 2g + l/16]*(q - 32).
 //   Q8_1 (activations, stored SoA): per 32 values int8 q[32], fp16 d, fp16 s = d * sum(q).
 #pragma once
 
@@ -32,6 +36,7 @@ constexpr int kQ4KBytes = 144;
 constexpr int kQ5KBytes = 176;
 constexpr int kQ80Bytes = 34;
 constexpr int kQ51Bytes = 24;
+constexpr int kQ6KBytes = 210;
 constexpr int kMaxK = 32;         // routed experts per token
 constexpr int kMaxE = 4096;       // experts per layer
 constexpr int kDecodeMaxT = 16;   // largest batch the dequant-GEMV path takes by default
@@ -46,6 +51,7 @@ __host__ __device__ inline int block_bytes(int fmt) {
     return fmt == MOE_FMT_Q4_K   ? kQ4KBytes
            : fmt == MOE_FMT_Q5_K ? kQ5KBytes
            : fmt == MOE_FMT_Q8_0 ? kQ80Bytes
+           : fmt == MOE_FMT_Q6_K ? kQ6KBytes
                                  : kQ51Bytes;
 }
 
@@ -64,7 +70,7 @@ struct Job {
     int32_t expert;
     int32_t slot0;
     int32_t n;
-    int32_t shared;           // 1 for the shared expert (slot i is token i, weight 1)
+    int32_t shared;           // 1 for the shared expert (slot i is token i, weight gate[i] or 1)
 };
 
 struct moe_arena_impl;
@@ -162,6 +168,7 @@ struct FfnArgs {
     float *h;              // optional fp32 h
     float *y;              // deterministic prefill: y per slot
     float *out;
+    const float *gate;     // optional [T]: weight of the shared expert's output (else 1)
     uint32_t *status;
     int T, k, H, F, hpad, max_jobs, fmt_mask;
     int max_stride01, max_stride2;   // largest gate/up and down row strides in the arena
@@ -218,6 +225,38 @@ cudaError_t launch_quant_rows(const float *x, int T, int H, int8_t *xq, uint16_t
 // The down operand of every used slot from its Q8_1(h) blocks.
 cudaError_t launch_h_rows(const int8_t *hq, const uint16_t *hd, int slots, int F, int hpad, int Kd,
                           __half *hh, float *hscale, cudaStream_t st);
+
+// ---- router, shared gate, lookahead (k_router.cu)
+
+// One pass over the hidden state for up to three sets of fp32 rows [*][H]: router rows Wr [E]
+// -> logits [T][E], lookahead rows Wn [En] -> logits_next [T][En], gate row wg -> gate [T].
+// With res, the hidden state is x + res (fp32), also written to x_out when x_out is set.  With
+// norm, the rows dotted are the hidden state times 1 / sqrt(mean square + eps), then times gamma
+// [H] when given, also written to xn_out when xn_out is set.
+struct RouterRowsArgs {
+    const float *x, *res;
+    float *x_out;
+    int norm;
+    float eps;
+    const float *gamma;
+    float *xn_out;
+    const float *Wr;
+    float *logits;
+    const float *Wn;
+    float *logits_next;
+    const float *wg;
+    float *gate;
+    int E, En, T, H;
+};
+cudaError_t launch_router_rows(const RouterRowsArgs &a, cudaStream_t st);
+// Top-k of logits [T][E] (T <= 16) and an L2 prefetch of the chosen experts' packed matrices
+// and the shared expert's; ids_out [T][k] may be null.
+size_t lookahead_smem_bytes(int E);
+cudaError_t launch_lookahead(const float *logits, int T, int E, int k, int shared,
+                             const ExpertDev *experts, int H, int F, int32_t *ids_out,
+                             cudaStream_t st);
+cudaError_t launch_residual(const float *x, const float *res, float *x_out, int T, int H,
+                            cudaStream_t st);
 
 cudaError_t launch_dequant(const uint8_t *m, int fmt, int rows, int nblocks, int stride,
                            float *out, cudaStream_t st);

@@ -44,6 +44,7 @@ struct GemmArgs {
     float *h;
     // down outputs
     float *out;
+    const float *gate;            // optional [T]: the shared expert's weight per token
     float *y;                     // deterministic mode: y per slot
     uint32_t *status;
     uint64_t wait_ns;

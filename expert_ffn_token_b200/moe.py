@@ -23,18 +23,21 @@ OK = 0
 ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_ALIGNMENT, ERR_CUDA = 1, 2, 3, 4
 ERR_NONFINITE, ERR_BOUNDS, ERR_TIMEOUT, ERR_WORKSPACE = 5, 6, 7, 8
 
-FMT_Q4_K, FMT_Q5_K, FMT_Q8_0, FMT_Q5_1 = 0, 1, 2, 3
+FMT_Q4_K, FMT_Q5_K, FMT_Q8_0, FMT_Q5_1, FMT_Q6_K = 0, 1, 2, 3, 4
 
 F_DETERMINISTIC = 1
 F_FORCE_DECODE = 2
 F_FORCE_PREFILL = 4
 F_KEEP_H = 8
+F_LOOKAHEAD = 16
 
 EXPORTED = ["moe_arena_create", "moe_arena_destroy", "moe_workspace_size", "moe_quantize_act",
             "moe_route_workspace_size", "moe_route_topk", "moe_forward", "moe_ws_views",
             "moe_read_status", "moe_debug_dequant", "moe_status_string",
             "moe_kernels_enqueued", "moe_forward_noalloc", "moe_set_timing_events",
-            "moe_router_logits", "moe_shared_gate", "moe_set_wait_limit"]
+            "moe_router_logits", "moe_shared_gate", "moe_set_wait_limit",
+            "moe_forward_routed", "moe_chain_workspace_size", "moe_chain_forward",
+            "moe_chain_status"]
 
 
 class ExpertDesc(ctypes.Structure):
@@ -50,6 +53,18 @@ class WsView(ctypes.Structure):
                 ("hq", ctypes.c_void_p), ("hd", ctypes.c_void_p), ("hs", ctypes.c_void_p),
                 ("h", ctypes.c_void_p), ("slots", ctypes.c_int32), ("hpad", ctypes.c_int32),
                 ("counters", ctypes.c_void_p)]
+
+
+class ChainLayer(ctypes.Structure):
+    _fields_ = [("arena", ctypes.c_void_p), ("d_router", ctypes.c_void_p),
+                ("d_gate_row", ctypes.c_void_p), ("d_norm_weight", ctypes.c_void_p)]
+
+
+class ChainTrace(ctypes.Structure):
+    _fields_ = [("x", ctypes.c_void_p), ("xn", ctypes.c_void_p), ("logits", ctypes.c_void_p),
+                ("ids", ctypes.c_void_p),
+                ("w", ctypes.c_void_p), ("gate", ctypes.c_void_p), ("out", ctypes.c_void_p),
+                ("early", ctypes.c_void_p)]
 
 
 _P = ctypes.c_void_p
@@ -75,6 +90,10 @@ _lib.moe_set_timing_events.argtypes = [_P, _P, _P, _P]
 _lib.moe_router_logits.argtypes = [_P, _I, _I, _P, _I, _P, _P]
 _lib.moe_shared_gate.argtypes = [_P, _I, _I, _P, _P, _P]
 _lib.moe_set_wait_limit.argtypes = [_P, ctypes.c_uint64]
+_lib.moe_forward_routed.argtypes = [_P, _P, _I, _I, _P, _P, _P, _P, _P, _P, _S, _U, _P]
+_lib.moe_chain_workspace_size.argtypes = [_P, _I, _I, _I, _U, ctypes.POINTER(_S)]
+_lib.moe_chain_forward.argtypes = [_P, _I, _P, _I, _I, _P, _P, _S, _U, _P, _P]
+_lib.moe_chain_status.argtypes = [_P, _I, _P, _I, _I, _U, ctypes.POINTER(_P)]
 _lib.moe_kernels_enqueued.argtypes = []
 _lib.moe_kernels_enqueued.restype = ctypes.c_uint64
 
@@ -178,6 +197,61 @@ def forward_noalloc_status(arena, d_x, d_logits, T, k, d_out, d_status=None, str
 def forward_status(arena, d_x, d_logits, T, k, d_out, d_ws, ws_bytes, flags=0, stream=None) -> int:
     """moe_forward returning its status code instead of raising (for error-path tests)."""
     return _lib.moe_forward(arena, d_x, d_logits, T, k, d_out, d_ws, ws_bytes, flags, stream)
+
+
+def forward_routed(arena: int, d_x: int, T: int, k: int, d_router: int, d_gate_row, d_logits: int,
+                   d_gate, d_out: int, d_ws: int, ws_bytes: int, flags: int = 0,
+                   stream=None) -> None:
+    """moe_forward_routed: router (and optional shared gate) then the layer."""
+    _check(forward_routed_status(arena, d_x, T, k, d_router, d_gate_row, d_logits, d_gate, d_out,
+                                 d_ws, ws_bytes, flags, stream), "moe_forward_routed")
+
+
+def forward_routed_status(arena, d_x, T, k, d_router, d_gate_row, d_logits, d_gate, d_out, d_ws,
+                          ws_bytes, flags=0, stream=None) -> int:
+    return _lib.moe_forward_routed(arena, d_x, T, k, d_router, d_gate_row, d_logits, d_gate, d_out,
+                                   d_ws, ws_bytes, flags, stream)
+
+
+def _chain_layers(layers):
+    """layers: sequence of (arena handle, d_router, d_gate_row or None[, d_norm_weight or None])."""
+    arr = (ChainLayer * len(layers))()
+    for i, ly in enumerate(layers):
+        arr[i].arena, arr[i].d_router, arr[i].d_gate_row = ly[0], ly[1], ly[2]
+        arr[i].d_norm_weight = ly[3] if len(ly) > 3 else None
+    return arr
+
+
+def chain_workspace_size(layers, max_tokens: int, k: int, flags: int = 0) -> int:
+    n = _S()
+    _check(_lib.moe_chain_workspace_size(_chain_layers(layers), len(layers), max_tokens, k, flags,
+                                         ctypes.byref(n)), "moe_chain_workspace_size")
+    return n.value
+
+
+def chain_forward_status(layers, d_x: int, T: int, k: int, d_x_out: int, d_ws: int,
+                         ws_bytes: int, flags: int = 0, trace=None, stream=None) -> int:
+    """moe_chain_forward returning its status; trace: dict of device pointers (ChainTrace
+    field names) or None."""
+    tr = None
+    if trace is not None:
+        tr = ChainTrace(**{k2: trace.get(k2) for k2, _ in ChainTrace._fields_})
+    return _lib.moe_chain_forward(_chain_layers(layers), len(layers), d_x, T, k, d_x_out, d_ws,
+                                  ws_bytes, flags, ctypes.byref(tr) if tr is not None else None,
+                                  stream)
+
+
+def chain_forward(layers, d_x: int, T: int, k: int, d_x_out: int, d_ws: int, ws_bytes: int,
+                  flags: int = 0, trace=None, stream=None) -> None:
+    _check(chain_forward_status(layers, d_x, T, k, d_x_out, d_ws, ws_bytes, flags, trace, stream),
+           "moe_chain_forward")
+
+
+def chain_status_word(layers, d_ws: int, T: int, k: int, flags: int = 0) -> int:
+    p = _P()
+    _check(_lib.moe_chain_status(_chain_layers(layers), len(layers), d_ws, T, k, flags,
+                                 ctypes.byref(p)), "moe_chain_status")
+    return p.value
 
 
 def ws_views(arena: int, d_ws: int, T: int, k: int, flags: int = 0) -> dict:

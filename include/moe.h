@@ -63,8 +63,19 @@ typedef enum {
  *   Q8_0  32 weights in 34 B: fp16 d, 32 int8 q; w = d*q
  *   Q5_1  32 weights in 24 B: fp16 d, fp16 m, 32 fifth bits (uint32), 16 B of 4-bit quants
  *         (element n < 16: low nibble of byte n, n >= 16: high nibble of byte n-16);
- *         w = d*q + m                                                                        */
-typedef enum { MOE_FMT_Q4_K = 0, MOE_FMT_Q5_K = 1, MOE_FMT_Q8_0 = 2, MOE_FMT_Q5_1 = 3 } moe_fmt;
+ *         w = d*q + m
+ *   Q6_K  256 weights in 210 B: 128 B of low 4 bits, 64 B of high 2 bits, 16 int8 scales (one
+ *         per 16 weights), fp16 d; w = d*sc*(q - 32).  The format real Q4_K_M model files mix
+ *         into their FFN tensors.  Dequant-GEMV and CUDA-core paths only: an arena holding a
+ *         Q6_K expert takes no tensor-core plan (its integer products sc*(q-32) reach 12
+ *         significant bits; the exact fp16 operands of that path hold 11).                    */
+typedef enum {
+    MOE_FMT_Q4_K = 0,
+    MOE_FMT_Q5_K = 1,
+    MOE_FMT_Q8_0 = 2,
+    MOE_FMT_Q5_1 = 3,
+    MOE_FMT_Q6_K = 4
+} moe_fmt;
 
 /* One expert inside the arena.  Matrices follow the GGUF convention: a row is one output
  * neuron, blocks run along the input dimension.  gate and up: ffn rows of `hidden` weights;
@@ -100,6 +111,8 @@ void moe_arena_destroy(moe_arena *arena);
                                     MOE_ERR_WORKSPACE); MOE_ERR_UNSUPPORTED when the arena's
                                     shape has no tensor-core plan (hidden % 256 or ffn % 64)   */
 #define MOE_F_KEEP_H 8u          /* also store fp32 h (SwiGLU output) in the workspace       */
+#define MOE_F_LOOKAHEAD 16u      /* moe_chain_forward: prefetch the next layer's predicted
+                                    experts into L2 while a layer runs (batches of <= 16)    */
 
 /* Bytes of device workspace moe_forward needs for up to max_tokens tokens, k routed experts
  * per token and the given flags.  The workspace is caller-owned scratch, 256-byte aligned. */
@@ -224,6 +237,70 @@ moe_status moe_set_timing_events(moe_arena *arena, void *ev_begin, void *ev_mid,
  * counterpart is the engine's stall watchdog ("Strata - the details", "Troubleshooting").
  * ns > 0; MOE_ERR_INVALID_ARG otherwise.                                                      */
 moe_status moe_set_wait_limit(moe_arena *arena, uint64_t ns);
+
+/* The layer with its router and the shared-expert gate in front: the pages keep the routers on
+ * the GPU in the per-token path ("Strata: a 125B MoE at 94 tok/s on a 12 GB Card", "Three
+ * architecture facts").  One kernel reads d_x once and writes d_logits fp32 [T][n_experts] =
+ * x . d_router rows (d_router fp32 [n_experts][hidden], as moe_router_logits) and, when
+ * d_gate_row (fp32 [hidden]) is not NULL, d_gate fp32 [T] = 1 / (1 + exp(-x . gate_row)) (as
+ * moe_shared_gate); then moe_forward runs on those logits with the shared expert's output
+ * scaled by d_gate[t] instead of 1 (a7: out[t] = sum_j w[t][j] y[t][e_j] + g[t] y[t][shared]).
+ * d_logits and d_gate are caller-owned outputs, left for inspection.  A gate row on an arena
+ * without a shared expert is MOE_ERR_INVALID_ARG.  Workspace, flags and errors as moe_forward;
+ * d_router, d_gate_row and d_x 16-byte aligned.                                             */
+moe_status moe_forward_routed(const moe_arena *arena, const float *d_x, int T, int k,
+                              const float *d_router, const float *d_gate_row, float *d_logits,
+                              float *d_gate, float *d_out, void *d_ws, size_t ws_bytes,
+                              uint32_t flags, void *stream);
+
+/* A chain of MoE layers on a residual stream, as a decoder runs them ("Strata - the details",
+ * "How it works": the verify pass runs the window through every layer).  Each layer reads the
+ * RMS-normalised stream, as the MoE block of a pre-norm decoder does.  For each layer l:
+ *   xn_l = x_l / sqrt(mean(x_l^2) + MOE_CHAIN_RMS_EPS) * norm_weight (per token; the
+ *          layer's RMSNorm weight, 1 when d_norm_weight is NULL),
+ *   logits_l = router_l(xn_l), g_l = gate_l(xn_l) (when the layer has a gate row),
+ *   out_l = the layer on xn_l (as moe_forward_routed), x_{l+1} = fp32(x_l + out_l);
+ * d_x_out fp32 [T][hidden] receives x_L.  Every layer's arena has the same hidden size.  The
+ * residual add and the normalisation are folded into the router kernel (one pass over x).
+ * MOE_F_LOOKAHEAD (T <= 16): the router kernel of layer l also computes layer l+1's logits on
+ * xn_l; a one-CTA kernel takes their top-k and prefetches those experts' packed rows (and the
+ * shared expert's) into L2 before layer l runs -- the engine's router lookahead ("Strata - the
+ * details", the STRATA_LOOKAHEAD paragraph), with L2 in place of the engine's VRAM cache.  A
+ * wrong prediction costs only bandwidth: layer l+1 always routes on its own logits.
+ * Workspace: moe_chain_workspace_size for the same layers, T, k and flags.
+ * trace (may be NULL; each pointer in it may be NULL) receives device copies of the
+ * intermediates: the layers' inputs and the result, logits, ids, weights, gates, outputs and
+ * (MOE_F_LOOKAHEAD) the predicted ids.  The status word of the workspace (moe_chain_status)
+ * collects device-side errors of every layer.                                                */
+typedef struct {
+    const moe_arena *arena;
+    const float *d_router;       /* fp32 [n_experts][hidden]                                */
+    const float *d_gate_row;     /* fp32 [hidden] or NULL                                   */
+    const float *d_norm_weight;  /* fp32 [hidden] or NULL (all ones): the RMSNorm weight    */
+} moe_chain_layer;
+
+#define MOE_CHAIN_RMS_EPS 1e-6f
+
+typedef struct {
+    float *x;          /* [n_layers + 1][T][hidden]: x_0 .. x_L                              */
+    float *xn;         /* [n_layers][T][hidden]: each layer's normalised input xn_l          */
+    float *logits;     /* [n_layers][T][max n_experts]: row stride = the largest n_experts  */
+    int32_t *ids;      /* [n_layers][T][k]                                                   */
+    float *w;          /* [n_layers][T][k]                                                   */
+    float *gate;       /* [n_layers][T] (layers without a gate row: left untouched)          */
+    float *out;        /* [n_layers][T][hidden]: each layer's output before the residual add */
+    int32_t *early;    /* [n_layers][T][k]: entry l >= 1 = layer l's ids predicted from
+                          xn_{l-1} (MOE_F_LOOKAHEAD); entry 0 left untouched                 */
+} moe_chain_trace;
+
+moe_status moe_chain_workspace_size(const moe_chain_layer *host_layers, int n_layers,
+                                    int max_tokens, int k, uint32_t flags, size_t *bytes);
+moe_status moe_chain_forward(const moe_chain_layer *host_layers, int n_layers, const float *d_x,
+                             int T, int k, float *d_x_out, void *d_ws, size_t ws_bytes,
+                             uint32_t flags, const moe_chain_trace *host_trace, void *stream);
+/* The status word of a chain workspace (for moe_read_status). */
+moe_status moe_chain_status(const moe_chain_layer *host_layers, int n_layers, void *d_ws, int T,
+                            int k, uint32_t flags, uint32_t **d_status_word);
 
 /* Number of kernels this library has enqueued (or recorded into a CUDA graph under stream
  * capture) in this process since it was loaded.  Counting a captured forward gives the

@@ -260,25 +260,42 @@ def forward(arena: np.ndarray, experts: np.ndarray, shared: int, hidden: int, ff
     return out, out64
 
 
+RMS_EPS = 1e-6
+
+
+def rmsnorm(x: np.ndarray, weight=None, eps: float = RMS_EPS) -> np.ndarray:
+    """The input of a pre-norm decoder's MoE block: every row of fp32 x divided by the root of
+    its mean square plus eps, times the fp32 norm weight [H] (all ones when None), in fp64
+    (squares summed in fp64), rounded once to fp32."""
+    x64 = np.ascontiguousarray(x, dtype=np.float32).astype(np.float64)
+    ms = (x64 * x64).sum(axis=1, keepdims=True) / x64.shape[1]
+    y = x64 / np.sqrt(ms + eps)
+    if weight is not None:
+        y = y * np.asarray(weight, dtype=np.float32).astype(np.float64)[None, :]
+    return y.astype(np.float32)
+
+
 def chain(layers, x0: np.ndarray, k: int, lookahead: bool = False):
-    """O12: a chain of MoE layers with a residual stream, as in a decoder: for each layer l,
-    logits = router(x_l, Wr_l) (O10), top-k (O3), out_l = O1-O9 (gated by O11 when the layer
-    has a gate row), and x_{l+1} = fp32(x_l + out_l).  `layers` is a sequence of dicts with
-    keys arena, experts, shared, hidden, ffn, router (Wr [E][H]) and optionally gate (wg [H]).
+    """O12: a chain of MoE layers on a residual stream, as in a pre-norm decoder: for each layer
+    l, xn_l = rmsnorm(x_l, norm weight), logits = router(xn_l, Wr_l) (O10), top-k (O3), out_l =
+    O1-O9 on xn_l (gated by O11 of xn_l when the layer has a gate row), and x_{l+1} =
+    fp32(x_l + out_l).  `layers` is a sequence of dicts with keys arena, experts, shared, hidden,
+    ffn, router (Wr [E][H]) and optionally gate (wg [H]) and norm (the RMSNorm weight [H]).
 
     Returns (x_L fp32 [T][H], per-layer ids).  With lookahead=True it also returns, for every
-    layer l >= 1, the ids that layer l's router picks from x_{l-1} (before layer l-1 has
+    layer l >= 1, the ids that layer l's router picks from xn_{l-1} (before layer l-1 has
     run): the experts a prefetch one layer ahead would fetch."""
     x = np.ascontiguousarray(x0, dtype=np.float32)
     all_ids, early = [], []
     for l, L in enumerate(layers):
-        logits, _ = router(x, L["router"])
+        xn = rmsnorm(x, L.get("norm"))
+        logits, _ = router(xn, L["router"])
         ids, w, _ = topk(logits, k)
-        g = shared_gate(x, L["gate"]) if L.get("gate") is not None else None
-        out, _ = forward(L["arena"], L["experts"], L["shared"], L["hidden"], L["ffn"], x, ids, w,
-                         gate=g)
+        g = shared_gate(xn, L["gate"]) if L.get("gate") is not None else None
+        out, _ = forward(L["arena"], L["experts"], L["shared"], L["hidden"], L["ffn"], xn, ids,
+                         w, gate=g)
         if lookahead and l + 1 < len(layers):
-            early.append(topk(router(x, layers[l + 1]["router"])[0], k)[0])
+            early.append(topk(router(xn, layers[l + 1]["router"])[0], k)[0])
         x = (x + out).astype(np.float32)
         all_ids.append(ids)
     return (x, all_ids, early) if lookahead else (x, all_ids)

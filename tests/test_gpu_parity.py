@@ -9,8 +9,7 @@ import pytest
 import oracle
 from expert_ffn_token_b200 import synth
 
-from gpu_helpers import (W_TOL, check_parity, device_layer, inputs, run_forward, torch_cuda,
-                         ws_array)
+from gpu_helpers import W_TOL, check_layer, device_layer, inputs, run_forward, torch_cuda
 
 pytestmark = pytest.mark.gpu
 
@@ -144,71 +143,27 @@ def test_route_bit_exact(torch, T, E, k, ties):
 # ------------------------------------------------------------------ a1-a7 the layer
 
 
-def _check_layer(torch, w, layer, x, logits, flags=0, tokens=None, L=None, name=""):
-    """One forward through the C ABI on any path (flags), checked against the oracle: the
-    intermediates left in the workspace bit for bit, the Q8_1 of the GPU's own h bit for bit,
-    and the outputs through gpu_helpers.check_parity (h, the chain after h, end to end)."""
-    from expert_ffn_token_b200 import moe
-    T = x.shape[0]
-    fl = flags | moe.F_KEEP_H
-    own = L is None
-    if own:
-        L, _, _ = device_layer(w, layer, max_tokens=T, flags=fl)
-    gpu = run_forward(L, x, logits, flags=fl)
-    assert L.status() == 0
-    # intermediates left in the workspace equal the standalone steps
-    v = L.views(T, fl)
-    k, E, H = w.k, w.n_experts, w.hidden
-    rid, rw, _ = oracle.topk(logits, k)
-    assert np.array_equal(ws_array(L, v["ids"], T * k, np.int32).reshape(T, k), rid)
-    assert np.abs(ws_array(L, v["w"], T * k, np.float32).reshape(T, k) - rw).max() <= W_TOL
-    rq, rd, rs, _ = oracle.quantize_q8_1(x)
-    assert np.array_equal(ws_array(L, v["xq"], T * H, np.int8), rq)
-    assert np.array_equal(ws_array(L, v["xd"], T * H // 32, np.uint16), rd)
-    assert np.array_equal(ws_array(L, v["xs"], T * H // 32, np.uint16), rs)
-    rc, ro, rp, ri = oracle.group(rid, E)
-    assert np.array_equal(ws_array(L, v["counts"], E, np.int32), rc)
-    assert np.array_equal(ws_array(L, v["offsets"], E + 1, np.int32), ro)
-    assert np.array_equal(ws_array(L, v["perm"], T * k, np.int32), rp)
-    # the quantizer applied to the GPU's own h is bit-exact (every slot)
-    hp, F = v["hpad"], w.ffn
-    n_slots = T * k + (T if w.shared else 0)
-    h = ws_array(L, v["h"], n_slots * F, np.float32).reshape(n_slots, F)
-    hq = ws_array(L, v["hq"], n_slots * hp, np.int8).reshape(n_slots, hp)
-    hd = ws_array(L, v["hd"], n_slots * hp // 32, np.uint16).reshape(n_slots, hp // 32)
-    hs = ws_array(L, v["hs"], n_slots * hp // 32, np.uint16).reshape(n_slots, hp // 32)
-    pad = np.zeros((n_slots, hp), np.float32)
-    pad[:, :F] = h
-    q2, d2, s2, _ = oracle.quantize_q8_1(pad)
-    assert np.array_equal(hq.ravel(), q2)
-    assert np.array_equal(hd.ravel(), d2)
-    assert np.array_equal(hs.ravel(), s2)
-    check_parity(L, w, layer, x, logits, gpu, fl, tokens=tokens,
-                 name=name or f"{w.name} T={T} flags={flags}")
-    if own:
-        L.close()
-    return gpu
 
 
 @pytest.mark.parametrize("flags", [0, 2, 4, 5])     # auto, force decode, prefill, prefill+det
 def test_layer_tiny_all_paths(torch, flags):
     w = W["tiny"]
     x, logits = inputs(w, 0)
-    _check_layer(torch, w, 0, x, logits, flags=flags)
+    check_layer(torch, w, 0, x, logits, flags=flags)
 
 
 @pytest.mark.parametrize("layer", [0, 23, 47])
 def test_layer_decode_full_size(torch, layer):
     w = W["decode"]
     x, logits = inputs(w, layer)
-    _check_layer(torch, w, layer, x, logits)
+    check_layer(torch, w, layer, x, logits)
 
 
 @pytest.mark.parametrize("layer", [0, 47])
 def test_layer_mtp_verify_full_size(torch, layer):
     w = W["mtp_verify"]
     x, logits = inputs(w, layer)
-    _check_layer(torch, w, layer, x, logits)
+    check_layer(torch, w, layer, x, logits)
 
 
 def _sample_tokens(T, ids, n=24, seed=0):
@@ -231,7 +186,7 @@ def test_layer_prefill_full_size_sampled(torch, name):
         # experts take > 1000 tokens, a long tail takes only a handful
         assert (counts > 1000).sum() >= 3 and (counts < 8).sum() >= 5 and (counts < 16).sum() >= 50
     # every token's integer outputs (views) and a seeded sample of 512 tokens' layer outputs
-    _check_layer(torch, w, 0, x, logits, tokens=_sample_tokens(w.tokens, ids, n=512))
+    check_layer(torch, w, 0, x, logits, tokens=_sample_tokens(w.tokens, ids, n=512))
 
 
 @pytest.mark.parametrize("T", [1, 2, 17, 65, 100, 300])
@@ -242,7 +197,7 @@ def test_layer_ragged_batches(torch, T):
     if T > 64:
         ids, _, _ = oracle.topk(logits, w.k)
         tokens = _sample_tokens(T, ids, n=20, seed=T)
-    _check_layer(torch, w, 5, x, logits, tokens=tokens)
+    check_layer(torch, w, 5, x, logits, tokens=tokens)
 
 
 def test_decode_and_prefill_paths_agree(torch):
@@ -252,8 +207,8 @@ def test_decode_and_prefill_paths_agree(torch):
     x, logits = inputs(w, 2)
     fl = moe.F_FORCE_PREFILL | moe.F_DETERMINISTIC | moe.F_KEEP_H
     L, _, _ = device_layer(w, 2, max_tokens=12, flags=fl)
-    a = _check_layer(torch, w, 2, x, logits, flags=moe.F_FORCE_DECODE, L=L, name="paths: decode")
-    b = _check_layer(torch, w, 2, x, logits, flags=moe.F_FORCE_PREFILL | moe.F_DETERMINISTIC,
+    a = check_layer(torch, w, 2, x, logits, flags=moe.F_FORCE_DECODE, L=L, name="paths: decode")
+    b = check_layer(torch, w, 2, x, logits, flags=moe.F_FORCE_PREFILL | moe.F_DETERMINISTIC,
                      L=L, name="paths: tensor cores, deterministic")
     c = run_forward(L, x, logits, flags=fl)
     assert np.array_equal(b, c)                       # deterministic mode repeats bit for bit
@@ -266,14 +221,14 @@ def test_edge_k1_and_k_equals_e(torch):
     for k, E in ((1, 16), (4, 4)):
         w = synth.Workload("edge", 60 + k, 256, 256, E, k, 5, True, 1, "normal")
         x, logits = inputs(w, 0)
-        _check_layer(torch, w, 0, x, logits)
+        check_layer(torch, w, 0, x, logits)
 
 
 def test_edge_one_expert_takes_every_token(torch):
     w = synth.with_tokens(W["tiny"], 300, layers=1)
     x, logits = inputs(w, 0)
     logits[:, 3] += 100.0
-    _check_layer(torch, w, 0, x, logits)
+    check_layer(torch, w, 0, x, logits)
 
 
 def test_nonfinite_activation_sets_status(torch):
@@ -327,7 +282,7 @@ def test_decode_large_expert_count_uses_grouped_kernels(torch):
     # 2048 experts exceed the fused decode kernel's plan: the three-kernel decode path runs
     w = synth.Workload("wideE", 70, 256, 256, 2048, 4, 3, True, 1, "normal", sigma=2.0)
     x, logits = inputs(w, 0)
-    _check_layer(torch, w, 0, x, logits)
+    check_layer(torch, w, 0, x, logits)
 
 
 # ------------------------------------------------------------------ Q5_1 experts
@@ -371,18 +326,18 @@ def test_q5_1_layer_every_path(torch, T, flags):
     # or to the tensor cores (4), deterministic (5)
     w = synth.with_tokens(Q51, T)
     x, logits = inputs(w, 0)
-    _check_layer(torch, w, 0, x, logits, flags=flags)
+    check_layer(torch, w, 0, x, logits, flags=flags)
 
 
 @pytest.mark.parametrize("T,flags", [(2, 0), (12, 0), (150, 2), (150, 4), (150, 5)])
 def test_four_formats_layer_every_path(torch, T, flags):
     w = synth.with_tokens(FOUR, T)
     x, logits = inputs(w, 0)
-    _check_layer(torch, w, 0, x, logits, flags=flags)
+    check_layer(torch, w, 0, x, logits, flags=flags)
 
 
 def test_q5_1_large_expert_count_grouped_decode(torch):
     w = synth.Workload("wideE_q51", 71, 256, 256, 2048, 4, 3, True, 1, "normal", sigma=2.0,
                        mix=((synth.Q5_1, 1.0),))
     x, logits = inputs(w, 0)
-    _check_layer(torch, w, 0, x, logits)
+    check_layer(torch, w, 0, x, logits)

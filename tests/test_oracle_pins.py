@@ -696,12 +696,43 @@ def test_chain_of_one_layer_is_the_layer_plus_residual():
     L = _chain_layer(w, 0, 31, gate=True)
     x0 = synth.activations(w, 0)
     xL, ids = oracle.chain([L], x0, w.k)
-    logits, _ = oracle.router(x0, L["router"])
+    xn = oracle.rmsnorm(x0)
+    logits, _ = oracle.router(xn, L["router"])
     rid, rw, _ = oracle.topk(logits, w.k)
-    out, _ = oracle.forward(L["arena"], L["experts"], L["shared"], w.hidden, w.ffn, x0, rid, rw,
-                            gate=oracle.shared_gate(x0, L["gate"]))
+    out, _ = oracle.forward(L["arena"], L["experts"], L["shared"], w.hidden, w.ffn, xn, rid, rw,
+                            gate=oracle.shared_gate(xn, L["gate"]))
     assert np.array_equal(ids[0], rid)
     assert np.array_equal(xL, (x0 + out).astype(np.float32))
+
+
+def test_rmsnorm_closed_forms():
+    eps = oracle.RMS_EPS
+    # a 3-4 row: mean square 12.5 (not the sum 25), so every value is divided by sqrt(12.5 + eps)
+    got = oracle.rmsnorm(np.array([[3.0, 4.0], [0.0, 0.0]], np.float32))
+    assert got[0, 0] == np.float32(3.0 / np.sqrt(12.5 + eps))
+    assert got[0, 1] == np.float32(4.0 / np.sqrt(12.5 + eps))
+    assert (got[1] == 0.0).all()                       # a zero row stays zero (eps > 0)
+    # a constant row a: a / sqrt(a^2 + eps), the sign kept
+    for a in (-7.0, 0.01, 2.0 ** 40):
+        row = np.full((1, 64), a, np.float32)
+        assert (oracle.rmsnorm(row) == np.float32(a / np.sqrt(a * a + eps))).all()
+    # one spike among zeros of a row of n: the spike becomes sqrt(n) (eps negligible), the rest 0
+    row = np.zeros((1, 256), np.float32)
+    row[0, 17] = 1e3
+    got = oracle.rmsnorm(row)
+    assert abs(got[0, 17] - 16.0) < 1e-6 and np.count_nonzero(got) == 1
+    # the norm weight scales each column after the division: [3, 4] with weight [2, 0.5]
+    got = oracle.rmsnorm(np.array([[3.0, 4.0]], np.float32), np.array([2.0, 0.5], np.float32))
+    assert got[0, 0] == np.float32(6.0 / np.sqrt(12.5 + eps))
+    assert got[0, 1] == np.float32(2.0 / np.sqrt(12.5 + eps))
+    # rows are independent, and the output's mean square is ms / (ms + eps)
+    rng = np.random.default_rng(5)
+    x = (rng.standard_normal((3, 512)) * [[1e-2], [1.0], [1e3]]).astype(np.float32)
+    got = oracle.rmsnorm(x).astype(np.float64)
+    for i in range(3):
+        assert np.array_equal(oracle.rmsnorm(x[i:i + 1])[0], got[i].astype(np.float32))
+        ms = (x[i].astype(np.float64) ** 2).mean()
+        assert abs((got[i] ** 2).mean() - ms / (ms + eps)) < 1e-6
 
 
 def test_chain_of_silent_layers_keeps_the_residual():
