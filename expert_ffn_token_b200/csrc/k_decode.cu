@@ -68,6 +68,7 @@ struct DecParams {
     int stage_bytes, nstages, max_jobs, slots;
     int keep_h;            // also store fp32 h
     uint64_t wait_ns;      // limit of every bounded wait
+    Lookahead look;        // the next layer's prediction (look.logits null: none)
     int o_bar, o_meta, o_xq, o_xd, o_xs, o_jobs, o_stok, o_sw, o_hq, o_hd, o_hs, o_gu, o_h,
         o_acc, o_misc;
     int smem_bytes;
@@ -326,11 +327,12 @@ __device__ __forceinline__ float key_value(uint32_t k) {
     return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
 }
 
-// One warp: top-k of a logit row held in registers (VPL values per lane, value e at lane e%32,
-// slot e/32).  Descending logit, ties to the lower id; weights = softmax over the chosen k.
+// One warp: the k largest of a logit row held in registers (VPL values per lane, value e at
+// lane e%32, slot e/32), descending, ties to the lower id.  Lane j < k gets the j-th choice's
+// order key and id.  Returns false (nothing chosen) when the row is not all finite.
 template <int VPL>
-__device__ __noinline__ void warp_topk_reg(const float *row, int E, int k, int *ids_out,
-                                              float *w_out, uint32_t *status) {
+__device__ __forceinline__ bool topk_select(const float *row, int E, int k, uint32_t &my_key,
+                                            int &my_id) {
     const int lane = threadIdx.x & 31;
     uint32_t key[VPL];
     bool fin = true;
@@ -341,16 +343,9 @@ __device__ __noinline__ void warp_topk_reg(const float *row, int E, int k, int *
         fin = fin && isfinite(v);
         key[i] = e < E ? order_key(v) : 0u;
     }
-    if (!__all_sync(kFullMask, fin)) {
-        if (lane < k) {
-            ids_out[lane] = lane;
-            w_out[lane] = __fdiv_rn(1.0f, (float)k);
-        }
-        if (lane == 0) set_status(status, MOE_ERR_NONFINITE);
-        return;
-    }
-    uint32_t my_key = 0;
-    int my_id = 0;
+    my_key = 0;
+    my_id = 0;
+    if (!__all_sync(kFullMask, fin)) return false;
     for (int j = 0; j < k; j++) {
         uint32_t bk = 0;
         int bi = 0;
@@ -372,6 +367,24 @@ __device__ __noinline__ void warp_topk_reg(const float *row, int E, int k, int *
             for (int i = 0; i < VPL; i++)
                 if (i == (int)(win >> 5)) key[i] = 0u;
         }
+    }
+    return true;
+}
+
+// One warp: top-k of a logit row (as topk_select) and weights = softmax over the chosen k.
+template <int VPL>
+__device__ __noinline__ void warp_topk_reg(const float *row, int E, int k, int *ids_out,
+                                              float *w_out, uint32_t *status) {
+    const int lane = threadIdx.x & 31;
+    uint32_t my_key;
+    int my_id;
+    if (!topk_select<VPL>(row, E, k, my_key, my_id)) {
+        if (lane < k) {
+            ids_out[lane] = lane;
+            w_out[lane] = __fdiv_rn(1.0f, (float)k);
+        }
+        if (lane == 0) set_status(status, MOE_ERR_NONFINITE);
+        return;
     }
     const float l0 = key_value(__shfl_sync(kFullMask, my_key, 0));
     const float ex = lane < k ? expf(key_value(my_key) - l0) : 0.f;
@@ -1088,6 +1101,20 @@ __device__ __forceinline__ void consumer(const DecParams &P, const Ctx &C) {
     }
 }
 
+// The router lookahead of a chain, inside the layer: on CTA 0, warp (kCW - 1 - t) takes token
+// t's top-k of the next layer's logits (the same selection as a2) and stores the predicted ids;
+// the next layer's router pass prefetches those experts into L2 before the next layer runs.  A
+// row of logits that is not finite predicts id -1 (nothing is prefetched for it; the next layer
+// reports the row).
+template <int VPL>
+__device__ __noinline__ void lookahead(const Lookahead A, int k, int t) {
+    const int lane = threadIdx.x & 31;
+    uint32_t key;
+    int id;
+    const bool ok = topk_select<VPL>(A.logits + (size_t)t * A.E, A.E, k, key, id);
+    if (lane < k) A.ids_out[t * k + lane] = ok ? id : -1;
+}
+
 // NT: activation rows per pass of rows_dot; TT: largest token count the down sums hold;
 // FK: format class of the arena; VPL: router logits per lane (E <= 32 * VPL).
 template <int NT, int TT, int FK, int VPL>
@@ -1153,6 +1180,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_fused(const DecParams P)
     C.i_lo = (int)((long long)P.H * cta / G);
     C.i_hi = (int)((long long)P.H * (cta + 1) / G);
 
+    if (P.look.logits && C.cta0 && warp < kCW && warp >= kCW - P.T)
+        lookahead<VPL>(P.look, P.k, kCW - 1 - warp);
     if (C.s_misc[3]) {
         // the descriptor table did not arrive in time: no work here (this CTA's blocks are never
         // published, so the grid-wide waits of the others give up too); the copy lands first
@@ -1207,10 +1236,11 @@ cudaError_t launch_variant(const cudaLaunchConfig_t &cfg, const DecParams &P, in
 cudaError_t launch_decode_fused(const FfnArgs &a, int E, int shared, const float *x,
                                 const float *logits, uint8_t *ws, const WsLayout &L,
                                 size_t sync_off, size_t blkcnt_off, bool pdl, cudaStream_t st,
-                                bool *taken) {
+                                bool *taken, bool *look_fused) {
     (void)sync_off;
     (void)blkcnt_off;
     *taken = false;
+    *look_fused = false;
     if (a.T > kDecodeMaxT || E > 1024 || a.T * a.k > kDecodeMaxT * kMaxK || a.F % 32) return cudaSuccess;
     int dev = 0, nsm = 0, cap = 0;
     cudaError_t err = cudaGetDevice(&dev);
@@ -1241,6 +1271,9 @@ cudaError_t launch_decode_fused(const FfnArgs &a, int E, int shared, const float
     P.slots = a.T * a.k + a.T;
     P.keep_h = a.h != nullptr;
     P.wait_ns = a.wait_ns;
+    // the lookahead runs inside when the next layer's logits fit this kernel's top-k width
+    const int top_width = E <= 256 ? 256 : E <= 512 ? 512 : 1024;
+    if (a.look.logits && a.look.ids_out && a.look.E <= top_width && a.T <= kCW) P.look = a.look;
     auto al = [](int v, int q) { return (v + q - 1) / q * q; };
     const int fk = a.fmt_mask == (1 << MOE_FMT_Q4_K) ? FK_Q4K
                    : a.fmt_mask == (1 << MOE_FMT_Q5_K) ? FK_Q5K : FK_ANY;
@@ -1294,6 +1327,7 @@ cudaError_t launch_decode_fused(const FfnArgs &a, int E, int shared, const float
     if (err != cudaSuccess) return err;
     note_launches(1);
     *taken = true;
+    *look_fused = P.look.logits != nullptr;
     return cudaSuccess;
 }
 

@@ -352,10 +352,14 @@ static moe_status forward_checks(const moe_arena *arena, const float *d_x, const
     return MOE_OK;
 }
 
-// moe_forward with an optional per-token weight of the shared expert's output (d_gate [T]).
+// moe_forward with an optional per-token weight of the shared expert's output (d_gate [T]) and
+// an optional router lookahead for the next layer of a chain, which the decode kernel runs
+// inside when it can (*look_fused; otherwise the caller runs it).
 static moe_status forward_impl(const moe_arena *arena, const float *d_x, const float *d_logits,
                                const float *d_gate, int T, int k, float *d_out, void *d_ws,
-                               size_t ws_bytes, uint32_t flags, void *stream) {
+                               size_t ws_bytes, uint32_t flags, void *stream,
+                               const Lookahead *look = nullptr, bool *look_fused = nullptr) {
+    if (look_fused) *look_fused = false;
     const moe_status chk = forward_checks(arena, d_x, d_logits, T, k, d_out, d_ws, ws_bytes, flags);
     if (chk != MOE_OK) return chk;
     const WsLayout L = ws_layout(arena, T, k, flags);
@@ -397,10 +401,12 @@ static moe_status forward_impl(const moe_arena *arena, const float *d_x, const f
         a.h = (flags & MOE_F_KEEP_H) ? reinterpret_cast<float *>(ws + L.h) : nullptr;
         a.gate = d_gate;
         a.wait_ns = arena->wait_ns;
-        bool taken = false;
+        if (look) a.look = *look;
+        bool taken = false, fused = false;
         cudaError_t e = launch_decode_fused(a, E, shared, d_x, d_logits, ws, L, L.sync, L.blkcnt,
-                                            true, st, &taken);
+                                            true, st, &taken, &fused);
         if (e != cudaSuccess) return MOE_ERR_CUDA;
+        if (look_fused) *look_fused = fused;
         if (taken) return MOE_OK;
     }
     // a1-a3
@@ -579,7 +585,7 @@ static moe_status check_router_rows(const moe_arena *arena, const float *d_route
 
 // A chain workspace: the largest layer workspace, then the chain's own buffers.
 struct ChainLayout {
-    size_t fwd, xa, xb, xn, out, logits, next, gate, total;
+    size_t fwd, xa, xb, xn, out, logits, next, gate, pred, total;
     int H, Emax;
 };
 
@@ -603,7 +609,7 @@ static moe_status chain_layout(const moe_chain_layer *ls, int n, int T, int k, u
         C.Emax = std::max(C.Emax, A->E);
     }
     if ((flags & MOE_F_LOOKAHEAD) && lookahead_smem_bytes(C.Emax) > 200 * 1024)
-        return MOE_ERR_UNSUPPORTED;
+        return MOE_ERR_UNSUPPORTED;   // the top-k kernel of layers without the decode kernel
     size_t p = align256(C.fwd);
     auto take = [&](size_t bytes) {
         const size_t o = p;
@@ -618,6 +624,7 @@ static moe_status chain_layout(const moe_chain_layer *ls, int n, int T, int k, u
     C.logits = take((size_t)T * C.Emax * 4);
     C.next = take((size_t)T * C.Emax * 4);
     C.gate = take((size_t)T * 4);
+    C.pred = take((size_t)T * k * 4);
     C.total = p;
     return MOE_OK;
 }
@@ -647,7 +654,7 @@ moe_status moe_forward_routed(const moe_arena *arena, const float *d_x, int T, i
     a.gate = d_gate_row ? d_gate : nullptr;
     a.T = T;
     a.H = arena->H;
-    if (launch_router_rows(a, st) != cudaSuccess) return MOE_ERR_CUDA;
+    if (launch_router_rows(a, st, false) != cudaSuccess) return MOE_ERR_CUDA;
     return forward_impl(arena, d_x, d_logits, a.gate, T, k, d_out, d_ws, ws_bytes, flags, stream);
 }
 
@@ -693,6 +700,7 @@ moe_status moe_chain_forward(const moe_chain_layer *host_layers, int n_layers, c
     float *logits = reinterpret_cast<float *>(ws + C.logits);
     float *next = reinterpret_cast<float *>(ws + C.next);
     float *gate = reinterpret_cast<float *>(ws + C.gate);
+    int32_t *pred = reinterpret_cast<int32_t *>(ws + C.pred);   // ids predicted for layer l+1
     const int H = C.H;
     const size_t xbytes = (size_t)T * H * 4;
     auto copy = [&](void *dst, const void *src, size_t bytes) {
@@ -727,17 +735,34 @@ moe_status moe_chain_forward(const moe_chain_layer *host_layers, int n_layers, c
         a.gate = Ly.d_gate_row ? gate : nullptr;
         a.T = T;
         a.H = H;
-        if (launch_router_rows(a, st) != cudaSuccess) return MOE_ERR_CUDA;
-        if (l > 0) x = xbuf[l & 1];
-        if (ahead) {
-            const moe_arena *B = host_layers[l + 1].arena;
-            int32_t *early = tr.early ? tr.early + (size_t)(l + 1) * T * k : nullptr;
-            if (launch_lookahead(next, T, B->E, k, B->shared >= 0 ? 1 : 0, B->d_experts, B->H,
-                                 B->F, early, st) != cudaSuccess)
-                return MOE_ERR_CUDA;
+        if (look && l > 0) {   // warm L2 with the experts layer l-1 predicted for this layer
+            const size_t mb = std::max((size_t)A->F * A->max_stride01, (size_t)A->H * A->max_stride2);
+            a.pf.ids = pred;
+            a.pf.n = T * k;
+            a.pf.shared = A->shared >= 0 ? 1 : 0;
+            a.pf.experts = A->d_experts;
+            a.pf.E = A->E;
+            a.pf.H = A->H;
+            a.pf.F = A->F;
+            a.pf.pmax = (int)((mb + kPrefetchPiece - 1) / kPrefetchPiece);
         }
-        r = forward_impl(A, xn, logits, a.gate, T, k, out, d_ws, C.fwd, ff, stream);
+        if (launch_router_rows(a, st, true) != cudaSuccess) return MOE_ERR_CUDA;
+        if (l > 0) x = xbuf[l & 1];
+        Lookahead look{};
+        if (ahead) {   // layer l+1's prediction, from the logits of the pass above
+            look.logits = next;
+            look.E = host_layers[l + 1].arena->E;
+            look.ids_out = pred;
+        }
+        bool fused = false;
+        r = forward_impl(A, xn, logits, a.gate, T, k, out, d_ws, C.fwd, ff, stream,
+                         ahead ? &look : nullptr, &fused);
         if (r != MOE_OK) return r;
+        if (ahead && !fused &&   // the layer ran without the decode kernel: a kernel of its own
+            launch_lookahead(next, T, look.E, k, pred, st) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        if (ahead && tr.early && !copy(tr.early + (size_t)(l + 1) * T * k, pred, (size_t)T * k * 4))
+            return MOE_ERR_CUDA;
         const WsLayout L = ws_layout(A, T, k, ff);
         bool ok = true;
         if (tr.x) ok = ok && copy(tr.x + (size_t)l * T * H, x, xbytes);

@@ -41,6 +41,7 @@ constexpr int kMaxK = 32;         // routed experts per token
 constexpr int kMaxE = 4096;       // experts per layer
 constexpr int kDecodeMaxT = 16;   // largest batch the dequant-GEMV path takes by default
 constexpr int kChunk = 64;        // tokens per histogram chunk in the grouping kernels
+constexpr uint32_t kPrefetchPiece = 16384;   // bytes per L2 prefetch instruction (lookahead)
 
 // Q8_0 and Q5_1 carry their scale per 32 weights; the K-quants per 256-weight super-block.
 __host__ __device__ inline bool small_block(int fmt) {
@@ -152,6 +153,23 @@ cudaError_t launch_group(const int32_t *ids, int T, int k, int E, int shared, in
                          int32_t *chunk_counts, int32_t *chunk_base, Job *jobs, int32_t *njobs,
                          cudaStream_t st);
 
+// The next layer's expert prediction of a chain of layers (the router lookahead): its router
+// logits for this batch [T][E] and where its predicted ids go ([T][k]).
+struct Lookahead {
+    const float *logits;          // null: no lookahead
+    int E;
+    int32_t *ids_out;
+};
+
+// An L2 prefetch of predicted experts' packed rows: ids [n] (-1: none), the layer's expert
+// table, its sizes, and the 16 KB pieces of its largest matrix.
+struct ExpertPrefetch {
+    const int32_t *ids;           // null: none
+    int n, shared;                // shared: also the shared expert (index E)
+    const ExpertDev *experts;
+    int E, H, F, pmax;
+};
+
 struct FfnArgs {
     const ExpertDev *experts;
     const Job *jobs;
@@ -173,6 +191,7 @@ struct FfnArgs {
     int T, k, H, F, hpad, max_jobs, fmt_mask;
     int max_stride01, max_stride2;   // largest gate/up and down row strides in the arena
     uint64_t wait_ns;                // limit of every bounded wait in the kernels
+    Lookahead look;                  // the decode kernel's fused lookahead (logits null: none)
 };
 
 cudaError_t launch_gateup_gemv(const FfnArgs &a, cudaStream_t st);
@@ -182,10 +201,12 @@ cudaError_t launch_combine(const FfnArgs &a, bool shared, cudaStream_t st);
 
 // The whole layer for small batches in one persistent kernel (k_decode.cu).  Sets *taken to
 // false, enqueueing nothing, when the shape does not fit its shared-memory plan.
+// *look_fused tells whether a.look (when given) runs inside the kernel (the next layer's
+// expert count must fit the kernel's top-k width).
 cudaError_t launch_decode_fused(const FfnArgs &a, int E, int shared, const float *x,
                                 const float *logits, uint8_t *ws, const WsLayout &L,
                                 size_t sync_off, size_t blkcnt_off, bool pdl, cudaStream_t st,
-                                bool *taken);
+                                bool *taken, bool *look_fused);
 
 // Zero Q8_1(h) (int8 layout) in the padded columns [F, hpad) of every slot.
 cudaError_t launch_hpad_zero(const FfnArgs &a, cudaStream_t st);
@@ -247,13 +268,14 @@ struct RouterRowsArgs {
     const float *wg;
     float *gate;
     int E, En, T, H;
+    ExpertPrefetch pf;   // issued by the whole grid before the rows
 };
-cudaError_t launch_router_rows(const RouterRowsArgs &a, cudaStream_t st);
-// Top-k of logits [T][E] (T <= 16) and an L2 prefetch of the chosen experts' packed matrices
-// and the shared expert's; ids_out [T][k] may be null.
+// pdl: launched behind the previous kernel of the stream (programmatic dependent launch); the
+// kernel prefetches its rows into L2 before it waits for that kernel.
+cudaError_t launch_router_rows(const RouterRowsArgs &a, cudaStream_t st, bool pdl);
+// Top-k of logits [T][E] (T <= 16) into ids_out [T][k] (-1 for a row that is not finite).
 size_t lookahead_smem_bytes(int E);
-cudaError_t launch_lookahead(const float *logits, int T, int E, int k, int shared,
-                             const ExpertDev *experts, int H, int F, int32_t *ids_out,
+cudaError_t launch_lookahead(const float *logits, int T, int E, int k, int32_t *ids_out,
                              cudaStream_t st);
 cudaError_t launch_residual(const float *x, const float *res, float *x_out, int T, int H,
                             cudaStream_t st);

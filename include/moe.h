@@ -263,10 +263,12 @@ moe_status moe_forward_routed(const moe_arena *arena, const float *d_x, int T, i
  * d_x_out fp32 [T][hidden] receives x_L.  Every layer's arena has the same hidden size.  The
  * residual add and the normalisation are folded into the router kernel (one pass over x).
  * MOE_F_LOOKAHEAD (T <= 16): the router kernel of layer l also computes layer l+1's logits on
- * xn_l; a one-CTA kernel takes their top-k and prefetches those experts' packed rows (and the
- * shared expert's) into L2 before layer l runs -- the engine's router lookahead ("Strata - the
- * details", the STRATA_LOOKAHEAD paragraph), with L2 in place of the engine's VRAM cache.  A
- * wrong prediction costs only bandwidth: layer l+1 always routes on its own logits.
+ * xn_l; layer l's decode kernel takes their top-k (the prediction), and the router kernel of
+ * layer l+1 first prefetches the predicted experts' packed rows (and the shared expert's) into
+ * L2 from every SM, so that they are on chip when layer l+1 runs -- the engine's router
+ * lookahead ("Strata - the details", the STRATA_LOOKAHEAD paragraph), with L2 in place of the
+ * engine's VRAM cache.  A wrong prediction costs only bandwidth: layer l+1 always routes on its
+ * own logits.
  * Workspace: moe_chain_workspace_size for the same layers, T, k and flags.
  * trace (may be NULL; each pointer in it may be NULL) receives device copies of the
  * intermediates: the layers' inputs and the result, logits, ids, weights, gates, outputs and
