@@ -86,7 +86,7 @@ struct Smem {
 __host__ __device__ inline size_t smem_plan(int DA, int DB, int DR, uint32_t rawb) {
     return 1024 + (size_t)DA * kAStage + (size_t)DB * kBStage + 2 * kMStage + 2 * (size_t)kSStage +
            (size_t)DR * rawb + 2 * sizeof(TileInfo) +
-           8 * (2 * kMaxDR + 2 * kMaxDA + 2 * kMaxDB + 15) + 16;
+           8 * (2 * kMaxDR + 2 * kMaxDA + 2 * kMaxDB + 21) + 16;
 }
 
 __device__ __forceinline__ Smem carve(uint8_t *base, const GemmArgs &a) {
