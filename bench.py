@@ -564,8 +564,8 @@ def run_chain(name, args, world, dev):
         "expert_gbs": step_bytes / (ms_step / 1e3) / 1e9,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                      "frac": achieved / hbm, "traffic": None,
-                     "kernel": "the chained layer (k_router_rows + k_lookahead + "
-                               "k_decode_fused per layer): expert bytes per layer / layer time",
+                     "kernel": "the chained layer (k_router_rows + k_decode_fused per layer): "
+                               "expert bytes per layer / layer time",
                      "peak_source": f"{src} HBM copy"},
         "e2e": {"value": job_throughput(T * w.layers, k2, world, ms_e2e), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(x0.nbytes), "d2h_bytes_per_step": int(xo_h.numel() * 4),

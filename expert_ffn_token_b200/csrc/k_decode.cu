@@ -1107,17 +1107,19 @@ __device__ __forceinline__ void consumer(const DecParams &P, const Ctx &C) {
 // row of logits that is not finite predicts id -1 (nothing is prefetched for it; the next layer
 // reports the row).
 template <int VPL>
-__device__ __noinline__ void lookahead(const Lookahead A, int k, int t) {
+__device__ __noinline__ void lookahead(const float *logits, int E, int k, int32_t *ids_out, int t) {
     const int lane = threadIdx.x & 31;
     uint32_t key;
     int id;
-    const bool ok = topk_select<VPL>(A.logits + (size_t)t * A.E, A.E, k, key, id);
-    if (lane < k) A.ids_out[t * k + lane] = ok ? id : -1;
+    const bool ok = topk_select<VPL>(logits + (size_t)t * E, E, k, key, id);
+    if (lane < k) ids_out[t * k + lane] = ok ? id : -1;
 }
 
 // NT: activation rows per pass of rows_dot; TT: largest token count the down sums hold;
-// FK: format class of the arena; VPL: router logits per lane (E <= 32 * VPL).
-template <int NT, int TT, int FK, int VPL>
+// FK: format class of the arena; VPL: router logits per lane (E <= 32 * VPL); LOOK: the chain's
+// lookahead is compiled in (a separate instantiation: its code alone costs the plain layer half a
+// microsecond of register allocation).
+template <int NT, int TT, int FK, int VPL, bool LOOK>
 __global__ void __launch_bounds__(kThreads, 1) k_decode_fused(const DecParams P) {
     extern __shared__ __align__(128) uint8_t sm[];
     const int tid = threadIdx.x, warp = tid >> 5;
@@ -1180,8 +1182,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_fused(const DecParams P)
     C.i_lo = (int)((long long)P.H * cta / G);
     C.i_hi = (int)((long long)P.H * (cta + 1) / G);
 
-    if (P.look.logits && C.cta0 && warp < kCW && warp >= kCW - P.T)
-        lookahead<VPL>(P.look, P.k, kCW - 1 - warp);
+    if (LOOK && P.look.logits && C.cta0 && warp < kCW && warp >= kCW - P.T)
+        lookahead<VPL>(P.look.logits, P.look.E, P.k, P.look.ids_out, kCW - 1 - warp);
     if (C.s_misc[3]) {
         // the descriptor table did not arrive in time: no work here (this CTA's blocks are never
         // published, so the grid-wide waits of the others give up too); the copy lands first
@@ -1202,30 +1204,32 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_fused(const DecParams P)
     }
 }
 
-template <int NT, int TT, int FK, int VPL>
+template <int NT, int TT, int FK, int VPL, bool LOOK>
 cudaError_t launch_one(const cudaLaunchConfig_t &cfg, const DecParams &P) {
-    cudaError_t err = ensure_smem(k_decode_fused<NT, TT, FK, VPL>, (size_t)P.smem_bytes);
+    cudaError_t err = ensure_smem(k_decode_fused<NT, TT, FK, VPL, LOOK>, (size_t)P.smem_bytes);
     if (err != cudaSuccess) return err;
-    return cudaLaunchKernelEx(&cfg, k_decode_fused<NT, TT, FK, VPL>, P);
+    return cudaLaunchKernelEx(&cfg, k_decode_fused<NT, TT, FK, VPL, LOOK>, P);
 }
 
-template <int NT, int TT, int FK>
+template <int NT, int TT, int FK, bool LOOK = false>
 cudaError_t launch_vpl(const cudaLaunchConfig_t &cfg, const DecParams &P, int E) {
-    if (E <= 256) return launch_one<NT, TT, FK, 8>(cfg, P);
-    if (E <= 512) return launch_one<NT, TT, FK, 16>(cfg, P);
-    return launch_one<NT, TT, FK, 32>(cfg, P);
+    if (E <= 256) return launch_one<NT, TT, FK, 8, LOOK>(cfg, P);
+    if (E <= 512) return launch_one<NT, TT, FK, 16, LOOK>(cfg, P);
+    return launch_one<NT, TT, FK, 32, LOOK>(cfg, P);
 }
 
-template <int NT, int TT>
+template <int NT, int TT, bool LOOK = false>
 cudaError_t launch_fk(const cudaLaunchConfig_t &cfg, const DecParams &P, int fk, int E) {
-    if (fk == FK_Q4K) return launch_vpl<NT, TT, FK_Q4K>(cfg, P, E);
-    if (fk == FK_Q5K) return launch_vpl<NT, TT, FK_Q5K>(cfg, P, E);
-    return launch_vpl<NT, TT, FK_ANY>(cfg, P, E);
+    if (fk == FK_Q4K) return launch_vpl<NT, TT, FK_Q4K, LOOK>(cfg, P, E);
+    if (fk == FK_Q5K) return launch_vpl<NT, TT, FK_Q5K, LOOK>(cfg, P, E);
+    return launch_vpl<NT, TT, FK_ANY, LOOK>(cfg, P, E);
 }
 
-// Instantiations: batch class (1, <= 4, <= 16 tokens) x format class x top-k width; the
-// largest batch class exists only for the any-format kernel, to bound the code size.
+// Instantiations: batch class (1, <= 4, <= 16 tokens) x format class x top-k width, and the
+// single-token class again with the chain's lookahead.  The largest batch class exists only for
+// the any-format kernel, to bound the code size.
 cudaError_t launch_variant(const cudaLaunchConfig_t &cfg, const DecParams &P, int T, int fk, int E) {
+    if (T <= 1 && P.look.logits) return launch_fk<1, 1, true>(cfg, P, fk, E);
     if (T <= 1) return launch_fk<1, 1>(cfg, P, fk, E);
     if (T <= 4) return launch_fk<4, 4>(cfg, P, fk, E);
     return launch_vpl<4, 16, FK_ANY>(cfg, P, E);
@@ -1271,9 +1275,10 @@ cudaError_t launch_decode_fused(const FfnArgs &a, int E, int shared, const float
     P.slots = a.T * a.k + a.T;
     P.keep_h = a.h != nullptr;
     P.wait_ns = a.wait_ns;
-    // the lookahead runs inside when the next layer's logits fit this kernel's top-k width
+    // the lookahead runs inside (single-token batches) when the next layer's logits fit this
+    // kernel's top-k width
     const int top_width = E <= 256 ? 256 : E <= 512 ? 512 : 1024;
-    if (a.look.logits && a.look.ids_out && a.look.E <= top_width && a.T <= kCW) P.look = a.look;
+    if (a.look.logits && a.look.ids_out && a.look.E <= top_width && a.T <= 1) P.look = a.look;
     auto al = [](int v, int q) { return (v + q - 1) / q * q; };
     const int fk = a.fmt_mask == (1 << MOE_FMT_Q4_K) ? FK_Q4K
                    : a.fmt_mask == (1 << MOE_FMT_Q5_K) ? FK_Q5K : FK_ANY;
