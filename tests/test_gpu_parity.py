@@ -166,12 +166,19 @@ def test_layer_mtp_verify_full_size(torch, layer):
     check_layer(torch, w, layer, x, logits)
 
 
-def _sample_tokens(T, ids, n=24, seed=0):
+def _sample_tokens(T, ids, n=24, seed=0, every_expert=False):
+    """First and last tokens, the hottest expert's first and last tokens, with every_expert the
+    last token routed to each expert that has any (its tail tile on the grouped paths), and
+    random tokens up to n."""
     rng = np.random.default_rng(seed)
     hot = np.bincount(ids.ravel()).argmax()
     hot_tokens = np.nonzero((ids == hot).any(axis=1))[0]
     pick = {0, T - 1, int(hot_tokens[0]), int(hot_tokens[-1])}
-    pick |= set(int(t) for t in rng.choice(T, n - len(pick), replace=False))
+    if every_expert:
+        for e in np.unique(ids):
+            pick.add(int(np.nonzero((ids == e).any(axis=1))[0][-1]))
+    rest = [t for t in rng.permutation(T) if int(t) not in pick]
+    pick |= set(int(t) for t in rest[:max(0, n - len(pick))])
     return np.array(sorted(pick))
 
 
@@ -185,8 +192,10 @@ def test_layer_prefill_full_size_sampled(torch, name):
         # Zipf(1.3) popularity sampled k at a time without replacement (Gumbel top-k): a few
         # experts take > 1000 tokens, a long tail takes only a handful
         assert (counts > 1000).sum() >= 3 and (counts < 8).sum() >= 5 and (counts < 16).sum() >= 50
-    # every token's integer outputs (views) and a seeded sample of 512 tokens' layer outputs
-    check_layer(torch, w, 0, x, logits, tokens=_sample_tokens(w.tokens, ids, n=512))
+    # every token's integer outputs (views); the layer outputs of the last token of every expert
+    # (each expert's tail tile) and random tokens, 512 or more in all
+    check_layer(torch, w, 0, x, logits,
+                tokens=_sample_tokens(w.tokens, ids, n=512, every_expert=True))
 
 
 @pytest.mark.parametrize("T", [1, 2, 17, 65, 100, 300])
