@@ -53,7 +53,9 @@ struct StageMeta {
 struct JobX {                // a job with its expert's descriptor, cached in shared memory
     const uint8_t *m[3];
     uint32_t stride[3];
-    int fmt, expert, slot0, n, shared;
+    int fmt, expert, slot0, n;
+    short shared;
+    short by_n;               // the job in position u of the order by token count, descending
 };
 
 struct DecParams {
@@ -450,7 +452,7 @@ __device__ __forceinline__ ExpertDev *desc_table(uint8_t *sm, int E, int T, int 
 }
 
 // a1-a3 for the whole batch (every CTA; CTA 0 also stores the intermediates).
-template <int VPL>
+template <int VPL, int TT>
 __device__ __forceinline__ void prologue(const DecParams &P, Ctx &C, uint8_t *sm) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const WsLayout &L = P.L;
@@ -677,6 +679,19 @@ __device__ __forceinline__ void prologue(const DecParams &P, Ctx &C, uint8_t *sm
         C.s_stok[A + t] = t;
         C.s_sw[A + t] = P.gate ? P.gate[t] : 1.0f;
     }
+    // the jobs by token count, descending (stable): the gate/up blocks are dealt to the CTAs in
+    // this order, so that the heavy blocks spread over the grid (multi-token kernels)
+#pragma unroll 1
+    for (int u = tid; u < U && TT > 1; u += kThreads) {
+        const int n = s_jobs[u].n;
+        int pos = 0;
+#pragma unroll 1
+        for (int v = 0; v < U; v++) {
+            const int m = s_jobs[v].n;
+            pos += (m > n || (m == n && v < u)) ? 1 : 0;
+        }
+        s_jobs[pos].by_n = (short)u;
+    }
     bool desc_ok = true;
     if (tid < U && !ptx::mbar_wait_bounded(C.desc_bar, 0, desc_wait_ns(P))) {
         desc_ok = false;   // the table is not there: this CTA does no work
@@ -735,6 +750,7 @@ __device__ __forceinline__ bool ring_acquire(const DecParams &P, const Ctx &C, R
 }
 
 // One thread: stream this CTA's gate/up blocks, then its down rows, into the ring.
+template <int TT>
 __device__ __forceinline__ void producer(const DecParams &P, const Ctx &C) {
     const uint64_t pol = ptx::policy_evict_first();
     Ring R{0, 0u};
@@ -743,8 +759,11 @@ __device__ __forceinline__ void producer(const DecParams &P, const Ctx &C) {
     const JobX *s_jobs = C.s_jobs;
 #pragma unroll 1
     for (int mb = 0; mb < C.my_blocks && ok; mb++) {
-        const int blk = cta + mb * G;
-        const int ju = blk / C.nb32, b = blk % C.nb32;
+        // multi-token kernels: block i of the order by token count goes to CTA i mod G,
+        // serpentine (rounds of G blocks alternate direction), so that every CTA gets a mix of
+        // heavy and light blocks; single-token jobs all weigh the same: block i to CTA i mod G
+        const int blk = TT > 1 ? mb * G + ((mb & 1) ? G - 1 - cta : cta) : cta + mb * G;
+        const int ju = TT > 1 ? s_jobs[blk / C.nb32].by_n : blk / C.nb32, b = blk % C.nb32;
         const JobX &J = s_jobs[ju];
 #pragma unroll 1
         for (int half = 0; half < 2 && ok; half++) {
@@ -898,13 +917,62 @@ __device__ __forceinline__ bool wait_and_stage_h(const DecParams &P, const Ctx &
 // split the (job, chunk) pairs of a row; each pair is dotted with Q8_1(h) of every slot of its
 // job and added, weighted, into the lane's per-token sums.  The order of the sums is fixed, so
 // the result is deterministic; the lanes are reduced once, at the end of the unit.
+// Chunk p of job J in one down row: its dot with Q8_1(h) of every slot of the job, weighted and
+// added into acc[token].
+template <int TT, int FK>
+__device__ __forceinline__ void down_item(const DecParams &P, const Ctx &C, const uint8_t *row,
+                                          const JobX &J, int fmt, int p, float (&acc)[TT]) {
+    const int hb = C.hb;
+    if (FK == FK_ANY && small_block(fmt)) {
+        const bool q80 = fmt == MOE_FMT_Q8_0;
+#pragma unroll 1
+        for (int t = 0; t < J.n; t++) {
+            const int slot = J.slot0 + t;
+            const ActChunk a = load_act(C.s_hq + (size_t)slot * P.hpad, C.s_hd + slot * hb,
+                                        C.s_hs + slot * hb, p, true);
+            const float v = q80 ? q80_chunk_dot(row + (size_t)p * kQ80Bytes, a)
+                                : q51_chunk_dot(row + (size_t)p * kQ51Bytes, a);
+            const int tok = C.s_stok[slot];
+            const float wv = C.s_sw[slot] * v;
+#pragma unroll
+            for (int tt = 0; tt < TT; tt++)
+                if (tt == tok) acc[tt] += wv;
+        }
+    } else {
+        const int SBB = fmt == MOE_FMT_Q5_K ? kQ5KBytes : kQ4KBytes;
+        const int sb = p >> 3, j = p & 7;
+        const WChunk w = fmt == MOE_FMT_Q5_K ? kq_chunk<true>(row + (size_t)sb * SBB, j)
+                         : (FK == FK_ANY && fmt == MOE_FMT_Q6_K)
+                             ? q6_chunk(row + (size_t)sb * kQ6KBytes, j)
+                             : kq_chunk<false>(row + (size_t)sb * SBB, j);
+        const float mf = (j & 1) ? 0.f : 1.f;
+#pragma unroll 1
+        for (int t = 0; t < J.n; t++) {
+            const int slot = J.slot0 + t;
+            const ActChunk a = load_act(C.s_hq + (size_t)slot * P.hpad, C.s_hd + slot * hb,
+                                        C.s_hs + slot * hb, p, false);
+            const float v = kq_chunk_dot(w, a, mf);
+            const int tok = C.s_stok[slot];
+            const float wv = C.s_sw[slot] * v;
+#pragma unroll
+            for (int tt = 0; tt < TT; tt++)
+                if (tt == tok) acc[tt] += wv;
+        }
+    }
+}
+
+// rows <= kCW + 2 (split; multi-token kernels only): warp w computes row w over every item of the
+// stage and, when rows > kCW, its 1/kCW share of the items of the one or two rows past kCW
+// (their partial sums are added across warps at the end of the unit, in warp order).  Otherwise
+// warp w computes rows w and w + kCW over every item.  (The single-token kernel keeps the plain
+// form: code it never runs still costs it instruction fetches.)
 template <int TT, int FK>
 __device__ __forceinline__ void down_stage(const DecParams &P, const Ctx &C, const uint8_t *stage,
                                            int rows, int j0, int j1, float (&dacc)[2][TT]) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const bool split = TT > 1 && rows <= kCW + 2;
     const int kq_chunks = P.hpad / 32;          // K-quant rows: 16-byte chunks of 32 weights
     const int sm_chunks = (C.F + 31) / 32;      // Q8_0 / Q5_1 rows: one chunk per block
-    const int hb = C.hb;
     uint32_t base = 0;                          // offset of job g0 inside the stage
 #pragma unroll 1
     for (int g0 = j0; g0 < j1; g0 += 32) {
@@ -951,44 +1019,34 @@ __device__ __forceinline__ void down_stage(const DecParams &P, const Ctx &C, con
 #pragma unroll
             for (int rr = 0; rr < 2; rr++) {
                 const int r = warp + kCW * rr;
-                if (r >= rows) break;
-                const uint8_t *row = stage + joff + (size_t)r * J.stride[2];
-                if (FK == FK_ANY && small_block(fmt)) {
-                    const bool q80 = fmt == MOE_FMT_Q8_0;
+                if (r >= rows || (split && rr > 0)) break;
+                down_item<TT, FK>(P, C, stage + joff + (size_t)r * J.stride[2], J, fmt, p, dacc[rr]);
+            }
+        }
+        if (split && rows > kCW) {
+            // the rows past kCW: lanes 0-15 take row kCW, lanes 16-31 row kCW + 1, and warp w the
+            // items [w * per, (w + 1) * per) of the group; partial sums in dacc[1]
+            const int e = lane >> 4, li = lane & 15;
+            const int per = (total + kCW - 1) / kCW;
 #pragma unroll 1
-                    for (int t = 0; t < J.n; t++) {
-                        const int slot = J.slot0 + t;
-                        const ActChunk a = load_act(C.s_hq + (size_t)slot * P.hpad, C.s_hd + slot * hb,
-                                                    C.s_hs + slot * hb, p, true);
-                        const float v = q80 ? q80_chunk_dot(row + (size_t)p * kQ80Bytes, a)
-                                            : q51_chunk_dot(row + (size_t)p * kQ51Bytes, a);
-                        const int tok = C.s_stok[slot];
-                        const float wv = C.s_sw[slot] * v;
-#pragma unroll
-                        for (int tt = 0; tt < TT; tt++)
-                            if (tt == tok) dacc[rr][tt] += wv;
-                    }
+            for (int q0 = 0; q0 < per; q0 += 16) {
+                const int f = warp * per + q0 + li;
+                const bool act = q0 + li < per && f < total && kCW + e < rows;
+                int jl = 0;
+                if (FK != FK_ANY) {
+                    jl = f / kq_chunks;
                 } else {
-                    const int SBB = fmt == MOE_FMT_Q5_K ? kQ5KBytes : kQ4KBytes;
-                    const int sb = p >> 3, j = p & 7;
-                    const WChunk w = fmt == MOE_FMT_Q5_K ? kq_chunk<true>(row + (size_t)sb * SBB, j)
-                                     : (FK == FK_ANY && fmt == MOE_FMT_Q6_K)
-                                         ? q6_chunk(row + (size_t)sb * kQ6KBytes, j)
-                                         : kq_chunk<false>(row + (size_t)sb * SBB, j);
-                    const float mf = (j & 1) ? 0.f : 1.f;
 #pragma unroll 1
-                    for (int t = 0; t < J.n; t++) {
-                        const int slot = J.slot0 + t;
-                        const ActChunk a = load_act(C.s_hq + (size_t)slot * P.hpad, C.s_hd + slot * hb,
-                                                    C.s_hs + slot * hb, p, false);
-                        const float v = kq_chunk_dot(w, a, mf);
-                        const int tok = C.s_stok[slot];
-                        const float wv = C.s_sw[slot] * v;
-#pragma unroll
-                        for (int tt = 0; tt < TT; tt++)
-                            if (tt == tok) dacc[rr][tt] += wv;
-                    }
+                    for (int l = 0; l < ng - 1; l++)
+                        if (f >= __shfl_sync(kFullMask, cend, l)) jl = l + 1;
                 }
+                const int cbeg = __shfl_sync(kFullMask, cend - nch, jl & 31);
+                const uint32_t joff = __shfl_sync(kFullMask, off, jl & 31);
+                if (!act) continue;
+                const JobX &J = C.s_jobs[g0 + jl];
+                const int fmt = FK == FK_Q4K ? MOE_FMT_Q4_K : FK == FK_Q5K ? MOE_FMT_Q5_K : J.fmt;
+                down_item<TT, FK>(P, C, stage + joff + (size_t)(kCW + e) * J.stride[2], J, fmt,
+                                  f - cbeg, dacc[1]);
             }
         }
         base = __shfl_sync(kFullMask, off + sz, ng - 1);
@@ -1077,15 +1135,45 @@ __device__ __forceinline__ void consumer(const DecParams &P, const Ctx &C) {
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(&C.empty[s]);
             if (m.e && !skip_down) {   // last stage of the unit: reduce across the lanes, write
+                const bool split = TT > 1 && rows <= kCW + 2;
 #pragma unroll
                 for (int rr = 0; rr < 2; rr++) {
                     const int r = warp + kCW * rr;
-                    if (r >= rows) break;
+                    if (r >= rows || (split && rr > 0)) break;
 #pragma unroll
                     for (int t = 0; t < TT; t++) {
                         if (t >= C.T) break;
                         const float v = warp_sum(dacc[rr][t]);
                         if (lane == 0) P.out[(size_t)t * H + i0 + r] = v;
+                    }
+                }
+                if (split && rows > kCW) {
+                    // the rows past kCW: each half-warp's partials into s_h ([kCW][2][TT], free
+                    // in the down phase); the last warp to arrive adds them in warp order (no
+                    // warp waits for another here)
+                    float *part = C.s_h;
+#pragma unroll
+                    for (int t = 0; t < TT; t++) {
+                        float v = dacc[1][t];
+#pragma unroll
+                        for (int o = 8; o >= 1; o >>= 1) v += __shfl_xor_sync(kFullMask, v, o);
+                        if ((lane & 15) == 0) part[(warp * 2 + (lane >> 4)) * TT + t] = v;
+                    }
+                    __threadfence_block();
+                    __syncwarp();
+                    int last = 0;
+                    if (lane == 0) last = atomicAdd(&C.s_misc[8], 1) == kCW - 1;
+                    last = __shfl_sync(kFullMask, last, 0);
+                    if (last) {
+                        __threadfence_block();
+                        const int e = lane >> 4, t = lane & 15;
+                        if (kCW + e < rows && t < C.T) {
+                            float v = 0.f;
+#pragma unroll 1
+                            for (int w = 0; w < kCW; w++) v += part[(w * 2 + e) * TT + t];
+                            P.out[(size_t)t * H + i0 + kCW + e] = v;
+                        }
+                        if (lane == 0) C.s_misc[8] = 0;
                     }
                 }
             }
@@ -1163,6 +1251,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_fused(const DecParams P)
         C.s_misc[2] = 0;
         C.s_misc[3] = 0;
         C.s_misc[5] = 0;
+        C.s_misc[8] = 0;
         // the descriptor table is the arena's (not written by the previous kernel): fetch it
         // now, in the background, before waiting for the previous grid
         const uint32_t nb = (uint32_t)((P.E + P.shared) * sizeof(ExpertDev));
@@ -1172,12 +1261,19 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_fused(const DecParams P)
     }
     ptx::grid_dependency_wait();
     ptx::launch_dependents();
-    prologue<VPL>(P, C, sm);
+    prologue<VPL, TT>(P, C, sm);
     // the prologue scratch in the stage ring is dead from here on
     const int G = gridDim.x, cta = blockIdx.x;
     C.U = C.s_misc[0];
     C.n_blk = C.U * C.nb32;
-    C.my_blocks = C.n_blk / G + (cta < C.n_blk % G ? 1 : 0);
+    if (TT > 1) {
+        C.my_blocks = 0;
+#pragma unroll 1
+        for (int r = 0; r * G < C.n_blk; r++)
+            C.my_blocks += r * G + ((r & 1) ? G - 1 - cta : cta) < C.n_blk ? 1 : 0;
+    } else {
+        C.my_blocks = C.n_blk / G + (cta < C.n_blk % G ? 1 : 0);
+    }
     // down rows: computed after the barrier by every CTA, so split evenly
     C.i_lo = (int)((long long)P.H * cta / G);
     C.i_hi = (int)((long long)P.H * (cta + 1) / G);
@@ -1189,7 +1285,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_fused(const DecParams P)
         // published, so the grid-wide waits of the others give up too); the copy lands first
         if (tid == 0) ptx::mbar_wait_bounded(C.desc_bar, 0, 50000000ull);
     } else if (warp == kCW) {
-        if ((tid & 31) == 0) producer(P, C);
+        if ((tid & 31) == 0) producer<TT>(P, C);
     } else {
         consumer<NT, TT, FK>(P, C);
     }
