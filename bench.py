@@ -239,12 +239,17 @@ def run_workload(name, args, world, dev):
         step_ops += o
         distinct.append(u)
 
-    def one_step(events=None):
+    # prefill: the gate/up phase on kind::i8 products (the default) or on exact kind::f16
+    # products (timed beside it)
+    main_flags = 0 if decode else moe.F_TC_I8
+
+    def one_step(events=None, flags=None):
+        fl = main_flags if flags is None else flags
         for l in range(w.layers):
             if events is not None:
                 moe.set_timing_events(handles[l], *[e.cuda_event for e in events[l]])
             moe.forward(handles[l], x_d[l].data_ptr(), lg_d[l].data_ptr(), T, w.k,
-                        out_d[l].data_ptr(), ws.data_ptr(), ws_bytes, 0,
+                        out_d[l].data_ptr(), ws.data_ptr(), ws_bytes, fl,
                         torch.cuda.current_stream().cuda_stream)
 
     # decode: one step (the layers' single launches) captured in a CUDA graph.  Prefill: eager
@@ -314,6 +319,26 @@ def run_workload(name, args, world, dev):
         dist.barrier()
     clock_rows = clocks.stop()
 
+    # prefill: the other gate/up kernel on the same inputs, same steps (its own warm-up)
+    alt = None
+    if not decode:
+        for _ in range(W):
+            one_step(flags=0)
+        torch.cuda.synchronize()
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record()
+        for i in range(K):
+            one_step(step_events[i], flags=0)
+        g1.record()
+        torch.cuda.synchronize()
+        for h in handles:
+            moe.set_timing_events(h)
+        alt = {"ms": max_over_ranks(g0.elapsed_time(g1), world, dev),
+               "gateup_ms": statistics.mean(t[0].elapsed_time(t[1])
+                                            for row in step_events for t in row),
+               "down_ms": statistics.mean(t[1].elapsed_time(t[2])
+                                          for row in step_events for t in row)}
+
     # end to end through the C ABI, eagerly: pinned host inputs in, every layer's moe_forward,
     # the result out, every step
     x_h = torch.from_numpy(xs).pin_memory()
@@ -378,19 +403,31 @@ def run_workload(name, args, world, dev):
                     "kernel": "k_decode_fused (one launch per layer)",
                     "peak_source": f"{src} HBM copy", "bytes_per_launch": bytes_per_layer}
     else:
-        # dominant kernel: the gate/up grouped GEMM (k_gemm_tc<0>); 2 flops per multiply-add
+        # dominant kernel: the gate/up grouped GEMM on int8 products (k_gateup_i8), against the
+        # int8 dense peak; 2 ops per multiply-add
         assign = T * (w.k + (1 if w.shared else 0))
         flops = 2.0 * assign * 2 * w.ffn * w.hidden
         achieved = flops / (gateup_ms / 1e3) / 1e12
-        roofline = {"bound": "tensor", "achieved": achieved, "peak": bf16, "unit": "TFLOP/s",
-                    "frac": achieved / bf16, "traffic": traffic_for("k_gateup_tc", name),
-                    "kernel": "k_gateup_tc (gate/up grouped GEMM, tcgen05 kind::f16: exact integer "
-                              "weight operands, hi/lo activation planes), one launch per layer",
-                    "peak_source": f"{src} bf16 dense (fp16 runs at the same rate)",
-                    "flops_per_launch": flops, "ms_per_launch": gateup_ms,
-                    "frac_of_int8_peak": achieved / int8_meas,
+        roofline = {"bound": "tensor", "achieved": achieved, "peak": int8_meas, "unit": "TOP/s",
+                    "frac": achieved / int8_meas, "traffic": traffic_for("k_gateup_i8", name),
+                    "kernel": "k_gateup_i8 (gate/up grouped GEMM, tcgen05 kind::i8: one s32 "
+                              "accumulator per 32-weight block, promoted in fp32), one launch "
+                              "per layer",
+                    "peak_source": f"int8 dense = 2 x {src} bf16 dense ({bf16:.1f} TFLOP/s)",
+                    "ops_per_launch": flops, "ms_per_launch": gateup_ms,
+                    "frac_of_bf16_peak": achieved / bf16,
                     "down_ms_per_launch": down_ms,
                     "down_note": "k_h_rows + k_down_tc, from the events around the down phase"}
+        f16_ach = flops / (alt["gateup_ms"] / 1e3) / 1e12
+        alt_layer_s = alt["ms"] / K / 1e3 / w.layers
+        roofline["f16_variant"] = {
+            "kernel": "k_gateup_tc (tcgen05 kind::f16: exact integer weight operands, hi/lo "
+                      "activation planes), timed on the same inputs after the main loop",
+            "ms_per_launch": alt["gateup_ms"], "achieved_tflops": f16_ach,
+            "frac_of_bf16_peak": f16_ach / bf16, "frac_of_int8_peak": f16_ach / int8_meas,
+            "traffic": traffic_for("k_gateup_tc", name),
+            "down_ms_per_launch": alt["down_ms"], "us_per_layer": 1e6 * alt_layer_s,
+            "value": job_throughput(T * w.layers, K, world, alt["ms"]), "unit": "tokens/s"}
     res = {
         "workload": w.note, "value": job_throughput(tok_per_step, K, world, ms),
         "unit": "tokens/s", "steps": K, "warmup": W, "ms_per_step": ms_step,

@@ -26,8 +26,8 @@ ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",
          "--expt-relaxed-constexpr", f"-I{INCLUDE}", f"-I{CSRC}"]
 
-LIB_SOURCES = ["k_route.cu", "k_ffn.cu", "k_decode.cu", "k_gateup_tc.cu", "k_down_tc.cu",
-               "k_router.cu", "moe_api.cu", "moe_noalloc.cu"]
+LIB_SOURCES = ["k_route.cu", "k_ffn.cu", "k_decode.cu", "k_gateup_tc.cu", "k_gateup_i8.cu",
+               "k_down_tc.cu", "k_router.cu", "moe_api.cu", "moe_noalloc.cu"]
 OPTIONAL_SOURCES: list[str] = []
 SYNTH_SOURCES = ["synth_fill.cu"]
 

@@ -779,7 +779,10 @@ size_t tc_smem_bytes(int fmt_mask) {
     if (!ring_plan(fmt_mask, DA, DB, DR)) return (size_t)-1;
     const size_t down = smem_plan(DA, DB, DR, raw_bytes(fmt_mask));
     const size_t gu = tc_gateup_smem_bytes(fmt_mask);
-    return gu == (size_t)-1 ? gu : (down > gu ? down : gu);
+    const size_t gi = tc_gateup_i8_smem_bytes(fmt_mask);
+    if (gu == (size_t)-1 || gi == (size_t)-1) return (size_t)-1;
+    const size_t m = down > gu ? down : gu;
+    return m > gi ? m : gi;
 }
 
 // The tensor-core phases of one layer: gate/up (k_gateup_tc.cu), then the down operand and the
@@ -787,7 +790,7 @@ size_t tc_smem_bytes(int fmt_mask) {
 cudaError_t launch_gemm_tc(const TcPhaseArgs &p, cudaStream_t st) {
     const int grid = sm_count();
     if (grid <= 0) return cudaErrorInvalidDevice;
-    if (p.phase == 0) return launch_gateup_tc(p, grid, st);
+    if (p.phase == 0) return p.i8 ? launch_gateup_i8(p, grid, st) : launch_gateup_tc(p, grid, st);
     const FfnArgs &f = p.ffn;
     GemmArgs a{};
     a.wmaps = reinterpret_cast<const CUtensorMap *>(p.wmaps);

@@ -475,6 +475,7 @@ static moe_status forward_impl(const moe_arena *arena, const float *d_x, const f
         p.wmaps = arena->d_wmaps;
         p.slots = L.slots;
         p.keep_h = (flags & MOE_F_KEEP_H) ? 1 : 0;
+        p.i8 = (flags & MOE_F_TC_I8) ? 1 : 0;
         p.Kd = L.kd;
         p.xh = reinterpret_cast<const __half *>(ws + L.xh);
         p.xl = reinterpret_cast<const __half *>(ws + L.xl);

@@ -218,6 +218,7 @@ struct TcPhaseArgs {
     FfnArgs ffn;
     const void *wmaps;          // device array of the experts' weight tensor maps
     int phase, slots, keep_h;
+    int i8;                     // gate/up on kind::i8 MMAs (k_gateup_i8) instead of kind::f16
     int Kd;                     // down contraction length: ffn rounded up to 64
     const __half *xh, *xl;      // [T][H] fp16 planes, x^ * 2^-e = hi + lo exactly
     const float *xsh, *xsl;     // [T][H/32] block sums xd * sum(q) * 2^-e, tf32 hi + lo
@@ -238,6 +239,10 @@ size_t tc_gateup_smem_bytes(int fmt_mask);
 // One tensor-core phase (phase 0: k_gateup_tc, phase 1: k_down_tc).
 cudaError_t launch_gemm_tc(const TcPhaseArgs &p, cudaStream_t st);
 cudaError_t launch_gateup_tc(const TcPhaseArgs &p, int grid, cudaStream_t st);
+// The gate/up phase with 8-bit integer products and a promotion per 32-weight block
+// (k_gateup_i8.cu), and its shared memory ((size_t)-1: no plan fits).
+cudaError_t launch_gateup_i8(const TcPhaseArgs &p, int grid, cudaStream_t st);
+size_t tc_gateup_i8_smem_bytes(int fmt_mask);
 // a1 per token for the tensor-core path: the Q8_1 blocks (as moe_quantize_act) plus the gate/up
 // operand planes, the block sums and 2^e.
 cudaError_t launch_quant_rows(const float *x, int T, int H, int8_t *xq, uint16_t *xd,

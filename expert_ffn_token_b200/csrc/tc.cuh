@@ -1,6 +1,6 @@
 // tc.cuh -- inline-PTX wrappers for the sm_100a tensor-core path: tiled TMA loads (tensor maps),
-// tensor-memory allocation, tcgen05.mma (kind::f16 and kind::tf32, operands in shared memory,
-// accumulator in tensor memory), commits to mbarriers and tensor-memory loads.
+// tensor-memory allocation, tcgen05.mma (kind::f16, kind::tf32 and kind::i8, operands in shared
+// memory, accumulator in tensor memory), commits to mbarriers and tensor-memory loads.
 #pragma once
 
 #include <stdint.h>
@@ -88,6 +88,17 @@ __device__ __forceinline__ void umma_tf32(uint32_t d_tmem, uint64_t a_desc, uint
         : "memory");
 }
 
+// Same with signed 8-bit integer inputs and an s32 accumulator (K = 32 per instruction).
+__device__ __forceinline__ void umma_i8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                        uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // Arrive once on `bar` when every MMA issued so far by this thread has completed.
 __device__ __forceinline__ void umma_commit(uint64_t *bar) {
     asm volatile(
@@ -138,6 +149,15 @@ __device__ __forceinline__ void tmem_ld_wait(uint32_t (&r)[16]) {
 }
 __device__ __forceinline__ void tmem_ld_wait() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+// Orders later uses of r after the preceding (volatile) wait, for a 16-register set.
+__device__ __forceinline__ void reg_tie(uint32_t (&r)[16]) {
+    asm volatile(""
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
+                   "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
+                   "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15])
+                 :
+                 : "memory");
 }
 // Orders later uses of r after the preceding (volatile) wait: a second register set loaded
 // before one tmem_ld_wait(r0) is tied with this.
@@ -190,6 +210,15 @@ __host__ __device__ constexpr uint32_t instr_desc(uint32_t ab_format, int M, int
            | (ab_format << 10)             // B format
            | ((uint32_t)(N >> 3) << 17)    // N / 8
            | ((uint32_t)(M >> 4) << 24);   // M / 16
+}
+
+// Instruction descriptor of kind::i8: both operands signed 8-bit, K-major, s32 accumulator.
+__host__ __device__ constexpr uint32_t instr_desc_i8(int M, int N) {
+    return (2u << 4)                       // D format s32
+           | (1u << 7)                     // A signed
+           | (1u << 10)                    // B signed
+           | ((uint32_t)(N >> 3) << 17)
+           | ((uint32_t)(M >> 4) << 24);
 }
 
 }  // namespace ptx

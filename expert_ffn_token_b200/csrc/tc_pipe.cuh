@@ -30,12 +30,16 @@ struct GemmArgs {
     const __half *act_lo;         // gate/up: x^ lo [T][H] (x^ = hi + lo exactly)
     const float *xs_hi, *xs_lo;   // gate/up: block sums xd * sum(q) [T][H/32], tf32 hi + lo
     const float *act_scale;       // 2^e per row of act
+    const int8_t *xq;             // gate/up, kind::i8: Q8_1 quants of x [T][H]
+    const uint16_t *xd;           //   their fp16 block scales [T][H/32]
+    const float *xsum;            //   block sums xd * sum(q) [T][H/32]
     int act_pitch;                // elements per row of act
     int T, k, H, F, hpad;
     int nst;                      // 64-wide contraction stages per tile
     int mt_count;                 // weight-row tiles per token slice
     int tn;                       // tokens per tile
     int DA, DB, DR, lag;          // ring depths and activation stages in flight
+    int DK, DC;                   // kind::i8 gate/up: row-constant and column-constant rings
     uint32_t rawb;                // bytes of one packed stage (128 rows x largest super-block)
     // gate/up outputs: Q8_1(h) per slot, optional fp32 h
     int8_t *hq;

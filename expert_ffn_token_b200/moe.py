@@ -30,6 +30,7 @@ F_FORCE_DECODE = 2
 F_FORCE_PREFILL = 4
 F_KEEP_H = 8
 F_LOOKAHEAD = 16
+F_TC_I8 = 32
 
 EXPORTED = ["moe_arena_create", "moe_arena_destroy", "moe_workspace_size", "moe_quantize_act",
             "moe_route_workspace_size", "moe_route_topk", "moe_forward", "moe_ws_views",

@@ -113,6 +113,9 @@ void moe_arena_destroy(moe_arena *arena);
 #define MOE_F_KEEP_H 8u          /* also store fp32 h (SwiGLU output) in the workspace       */
 #define MOE_F_LOOKAHEAD 16u      /* moe_chain_forward: prefetch the next layer's predicted
                                     experts into L2 while a layer runs (batches of <= 16)    */
+#define MOE_F_TC_I8 32u          /* tensor-core path: gate/up as 8-bit integer products
+                                    (tcgen05 kind::i8, one s32 accumulator per 32-weight block,
+                                    promoted in fp32) instead of exact kind::f16 products     */
 
 /* Bytes of device workspace moe_forward needs for up to max_tokens tokens, k routed experts
  * per token and the given flags.  The workspace is caller-owned scratch, 256-byte aligned. */
