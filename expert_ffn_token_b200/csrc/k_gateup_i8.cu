@@ -25,11 +25,11 @@
 //                prefetch two super-blocks ahead
 //   warp 1       tensor-memory allocation and the MMA issuer: per 32-weight block two MMAs (gate,
 //                up) into one of four rotating accumulator slots of 64 + 64 columns
-//   warp 2       unpack: lane u holds rows u + 32 i (i = 0..3) of gate and of up: the int8
+//   warp 2       loader: the tile's token rows of Q8_1(x) gathered with 16-byte cp.async, per
+//                stage the columns' block scales and block sums (loaded a stage ahead), and the
+//                block constants (s_b, -wm_b) of rows lane + 32 i read from the packed rows
+//   warp 3       unpack: lane u holds rows u + 32 i (i = 0..3) of gate and of up: their int8
 //                operands of every 128-wide stage
-//   warp 3       loader: the tile's token rows of Q8_1(x) gathered with 16-byte cp.async; per
-//                stage the columns' block scales and block sums, and the rows' block constants
-//                (s_b, -wm_b) read from the packed rows
 //   warps 4-19   epilogue: four warps per tensor-memory lane quarter, 16 tokens each: promotion,
 //                SwiGLU, Q8_1(h)
 // Every hand-off is an mbarrier; every wait is bounded and a timeout ends the kernel with
@@ -47,10 +47,11 @@ using namespace ptx;
 using namespace tcp;
 
 constexpr int kTN = 64;                              // tokens per tile
-constexpr int kUnpackWarp = 2;
-constexpr int kLoadWarp = 3;
+constexpr int kLoadWarp = 2;
+constexpr int kUnpackWarp = 3;
 constexpr int kEpiWarp0 = 4;
-constexpr int kEpiWarps = 16;
+constexpr int kEpiCols = 16;                         // tokens per epilogue warp
+constexpr int kEpiWarps = 4 * kTN / kEpiCols;        // four lane quarters x the tile's tokens
 constexpr int kThreads = (kEpiWarp0 + kEpiWarps) * 32;   // 640: five warps per scheduler
 constexpr uint32_t kAtomA = 16384;                   // 128 rows x 128 int8
 constexpr uint32_t kAStage = 2 * kAtomA;             // gate, up
@@ -112,37 +113,6 @@ __device__ __forceinline__ Smem carve(uint8_t *base, const GemmArgs &a) {
     return s;
 }
 
-// ---------------------------------------------------------------- packed fp32 pairs
-
-__device__ __forceinline__ uint64_t pk(float lo, float hi) {
-    uint64_t r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-    return r;
-}
-__device__ __forceinline__ uint64_t pku(uint32_t lo, uint32_t hi) {
-    uint64_t r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
-    return r;
-}
-__device__ __forceinline__ void unpk(uint64_t v, float &lo, float &hi) {
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-}
-__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
-    uint64_t r;
-    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-    return r;
-}
-__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
-    uint64_t r;
-    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-    return r;
-}
-__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
-    uint64_t r;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
-    return r;
-}
-
 // ---------------------------------------------------------------- warp 0: weight producer
 
 __device__ void role_producer(const GemmArgs &a, const Smem &S, int nj, Ring &rr, int &issued) {
@@ -172,7 +142,7 @@ __device__ void role_producer(const GemmArgs &a, const Smem &S, int nj, Ring &rr
     }
 }
 
-// ---------------------------------------------------------------- warp 2: unpack
+// ---------------------------------------------------------------- warp 3: unpack
 
 // Four bits t0..t3 of t to the low bit of bytes 0..3 (the four partial products land on
 // distinct bits, so nothing carries).
@@ -277,8 +247,8 @@ __device__ __forceinline__ void row_consts(const uint8_t *rowp, int hs, float (&
 
 template <int FMT>
 __device__ __forceinline__ bool unpack_sb(const GemmArgs &a, const Smem &S, Ring &ra,
-                                          const uint8_t *gbase, const uint8_t *ubase,
-                                          uint32_t sbb, int u) {
+                                          const uint8_t *gb, const uint8_t *ub, uint32_t sbb) {
+    const int u = threadIdx.x & 31;
 #pragma unroll 1
     for (int hs = 0; hs < 2; hs++) {
         if (!waitw(a, S.abort, S.a_empty + ra.s, ra.ph ^ 1u)) return false;
@@ -287,9 +257,9 @@ __device__ __forceinline__ bool unpack_sb(const GemmArgs &a, const Smem &S, Ring
         for (int i = 0; i < 4; i++) {
             const int r = u + 32 * i;
             uint32_t v[32];
-            i8_stage<FMT>(gbase + (size_t)r * sbb, hs, v);
+            i8_stage<FMT>(gb + (size_t)r * sbb, hs, v);
             store_row(as, r, v);
-            i8_stage<FMT>(ubase + (size_t)r * sbb, hs, v);
+            i8_stage<FMT>(ub + (size_t)r * sbb, hs, v);
             store_row(as + kAtomA, r, v);
         }
         fence_proxy_async_smem();
@@ -301,7 +271,7 @@ __device__ __forceinline__ bool unpack_sb(const GemmArgs &a, const Smem &S, Ring
 }
 
 __device__ void role_unpack(const GemmArgs &a, const Smem &S, int nj) {
-    const int u = threadIdx.x & 31;          // rows u + 32 i
+    const int u = threadIdx.x & 31;
     Cursor cur;
     Ring rr, ra;
     const int nsb = a.H / 256;
@@ -317,10 +287,10 @@ __device__ void role_unpack(const GemmArgs &a, const Smem &S, int nj) {
             const uint8_t *gb = S.raw + (size_t)rr.s * a.rawb;
             const uint8_t *ub = S.raw + (size_t)ru.s * a.rawb;
             bool ok;
-            if (t.fmt == MOE_FMT_Q4_K) ok = unpack_sb<MOE_FMT_Q4_K>(a, S, ra, gb, ub, sbb, u);
-            else if (t.fmt == MOE_FMT_Q5_K) ok = unpack_sb<MOE_FMT_Q5_K>(a, S, ra, gb, ub, sbb, u);
-            else if (t.fmt == MOE_FMT_Q8_0) ok = unpack_sb<MOE_FMT_Q8_0>(a, S, ra, gb, ub, sbb, u);
-            else ok = unpack_sb<MOE_FMT_Q5_1>(a, S, ra, gb, ub, sbb, u);
+            if (t.fmt == MOE_FMT_Q4_K) ok = unpack_sb<MOE_FMT_Q4_K>(a, S, ra, gb, ub, sbb);
+            else if (t.fmt == MOE_FMT_Q5_K) ok = unpack_sb<MOE_FMT_Q5_K>(a, S, ra, gb, ub, sbb);
+            else if (t.fmt == MOE_FMT_Q8_0) ok = unpack_sb<MOE_FMT_Q8_0>(a, S, ra, gb, ub, sbb);
+            else ok = unpack_sb<MOE_FMT_Q5_1>(a, S, ra, gb, ub, sbb);
             if (!ok) return;
             __syncwarp();
             if (u == 0) {
@@ -368,7 +338,42 @@ __device__ void role_mma(const GemmArgs &a, const Smem &S, int nj, uint32_t tbas
     }
 }
 
-// ---------------------------------------------------------------- warp 3: loader
+// ---------------------------------------------------------------- warp 2: loader
+
+__device__ __forceinline__ int column_token(const GemmArgs &a, const Tile &t, int n) {
+    if (n >= t.n_valid) return -1;
+    const int slot = t.slot_base + n;
+    return t.shared ? slot - a.T * a.k : a.perm[slot] / a.k;
+}
+
+// The scales and block sums of blocks 4 st .. 4 st + 3 of token tok (0 for no token, so that
+// padded columns add nothing).
+struct ColConsts {
+    uint2 d;
+    float4 s;
+};
+__device__ __forceinline__ ColConsts col_consts(const GemmArgs &a, int tok, int st) {
+    ColConsts c;
+    c.d = make_uint2(0u, 0u);
+    c.s = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    if (tok >= 0) {
+        const int H32 = a.H / 32;
+        c.d = *reinterpret_cast<const uint2 *>(a.xd + (size_t)tok * H32 + 4 * st);
+        c.s = *reinterpret_cast<const float4 *>(a.xsum + (size_t)tok * H32 + 4 * st);
+    }
+    return c;
+}
+
+__device__ __forceinline__ void store_cols(float *cc, int n, const ColConsts &c) {
+    cc[0 * kTN + n] = half_bits_to_float(c.d.x);
+    cc[1 * kTN + n] = half_bits_to_float(c.d.x >> 16);
+    cc[2 * kTN + n] = half_bits_to_float(c.d.y);
+    cc[3 * kTN + n] = half_bits_to_float(c.d.y >> 16);
+    cc[4 * kTN + 0 * kTN + n] = c.s.x;
+    cc[4 * kTN + 1 * kTN + n] = c.s.y;
+    cc[4 * kTN + 2 * kTN + n] = c.s.z;
+    cc[4 * kTN + 3 * kTN + n] = c.s.w;
+}
 
 // The block constants of stage hs for rows lane + 32 i of gate and up, into a constant stage.
 template <int FMT>
@@ -385,12 +390,6 @@ __device__ __forceinline__ void consts_stage(const uint8_t *gb, const uint8_t *u
     }
 }
 
-__device__ __forceinline__ int column_token(const GemmArgs &a, const Tile &t, int n) {
-    if (n >= t.n_valid) return -1;
-    const int slot = t.slot_base + n;
-    return t.shared ? slot - a.T * a.k : a.perm[slot] / a.k;
-}
-
 __device__ void role_loader(const GemmArgs &a, const Smem &S, int nj) {
     const int lane = threadIdx.x & 31;
     const int c = lane & 7;                      // 16-byte chunk of a 128-byte row
@@ -400,7 +399,6 @@ __device__ void role_loader(const GemmArgs &a, const Smem &S, int nj) {
     int npend = 0;
     bool ok = true;
     const int nsb = a.H / 256;
-    const int H32 = a.H / 32;
     for (int i = blockIdx.x; ok; i += gridDim.x) {
         Tile t;
         if (!tile_at(a, nj, cur, i, t)) break;
@@ -409,6 +407,7 @@ __device__ void role_loader(const GemmArgs &a, const Smem &S, int nj) {
         int src[16];                             // this lane's gather rows
 #pragma unroll
         for (int j = 0; j < 16; j++) src[j] = column_token(a, t, rg + 4 * j);
+        ColConsts n0 = col_consts(a, tok0, 0), n1 = col_consts(a, tok1, 0);
         ob = rb;
         auto signal_oldest = [&]() {
             if (lane == 0) mbar_arrive(S.b_full + ob.s);
@@ -416,17 +415,10 @@ __device__ void role_loader(const GemmArgs &a, const Smem &S, int nj) {
             npend--;
         };
         for (int sb = 0; sb < nsb && ok; sb++) {
-            Ring ru = rr;
-            ru.adv(1, a.DR);
-            if (!(ok = waitw(a, S.abort, S.raw_full + rr.s, rr.ph))) break;
-            if (!(ok = waitw(a, S.abort, S.raw_full + ru.s, ru.ph))) break;
-            const uint8_t *gb = S.raw + (size_t)rr.s * a.rawb;
-            const uint8_t *ub = S.raw + (size_t)ru.s * a.rawb;
             for (int hs = 0; hs < 2 && ok; hs++) {
                 const int st = 2 * sb + hs;
-                // the token rows of this 128-wide stage first: its copies are in flight while
-                // the constants below are written, and the oldest stage is signalled before any
-                // wait on a ring that the epilogue frees
+                // the token rows of this 128-wide stage first: the oldest stage in flight is
+                // signalled before the waits below on rings that the epilogue frees
                 if (!(ok = waitw(a, S.abort, S.b_empty + rb.s, rb.ph ^ 1u))) break;
                 uint8_t *bs = S.B + (size_t)rb.s * kBStage;
                 const int8_t *col = a.xq + 128 * st + 16 * c;
@@ -449,43 +441,29 @@ __device__ void role_loader(const GemmArgs &a, const Smem &S, int nj) {
                     __syncwarp();
                     signal_oldest();
                 }
-                // the columns' scales and block sums of blocks 4 st .. 4 st + 3 (0 past the
-                // tile's tokens, so that padded columns add nothing)
-                float xd[2][4];
-                float4 xs[2];
-#pragma unroll
-                for (int h2 = 0; h2 < 2; h2++) {
-                    const int tok = h2 ? tok1 : tok0;
-                    xs[h2] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-                    xd[h2][0] = xd[h2][1] = xd[h2][2] = xd[h2][3] = 0.0f;
-                    if (tok >= 0) {
-                        const uint2 dv =
-                            *reinterpret_cast<const uint2 *>(a.xd + (size_t)tok * H32 + 4 * st);
-                        xs[h2] =
-                            *reinterpret_cast<const float4 *>(a.xsum + (size_t)tok * H32 + 4 * st);
-                        xd[h2][0] = half_bits_to_float(dv.x);
-                        xd[h2][1] = half_bits_to_float(dv.x >> 16);
-                        xd[h2][2] = half_bits_to_float(dv.y);
-                        xd[h2][3] = half_bits_to_float(dv.y >> 16);
-                    }
+                // the columns' scales and block sums (loaded one stage ahead)
+                const ColConsts c0 = n0, c1 = n1;
+                if (st + 1 < 2 * nsb) {
+                    n0 = col_consts(a, tok0, st + 1);
+                    n1 = col_consts(a, tok1, st + 1);
                 }
                 if (!(ok = waitw(a, S.abort, S.c_empty + rc.s, rc.ph ^ 1u))) break;
                 float *cc = S.cc + (size_t)rc.s * (kCStage / 4);
-#pragma unroll
-                for (int h2 = 0; h2 < 2; h2++) {
-                    const int n = lane + 32 * h2;
-#pragma unroll
-                    for (int j = 0; j < 4; j++) cc[j * kTN + n] = xd[h2][j];
-                    cc[4 * kTN + 0 * kTN + n] = xs[h2].x;
-                    cc[4 * kTN + 1 * kTN + n] = xs[h2].y;
-                    cc[4 * kTN + 2 * kTN + n] = xs[h2].z;
-                    cc[4 * kTN + 3 * kTN + n] = xs[h2].w;
-                }
+                store_cols(cc, lane, c0);
+                store_cols(cc, lane + 32, c1);
                 __syncwarp();
                 if (lane == 0) mbar_arrive(S.c_full + rc.s);
                 rc.adv(1, a.DC);
-                // the rows' block constants
+                // the rows' block constants, from the packed rows
+                Ring ru = rr;
+                ru.adv(1, a.DR);
+                if (hs == 0) {
+                    if (!(ok = waitw(a, S.abort, S.raw_full + rr.s, rr.ph))) break;
+                    if (!(ok = waitw(a, S.abort, S.raw_full + ru.s, ru.ph))) break;
+                }
                 if (!(ok = waitw(a, S.abort, S.k_empty + rk.s, rk.ph ^ 1u))) break;
+                const uint8_t *gb = S.raw + (size_t)rr.s * a.rawb;
+                const uint8_t *ub = S.raw + (size_t)ru.s * a.rawb;
                 float4 *kc = S.kc + (size_t)rk.s * (kKStage / 16);
                 if (t.fmt == MOE_FMT_Q4_K) consts_stage<MOE_FMT_Q4_K>(gb, ub, sbb, hs, kc, lane);
                 else if (t.fmt == MOE_FMT_Q5_K) consts_stage<MOE_FMT_Q5_K>(gb, ub, sbb, hs, kc, lane);
@@ -494,14 +472,14 @@ __device__ void role_loader(const GemmArgs &a, const Smem &S, int nj) {
                 __syncwarp();
                 if (lane == 0) mbar_arrive(S.k_full + rk.s);
                 rk.adv(1, a.DK);
+                if (hs == 1) {
+                    if (lane == 0) {
+                        mbar_arrive(S.raw_empty + rr.s);
+                        mbar_arrive(S.raw_empty + ru.s);
+                    }
+                    rr.adv(2, a.DR);
+                }
             }
-            if (!ok) break;
-            __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(S.raw_empty + rr.s);
-                mbar_arrive(S.raw_empty + ru.s);
-            }
-            rr.adv(2, a.DR);
         }
         // the tile's last stages: land them now rather than after the next tile's set-up
         cp_async_wait<0>();
@@ -514,25 +492,63 @@ __device__ void role_loader(const GemmArgs &a, const Smem &S, int nj) {
 
 // ---------------------------------------------------------------- warps 4-19: epilogue
 
-// acc (8 pairs of this warp's 16 columns) += I * (s * xd) - wm * xs for one block.
-__device__ __forceinline__ void promote(uint64_t (&acc)[8], const uint32_t (&P)[16], float s,
+// ---------------------------------------------------------------- the promotion (epilogue)
+
+__device__ __forceinline__ uint64_t pk(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ uint64_t pku(uint32_t lo, uint32_t hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
+    return r;
+}
+__device__ __forceinline__ void unpk(uint64_t v, float &lo, float &hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+// acc (this warp's 16 columns) += I * (s * xd) - wm * xs for one block, two columns per
+// instruction.  The s32 value I becomes a float with an integer add and a subtraction: |I| <
+// 2^22, so the bits 0x4B400000 + I are the float 1.5 * 2^23 + I exactly.
+__device__ __forceinline__ void promote(float (&acc)[kEpiCols], const uint32_t (&P)[16], float s,
                                         float nw, const float *xd, const float *xs) {
     const uint64_t s2 = pk(s, s), nw2 = pk(nw, nw);
     const uint64_t negc = pk(-12582912.0f, -12582912.0f);
 #pragma unroll
-    for (int i = 0; i < 8; i++) {
-        const uint64_t xd2 = *reinterpret_cast<const uint64_t *>(xd + 2 * i);
-        const uint64_t xs2 = *reinterpret_cast<const uint64_t *>(xs + 2 * i);
-        const uint64_t f = add2(pku(P[2 * i] + kMagic, P[2 * i + 1] + kMagic), negc);
-        acc[i] = fma2(f, mul2(s2, xd2), acc[i]);
-        acc[i] = fma2(nw2, xs2, acc[i]);
+    for (int i = 0; i < 16; i += 4) {
+        const ulonglong2 xd4 = *reinterpret_cast<const ulonglong2 *>(xd + i);
+        const ulonglong2 xs4 = *reinterpret_cast<const ulonglong2 *>(xs + i);
+        uint64_t a0 = pk(acc[i], acc[i + 1]), a1 = pk(acc[i + 2], acc[i + 3]);
+        const uint64_t f0 = add2(pku(P[i] + kMagic, P[i + 1] + kMagic), negc);
+        const uint64_t f1 = add2(pku(P[i + 2] + kMagic, P[i + 3] + kMagic), negc);
+        a0 = fma2(f0, mul2(s2, xd4.x), a0);
+        a1 = fma2(f1, mul2(s2, xd4.y), a1);
+        a0 = fma2(nw2, xs4.x, a0);
+        a1 = fma2(nw2, xs4.y, a1);
+        unpk(a0, acc[i], acc[i + 1]);
+        unpk(a1, acc[i + 2], acc[i + 3]);
     }
 }
 
 __device__ void role_epilogue(const GemmArgs &a, const Smem &S, int nj, uint32_t tbase) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int q = warp & 3;                  // tensor-memory lane quarter: rows 32q + lane
-    const int ch = (warp - kEpiWarp0) >> 2;  // columns (tokens) 16ch .. 16ch + 15
+    const int ch = (warp - kEpiWarp0) >> 2;  // columns (tokens) 16 ch .. 16 ch + 15
     const int r = 32 * q + lane;
     const uint32_t lane_addr = (uint32_t)(32 * q) << 16;
     Cursor cur;
@@ -541,10 +557,10 @@ __device__ void role_epilogue(const GemmArgs &a, const Smem &S, int nj, uint32_t
     for (int i = blockIdx.x;; i += gridDim.x) {
         Tile t;
         if (!tile_at(a, nj, cur, i, t)) break;
-        const bool active = 16 * ch < t.n_mma;
-        uint64_t ag[8], au[8];
+        const bool active = kEpiCols * ch < t.n_mma;
+        float ag[kEpiCols], au[kEpiCols];
 #pragma unroll
-        for (int j = 0; j < 8; j++) ag[j] = au[j] = 0ull;
+        for (int j = 0; j < kEpiCols; j++) ag[j] = au[j] = 0.0f;
         for (int st = 0; st < nst; st++) {
             if (!waitw(a, S.abort, S.k_full + rk.s, rk.ph)) return;
             if (!waitw(a, S.abort, S.c_full + rc.s, rc.ph)) return;
@@ -554,12 +570,12 @@ __device__ void role_epilogue(const GemmArgs &a, const Smem &S, int nj, uint32_t
             for (int j = 0; j < 4; j++) {
                 if (!waitw(a, S.abort, S.s_full + rs.s, rs.ph)) return;
                 tc_fence_after();
-                // gate columns first, then up: one 16-register set live at a time
+                // gate columns, then up; the slot is released once the second load has landed
                 uint32_t P[16];
                 float4 k4 = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-                const float *xd = cc + j * kTN + 16 * ch;
-                const float *xs = cc + 4 * kTN + j * kTN + 16 * ch;
-                const uint32_t col = tbase + lane_addr + (uint32_t)rs.s * 128 + 16 * ch;
+                const float *xd = cc + j * kTN + kEpiCols * ch;
+                const float *xs = cc + 4 * kTN + j * kTN + kEpiCols * ch;
+                const uint32_t col = tbase + lane_addr + (uint32_t)rs.s * 128 + kEpiCols * ch;
                 if (active) {
                     k4 = kc[j * 128 + r];
                     tmem_ld16(col, P);
@@ -583,17 +599,11 @@ __device__ void role_epilogue(const GemmArgs &a, const Smem &S, int nj, uint32_t
             rc.adv(1, a.DC);
         }
         const int f = 128 * t.mt + r;
-        const int nc = min(16, t.n_valid - 16 * ch);
+        const int nc = min(kEpiCols, t.n_valid - kEpiCols * ch);
         if (128 * t.mt + 32 * q < a.F) {   // the warp's 32 rows are one block of f, in range
 #pragma unroll
-            for (int j = 0; j < 8; j++) {
-                float g0, g1, u0, u1;
-                unpk(ag[j], g0, g1);
-                unpk(au[j], u0, u1);
-                if (2 * j < nc) quantize_h_lane(a, silu_mul(g0, u0), t.slot_base + 16 * ch + 2 * j, f);
-                if (2 * j + 1 < nc)
-                    quantize_h_lane(a, silu_mul(g1, u1), t.slot_base + 16 * ch + 2 * j + 1, f);
-            }
+            for (int j = 0; j < kEpiCols; j++)
+                if (j < nc) quantize_h_lane(a, silu_mul(ag[j], au[j]), t.slot_base + kEpiCols * ch + j, f);
         }
     }
 }
@@ -672,11 +682,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_gateup_i8(const GemmArgs a) {
             mbar_wait_bounded(S.done, 0, 20000000ull);
         }
         __syncwarp();
-    } else if (warp == kUnpackWarp) {
-        role_unpack(a, S, nj);
-        __syncwarp();
     } else if (warp == kLoadWarp) {
         role_loader(a, S, nj);
+        __syncwarp();
+    } else if (warp == kUnpackWarp) {
+        role_unpack(a, S, nj);
         __syncwarp();
     } else {
         role_epilogue(a, S, nj, tbase);
