@@ -417,7 +417,7 @@ static moe_status forward_impl(const moe_arena *arena, const float *d_x, const f
     if (small_route && !tc) {
         err = launch_route_small(d_x, d_logits, T, H, E, k, shared, L, ws, st);
     } else {
-        if (tc)
+        if (tc && !(flags & MOE_F_TC_I8))   // the kind::f16 operand planes as well
             err = launch_quant_rows(d_x, T, H, xq, xd, xs, xsum,
                                     reinterpret_cast<__half *>(ws + L.xh),
                                     reinterpret_cast<__half *>(ws + L.xl),
