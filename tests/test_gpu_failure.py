@@ -65,3 +65,10 @@ def test_tensor_core_wait_times_out_and_next_call_is_clean(torch):
     from expert_ffn_token_b200 import moe
     # the grouped tensor-core kernels: the mbarrier rings give up
     _timeout_then_recover(torch, W["tiny"], 0, moe.F_FORCE_PREFILL)
+
+
+def test_tensor_core_i8_wait_times_out_and_next_call_is_clean(torch):
+    from expert_ffn_token_b200 import moe
+    # gate/up on kind::i8 products: its rings (operands, activations, row and column constants,
+    # accumulator slots) give up the same way
+    _timeout_then_recover(torch, W["tiny"], 0, moe.F_FORCE_PREFILL | moe.F_TC_I8)
