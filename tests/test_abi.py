@@ -137,3 +137,18 @@ def test_binding_signatures_match_the_header(moe):
         if fn.argtypes is None:
             continue
         assert len(fn.argtypes) == arity[name], (name, len(fn.argtypes), arity[name])
+
+
+def test_header_constants_match_the_binding(moe):
+    # every status code, expert format and forward flag the header defines has the same value
+    # in the binding
+    with open(os.path.join(ROOT, "include", "moe.h")) as f:
+        hdr = f.read()
+    consts = {}
+    for name, val in re.findall(r"#define (MOE_F_[A-Z0-9_]+) (\d+)u", hdr):
+        consts[name[len("MOE_"):]] = int(val)
+    for name, val in re.findall(r"\b(MOE_(?:ERR_[A-Z_]+|OK|FMT_[A-Z0-9_]+))\s*=\s*(\d+)", hdr):
+        consts[name[len("MOE_"):]] = int(val)
+    assert {"F_TC_I8", "F_LOOKAHEAD", "ERR_TIMEOUT", "FMT_Q6_K", "OK"} <= set(consts)
+    for name, val in consts.items():
+        assert getattr(moe, name) == val, name
