@@ -16,9 +16,8 @@
 //
 // Cost model.  One MMA per 32 weights per matrix (kind::f16 with exact operands needs four per
 // 16), so the tensor pipe is nowhere near busy; the epilogue's per-block promotion is the work:
-// per element and block an integer add and four fp32 operations, issued as packed f32x2 pairs.
-// The s32 accumulator becomes a float without a conversion instruction: |I| < 2^22, and the bits
-// of 0x4B400000 + I are the float 1.5 * 2^23 + I exactly, from which 1.5 * 2^23 is subtracted.
+// per element and block a conversion and three fp32 operations (the scale product, the product
+// and the min term), the fp32 ones issued as packed f32x2 pairs.
 //
 // Roles (640 threads, 96 registers each):
 //   warp 0       TMA producer: per super-block the packed gate rows and up rows (128 each), L2
@@ -62,7 +61,6 @@ constexpr int kSlots = 4;                            // accumulator slots of 128
 constexpr int kMaxDR = 8, kMaxDA = 2, kMaxDB = 4, kMaxDK = 4, kMaxDC = 6;
 constexpr uint32_t kTmemCols = 512;
 constexpr size_t kSmemCap = 232448;
-constexpr uint32_t kMagic = 0x4B400000u;             // 1.5 * 2^23
 
 struct Smem {
     uint8_t *A, *B, *raw;
@@ -499,18 +497,8 @@ __device__ __forceinline__ uint64_t pk(float lo, float hi) {
     asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
     return r;
 }
-__device__ __forceinline__ uint64_t pku(uint32_t lo, uint32_t hi) {
-    uint64_t r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
-    return r;
-}
 __device__ __forceinline__ void unpk(uint64_t v, float &lo, float &hi) {
     asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-}
-__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
-    uint64_t r;
-    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-    return r;
 }
 __device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
     uint64_t r;
@@ -523,19 +511,17 @@ __device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
     return r;
 }
 // acc (this warp's 16 columns) += I * (s * xd) - wm * xs for one block, two columns per
-// instruction.  The s32 value I becomes a float with an integer add and a subtraction: |I| <
-// 2^22, so the bits 0x4B400000 + I are the float 1.5 * 2^23 + I exactly.
+// instruction.  The s32 value I converts to fp32 exactly (|I| < 2^24).
 __device__ __forceinline__ void promote(float (&acc)[kEpiCols], const uint32_t (&P)[16], float s,
                                         float nw, const float *xd, const float *xs) {
     const uint64_t s2 = pk(s, s), nw2 = pk(nw, nw);
-    const uint64_t negc = pk(-12582912.0f, -12582912.0f);
 #pragma unroll
     for (int i = 0; i < 16; i += 4) {
         const ulonglong2 xd4 = *reinterpret_cast<const ulonglong2 *>(xd + i);
         const ulonglong2 xs4 = *reinterpret_cast<const ulonglong2 *>(xs + i);
         uint64_t a0 = pk(acc[i], acc[i + 1]), a1 = pk(acc[i + 2], acc[i + 3]);
-        const uint64_t f0 = add2(pku(P[i] + kMagic, P[i + 1] + kMagic), negc);
-        const uint64_t f1 = add2(pku(P[i + 2] + kMagic, P[i + 3] + kMagic), negc);
+        const uint64_t f0 = pk(__int2float_rn((int)P[i]), __int2float_rn((int)P[i + 1]));
+        const uint64_t f1 = pk(__int2float_rn((int)P[i + 2]), __int2float_rn((int)P[i + 3]));
         a0 = fma2(f0, mul2(s2, xd4.x), a0);
         a1 = fma2(f1, mul2(s2, xd4.y), a1);
         a0 = fma2(nw2, xs4.x, a0);
