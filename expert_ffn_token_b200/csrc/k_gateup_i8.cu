@@ -512,22 +512,19 @@ __device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
 }
 // acc (this warp's 16 columns) += I * (s * xd) - wm * xs for one block, two columns per
 // instruction.  The s32 value I converts to fp32 exactly (|I| < 2^24).
-__device__ __forceinline__ void promote(float (&acc)[kEpiCols], const uint32_t (&P)[16], float s,
-                                        float nw, const float *xd, const float *xs) {
+__device__ __forceinline__ void promote(uint64_t (&acc)[kEpiCols / 2], const uint32_t (&P)[16],
+                                        float s, float nw, const float *xd, const float *xs) {
     const uint64_t s2 = pk(s, s), nw2 = pk(nw, nw);
 #pragma unroll
-    for (int i = 0; i < 16; i += 4) {
-        const ulonglong2 xd4 = *reinterpret_cast<const ulonglong2 *>(xd + i);
-        const ulonglong2 xs4 = *reinterpret_cast<const ulonglong2 *>(xs + i);
-        uint64_t a0 = pk(acc[i], acc[i + 1]), a1 = pk(acc[i + 2], acc[i + 3]);
-        const uint64_t f0 = pk(__int2float_rn((int)P[i]), __int2float_rn((int)P[i + 1]));
-        const uint64_t f1 = pk(__int2float_rn((int)P[i + 2]), __int2float_rn((int)P[i + 3]));
-        a0 = fma2(f0, mul2(s2, xd4.x), a0);
-        a1 = fma2(f1, mul2(s2, xd4.y), a1);
-        a0 = fma2(nw2, xs4.x, a0);
-        a1 = fma2(nw2, xs4.y, a1);
-        unpk(a0, acc[i], acc[i + 1]);
-        unpk(a1, acc[i + 2], acc[i + 3]);
+    for (int i = 0; i < 8; i += 2) {
+        const ulonglong2 xd4 = *reinterpret_cast<const ulonglong2 *>(xd + 2 * i);
+        const ulonglong2 xs4 = *reinterpret_cast<const ulonglong2 *>(xs + 2 * i);
+        const uint64_t f0 = pk(__int2float_rn((int)P[2 * i]), __int2float_rn((int)P[2 * i + 1]));
+        const uint64_t f1 = pk(__int2float_rn((int)P[2 * i + 2]), __int2float_rn((int)P[2 * i + 3]));
+        acc[i] = fma2(f0, mul2(s2, xd4.x), acc[i]);
+        acc[i + 1] = fma2(f1, mul2(s2, xd4.y), acc[i + 1]);
+        acc[i] = fma2(nw2, xs4.x, acc[i]);
+        acc[i + 1] = fma2(nw2, xs4.y, acc[i + 1]);
     }
 }
 
@@ -544,9 +541,9 @@ __device__ void role_epilogue(const GemmArgs &a, const Smem &S, int nj, uint32_t
         Tile t;
         if (!tile_at(a, nj, cur, i, t)) break;
         const bool active = kEpiCols * ch < t.n_mma;
-        float ag[kEpiCols], au[kEpiCols];
+        uint64_t ag[kEpiCols / 2], au[kEpiCols / 2];   // pairs of columns
 #pragma unroll
-        for (int j = 0; j < kEpiCols; j++) ag[j] = au[j] = 0.0f;
+        for (int j = 0; j < kEpiCols / 2; j++) ag[j] = au[j] = 0ull;
         for (int st = 0; st < nst; st++) {
             if (!waitw(a, S.abort, S.k_full + rk.s, rk.ph)) return;
             if (!waitw(a, S.abort, S.c_full + rc.s, rc.ph)) return;
@@ -588,8 +585,14 @@ __device__ void role_epilogue(const GemmArgs &a, const Smem &S, int nj, uint32_t
         const int nc = min(kEpiCols, t.n_valid - kEpiCols * ch);
         if (128 * t.mt + 32 * q < a.F) {   // the warp's 32 rows are one block of f, in range
 #pragma unroll
-            for (int j = 0; j < kEpiCols; j++)
-                if (j < nc) quantize_h_lane(a, silu_mul(ag[j], au[j]), t.slot_base + kEpiCols * ch + j, f);
+            for (int j = 0; j < kEpiCols / 2; j++) {
+                float g0, g1, u0, u1;
+                unpk(ag[j], g0, g1);
+                unpk(au[j], u0, u1);
+                const int n = t.slot_base + kEpiCols * ch + 2 * j;
+                if (2 * j < nc) quantize_h_lane(a, silu_mul(g0, u0), n, f);
+                if (2 * j + 1 < nc) quantize_h_lane(a, silu_mul(g1, u1), n + 1, f);
+            }
         }
     }
 }
