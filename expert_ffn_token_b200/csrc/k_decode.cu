@@ -946,6 +946,14 @@ __device__ __forceinline__ void down_item(const DecParams &P, const Ctx &C, cons
                              ? q6_chunk(row + (size_t)sb * kQ6KBytes, j)
                              : kq_chunk<false>(row + (size_t)sb * SBB, j);
         const float mf = (j & 1) ? 0.f : 1.f;
+        if (TT == 1) {   // one token: every job has exactly one slot (straight-line, so that the
+                         // caller's unrolled items overlap)
+            const int slot = J.slot0;
+            const ActChunk a = load_act(C.s_hq + (size_t)slot * P.hpad, C.s_hd + slot * hb,
+                                        C.s_hs + slot * hb, p, false);
+            acc[0] += C.s_sw[slot] * kq_chunk_dot(w, a, mf);
+            return;
+        }
 #pragma unroll 1
         for (int t = 0; t < J.n; t++) {
             const int slot = J.slot0 + t;
