@@ -952,19 +952,19 @@ __device__ __forceinline__ void down_item(const DecParams &P, const Ctx &C, cons
             const ActChunk a = load_act(C.s_hq + (size_t)slot * P.hpad, C.s_hd + slot * hb,
                                         C.s_hs + slot * hb, p, false);
             acc[0] += C.s_sw[slot] * kq_chunk_dot(w, a, mf);
-            return;
-        }
+        } else {
 #pragma unroll 1
-        for (int t = 0; t < J.n; t++) {
-            const int slot = J.slot0 + t;
-            const ActChunk a = load_act(C.s_hq + (size_t)slot * P.hpad, C.s_hd + slot * hb,
-                                        C.s_hs + slot * hb, p, false);
-            const float v = kq_chunk_dot(w, a, mf);
-            const int tok = C.s_stok[slot];
-            const float wv = C.s_sw[slot] * v;
+            for (int t = 0; t < J.n; t++) {
+                const int slot = J.slot0 + t;
+                const ActChunk a = load_act(C.s_hq + (size_t)slot * P.hpad, C.s_hd + slot * hb,
+                                            C.s_hs + slot * hb, p, false);
+                const float v = kq_chunk_dot(w, a, mf);
+                const int tok = C.s_stok[slot];
+                const float wv = C.s_sw[slot] * v;
 #pragma unroll
-            for (int tt = 0; tt < TT; tt++)
-                if (tt == tok) acc[tt] += wv;
+                for (int tt = 0; tt < TT; tt++)
+                    if (tt == tok) acc[tt] += wv;
+            }
         }
     }
 }
