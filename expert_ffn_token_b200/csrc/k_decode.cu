@@ -403,15 +403,13 @@ __device__ __noinline__ void warp_topk_reg(const float *row, int E, int k, int *
 __device__ __noinline__ int q8_1_lane(float v, bool &fin, uint16_t &d16, uint16_t &s16,
                                       float &dsum) {
     fin = __all_sync(kFullMask, isfinite(v));
-    float a = fabsf(v);
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) a = fmaxf(a, __shfl_xor_sync(kFullMask, a, o));
+    // the largest |v| as the largest bit pattern (non-negative floats order as unsigned
+    // integers; a non-finite block is zeroed below whatever this gives)
+    const float a = __uint_as_float(__reduce_max_sync(kFullMask, __float_as_uint(fabsf(v))));
     const float d = __fdiv_rn(a, 127.0f);
     int qi = 0;
     if (fin && d != 0.0f) qi = max(-127, min(127, (int)roundf(__fdiv_rn(v, d))));
-    int sum = qi;
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) sum += __shfl_xor_sync(kFullMask, sum, o);
+    const int sum = __reduce_add_sync(kFullMask, qi);
     if (fin) {
         const __half dh = __float2half_rn(d);
         d16 = __half_as_ushort(dh);
