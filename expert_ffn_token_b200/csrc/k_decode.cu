@@ -658,18 +658,37 @@ __device__ __forceinline__ void prologue(const DecParams &P, Ctx &C, uint8_t *sm
     }
     __syncthreads();
     const int U = C.s_misc[0];
+    // the slot of assignment a: its expert's offset + the number of earlier assignments of the
+    // same expert (token-stable).  Up to 32 assignments one warp finds that rank at once (the
+    // lanes holding the same expert, below this lane); more take the plain count.
+    if (A <= 32) {
+        if (warp == 0) {
+            const int e = lane < A ? s_ids[lane] : -1 - lane;   // idle lanes match no one
+            const unsigned same = __match_any_sync(kFullMask, e);
+            if (lane < A) {
+                const int slot = s_off[e] + __popc(same & ((1u << lane) - 1u));
+                C.s_stok[slot] = lane / k;
+                C.s_sw[slot] = s_wt[lane];
+                if (cta0) {
+                    reinterpret_cast<int32_t *>(ws + L.perm)[slot] = lane;
+                    reinterpret_cast<int32_t *>(ws + L.inv_perm)[lane] = slot;
+                }
+            }
+        }
+    } else {
 #pragma unroll 1
-    for (int a = tid; a < A; a += kThreads) {
-        const int e = s_ids[a];
-        int rank = 0;
+        for (int a = tid; a < A; a += kThreads) {
+            const int e = s_ids[a];
+            int rank = 0;
 #pragma unroll 1
-        for (int b = 0; b < a; b++) rank += s_ids[b] == e;
-        const int slot = s_off[e] + rank;
-        C.s_stok[slot] = a / k;
-        C.s_sw[slot] = s_wt[a];
-        if (cta0) {
-            reinterpret_cast<int32_t *>(ws + L.perm)[slot] = a;
-            reinterpret_cast<int32_t *>(ws + L.inv_perm)[a] = slot;
+            for (int b = 0; b < a; b++) rank += s_ids[b] == e;
+            const int slot = s_off[e] + rank;
+            C.s_stok[slot] = a / k;
+            C.s_sw[slot] = s_wt[a];
+            if (cta0) {
+                reinterpret_cast<int32_t *>(ws + L.perm)[slot] = a;
+                reinterpret_cast<int32_t *>(ws + L.inv_perm)[a] = slot;
+            }
         }
     }
 #pragma unroll 1
@@ -679,16 +698,29 @@ __device__ __forceinline__ void prologue(const DecParams &P, Ctx &C, uint8_t *sm
     }
     // the jobs by token count, descending (stable): the gate/up blocks are dealt to the CTAs in
     // this order, so that the heavy blocks spread over the grid (multi-token kernels)
-#pragma unroll 1
-    for (int u = tid; u < U && TT > 1; u += kThreads) {
-        const int n = s_jobs[u].n;
-        int pos = 0;
-#pragma unroll 1
-        for (int v = 0; v < U; v++) {
-            const int m = s_jobs[v].n;
-            pos += (m > n || (m == n && v < u)) ? 1 : 0;
+    if (TT > 1 && U <= 32) {   // one warp: every job's count against all the others at once
+        if (warp == 1) {
+            const int n = lane < U ? s_jobs[lane].n : -1;
+            int pos = 0;
+#pragma unroll
+            for (int v = 0; v < 32; v++) {
+                const int m = __shfl_sync(kFullMask, n, v);
+                pos += (v < U && (m > n || (m == n && v < lane))) ? 1 : 0;
+            }
+            if (lane < U) s_jobs[pos].by_n = (short)lane;
         }
-        s_jobs[pos].by_n = (short)u;
+    } else {
+#pragma unroll 1
+        for (int u = tid; u < U && TT > 1; u += kThreads) {
+            const int n = s_jobs[u].n;
+            int pos = 0;
+#pragma unroll 1
+            for (int v = 0; v < U; v++) {
+                const int m = s_jobs[v].n;
+                pos += (m > n || (m == n && v < u)) ? 1 : 0;
+            }
+            s_jobs[pos].by_n = (short)u;
+        }
     }
     bool desc_ok = true;
     if (tid < U && !ptx::mbar_wait_bounded(C.desc_bar, 0, desc_wait_ns(P))) {
