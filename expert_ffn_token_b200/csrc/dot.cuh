@@ -29,6 +29,12 @@ __device__ __forceinline__ uint2 ld_stream8(const uint8_t *p) {
     return v;
 }
 
+__device__ __forceinline__ uint32_t ld_stream_u32(const uint8_t *p) {
+    uint32_t v;
+    asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
+    return v;
+}
+
 __device__ __forceinline__ uint32_t ld_stream_u16(const uint8_t *p) {
     unsigned short v;
     asm volatile("ld.global.nc.L1::no_allocate.u16 %0, [%1];" : "=h"(v) : "l"(p));
@@ -182,13 +188,25 @@ struct Q80Block {
     float d;
 };
 
+// Rows start 16-byte aligned, so block b starts on a word boundary when b is even and 2 bytes
+// past one when b is odd: word loads cover it either way, none past the block's last byte.
 __device__ __forceinline__ Q80Block q80_load(const uint8_t *row, int b) {
     const uint8_t *p = row + (size_t)b * kQ80Bytes;
     Q80Block r;
-    r.d = half_bits_to_float(ld_stream_u16(p));
+    if (b & 1) {   // p - 2 is aligned: d in the upper half of word 0, the quants in words 1..8
+        const uint32_t w0 = ld_stream_u32(p - 2);
+        r.d = half_bits_to_float(w0 >> 16);
 #pragma unroll
-    for (int i = 0; i < 8; i++)
-        r.w[i] = ld_stream_u16(p + 2 + 4 * i) | (ld_stream_u16(p + 4 + 4 * i) << 16);
+        for (int i = 0; i < 8; i++) r.w[i] = ld_stream_u32(p + 2 + 4 * i);
+    } else {       // p is aligned: d and the first 30 quants in 8 words, the last 2 quants alone
+        uint32_t v[9];
+#pragma unroll
+        for (int i = 0; i < 8; i++) v[i] = ld_stream_u32(p + 4 * i);
+        v[8] = ld_stream_u16(p + 32);
+        r.d = half_bits_to_float(v[0]);
+#pragma unroll
+        for (int i = 0; i < 8; i++) r.w[i] = __funnelshift_r(v[i], v[i + 1], 16);
+    }
     return r;
 }
 
